@@ -27,7 +27,7 @@
  *
  * The pages give no formula for the quantizer. The fp32 recipe used here is
  * the plainest asymmetric min/max reading, fixed so that codes are unique:
- *   z = fp16 rounded toward -inf of min(x)
+ *   z = fp16 rounded toward -inf of min(x)   (a zero minimum taken as +0)
  *   s = fp16 rounded toward +inf of fp32(fp32(max(x) - z) / L),  L = 2^bits - 1
  *   s == 0 -> every code is 0
  *   else r = fp32(1 / s), q = clamp(rint_even(fp32(fp32(x - z) * r)), 0, L)
@@ -270,6 +270,11 @@ void oracle_quantize_group(const float *x, int n, int stride, int bits,
         if (v > mx)
             mx = v;
     }
+    /* A zero extreme is taken as +0 (adding +0 turns -0 into +0), so the
+     * zero-point's bit pattern does not depend on which signed zero comes
+     * first in the group. */
+    mn = mn + 0.0f;
+    mx = mx + 0.0f;
     uint16_t zb = oracle_f32_to_f16(mn, ORACLE_RD);
     float z = oracle_f16_to_f32(zb);
     float range = mx - z;

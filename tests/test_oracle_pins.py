@@ -395,3 +395,18 @@ def test_dequant_x_is_bf16_near_exact_value():
     # bf16 values (low 16 bits zero) within half a bf16 ulp (2^-8 relative) of q*s+z
     assert np.all((xh.view(np.uint32) & 0xFFFF) == 0)
     assert np.all(np.abs(xh - exact) <= np.abs(exact) * 2.0 ** -8 * (1 + 2.0 ** -15) + 1e-30)
+
+
+def test_quantizer_permutation_invariance_with_signed_zeros():
+    # Scale and zero depend on the group's values only, not on their order;
+    # with both signed zeros present at the minimum this needs the zero
+    # extreme taken as +0.
+    g = np.random.default_rng(16)
+    for trial in range(50):
+        x = np.abs(g.standard_normal(32)).astype(np.float32)
+        x[g.choice(32, 6, replace=False)] = np.where(g.random(6) < 0.5, -0.0, 0.0).astype(np.float32)
+        perm = g.permutation(32)
+        s1, z1, q1 = oracle.quantize_group(x, 4)
+        s2, z2, q2 = oracle.quantize_group(x[perm], 4)
+        assert (s1, z1) == (s2, z2)
+        assert np.array_equal(q1[perm], q2)
