@@ -1,0 +1,431 @@
+"""Benchmark of the low-bit KV-cache hot path on B200.
+
+Workload (the metric's configuration): a Llama-3.1-8B-shaped attention layer,
+16 sequences x 32 query / 8 KV heads x head_dim 128, bf16 inputs, keys with 4
+outlier channels (x20), keys and queries Hadamard-rotated, K and V INT4 in
+groups of 128 (fp16 scale/zero), contiguous cache, context 8192. A step is
+one decode step: quantize-append one new token per sequence, then split-K
+decode attention over the whole packed cache (split pass + merge pass).
+Steps run as episodes of 64 decode steps (context 8193..8256); after each
+episode the sequence lengths are rewound to 8192 outside the timed region.
+
+value  = algorithmic packed-KV bytes attended per step (codes + fp16
+         scale/zero of every cached token, K and V) / device step time
+e2e    = the same bytes / wall time of a step driven from pinned host buffers
+         (new K/V and q uploaded, output read back) through the C-ABI calls
+roofline (dominant kernel = the split-K attention pass): packed bytes / its
+         CUDA-event duration against the measured HBM copy bandwidth
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs its own replica (weak scaling); no collective
+touches the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn packed-KV GB/s (% of 8 TB/s HBM); quantize-append tokens/s"
+WORKLOAD = ("llama8b_layer: 16 seqs x 32 q / 8 kv heads x d128, bf16 in, context 8192 + 64 decode "
+            "steps of 1 token, INT4 g128 K and V with fp16 scale/zero, Hadamard(128) on K and Q, "
+            "contiguous cache")
+BATCH, HQ, HKV, D, CTX, EPISODE = 16, 32, 8, 128, 8192, 64
+BYTES_PER_TOKEN_HEAD = 2 * (D * 4 // 8 + (D // 128) * 4)   # K + V: 64 B codes + 4 B scale/zero
+NOMINAL_HBM_GBS = 8000.0
+FLUSH_BYTES = 256 << 20
+DECODE_SRC = os.path.join(ROOT, "bit_kv_cache_21_b200", "csrc", "kvq_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_splitk_llama8b_traffic.json")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """dram bytes per split-K launch from the committed ncu summary, or None
+    when the kernel source changed since it was captured."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        if d.get("source_sha256_16") != source_hash(DECODE_SRC):
+            return None
+        return float(d["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML)
+# ---------------------------------------------------------------------------
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, torch_device):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            props = torch.cuda.get_device_properties(torch_device)
+            h = None
+            uuid = str(getattr(props, "uuid", ""))
+            if uuid:
+                for cand in (uuid if uuid.startswith("GPU-") else "GPU-" + uuid, uuid):
+                    try:
+                        h = pynvml.nvmlDeviceGetHandleByUUID(cand)
+                        break
+                    except Exception:
+                        pass
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.h, self.nv = h, pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        names = [n for b, n in _REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# inputs
+# ---------------------------------------------------------------------------
+def make_inputs(seed_offset, n_decode):
+    """History for the prefill plus the tokens and queries of n_decode steps."""
+    import workloads as W
+    w = W.LLAMA8B_LAYER
+    ks, vs, _ = W.kv_history(w, [CTX + n_decode] * BATCH, seed_offset=seed_offset)
+    k = np.stack(ks)  # [B][T][H][D]
+    v = np.stack(vs)
+    qs = np.stack([W.queries(w, BATCH, seed_offset=seed_offset * 1000 + i) for i in range(n_decode)])
+    return k, v, qs
+
+
+def bf16(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import bit_kv_cache_21_b200 as K
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    k, v, qs = make_inputs(rank, EPISODE)
+
+    cap = CTX + EPISODE + 64
+    spec = K.CacheSpec(BATCH, HKV, bits_k=4, bits_v=4, group_k=128, group_v=128,
+                       hadamard_block_k=128, capacity_tokens=cap)
+    cache = K.KVCache(spec, device=dev)
+    lens = torch.zeros(BATCH, dtype=torch.int32, device=dev)
+    cu_pre = torch.arange(0, (BATCH + 1) * CTX, CTX, dtype=torch.int32, device=dev)
+    k_pre = bf16(k[:, :CTX].reshape(-1, HKV, D)).to(dev)
+    v_pre = bf16(v[:, :CTX].reshape(-1, HKV, D)).to(dev)
+
+    # quantize-append throughput on the bulk prefill (16 x 8192 tokens)
+    pre_ms = []
+    for _ in range(3):
+        lens.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        K.quantize_append(cache.desc, k_pre, v_pre, cu_pre, lens)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pre_ms.append(e0.elapsed_time(e1))
+    del k_pre, v_pre
+    append_ms = min(pre_ms)
+    n_tok = BATCH * CTX
+    append_bytes = n_tok * HKV * 2 * (D * 2 + D // 2 + 4)   # bf16 in + packed out, K and V
+    append_info = {"metric": "quantize-append tokens/s", "value": n_tok / (append_ms * 1e-3),
+                   "unit": "tokens/s", "GBps": append_bytes / (append_ms * 1e-3) / 1e9,
+                   "workload": "bulk prefill 16 x 8192 tokens x 8 KV heads, K and V, INT4 g128, "
+                               "Hadamard K", "ms": append_ms}
+
+    # per-step device inputs for the episode
+    k_steps = [bf16(k[:, CTX + i]).to(dev) for i in range(EPISODE)]       # [B][H][D]
+    v_steps = [bf16(v[:, CTX + i]).to(dev) for i in range(EPISODE)]
+    q_steps = [bf16(qs[i]).to(dev) for i in range(EPISODE)]
+    cu_one = torch.arange(0, BATCH + 1, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    ws = torch.empty(K.decode_workspace_size(cache.desc, BATCH, HQ, cap), dtype=torch.uint8, device=dev)
+    out = torch.empty((BATCH, HQ, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ctx_lens = torch.full((BATCH,), CTX, dtype=torch.int32, device=dev)
+
+    def step(i, evs=None):
+        j = i % EPISODE
+        if j == 0:
+            lens.copy_(ctx_lens)
+        if evs:
+            evs[0].record(stream)
+        K.quantize_append(cache.desc, k_steps[j], v_steps[j], cu_one, lens)
+        if evs:
+            evs[1].record(stream)
+        K.decode_splitk(cache.desc, q_steps[j], lens, cap, scale, ws)
+        if evs:
+            evs[2].record(stream)
+        K.decode_merge(cache.desc, HQ, lens, cap, out, ws)
+        if evs:
+            evs[3].record(stream)
+        return CTX + j + 1   # tokens attended per sequence
+
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    # start the timed episodes at a step boundary of the episode
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    tokens = []
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            tokens.append(step(i, evs[i]))
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    split_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    append1_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = sum(step_ms)
+    bytes_total = sum(t * BATCH * HKV * BYTES_PER_TOKEN_HEAD for t in tokens)
+    assert cache.device_status() == 0, "device status %d" % cache.device_status()
+
+    # end to end from pinned host buffers
+    import torch.cuda
+    hk = [bf16(k[:, CTX + i]).pin_memory() for i in range(EPISODE)]
+    hv = [bf16(v[:, CTX + i]).pin_memory() for i in range(EPISODE)]
+    hq = [bf16(qs[i]).pin_memory() for i in range(EPISODE)]
+    hout = torch.empty((BATCH, HQ, D), dtype=torch.float32).pin_memory()
+    dk = torch.empty_like(k_steps[0])
+    dv = torch.empty_like(v_steps[0])
+    dq = torch.empty_like(q_steps[0])
+    e2e_s, e2e_bytes = [], 0
+    for i in range(args.warmup + args.steps):
+        j = i % EPISODE
+        if j == 0:
+            lens.copy_(ctx_lens)
+        flush.zero_()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        dk.copy_(hk[j], non_blocking=True)
+        dv.copy_(hv[j], non_blocking=True)
+        dq.copy_(hq[j], non_blocking=True)
+        K.quantize_append(cache.desc, dk, dv, cu_one, lens)
+        K.decode_attention(cache.desc, dq, lens, cap, scale, out=out, workspace=ws)
+        hout.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        if i >= args.warmup:
+            e2e_s.append(t1 - t0)
+            e2e_bytes += (CTX + j + 1) * BATCH * HKV * BYTES_PER_TOKEN_HEAD
+    h2d = dk.numel() * 2 + dv.numel() * 2 + dq.numel() * 2
+    d2h = hout.numel() * 4
+
+    res = {"total_ms": total_ms, "bytes": bytes_total, "split_ms": split_ms, "merge_ms": merge_ms,
+           "append1_ms": append1_ms, "step_ms": step_ms, "clocks": clocks.summary(),
+           "append": append_info, "e2e_s": sum(e2e_s), "e2e_bytes": e2e_bytes,
+           "h2d": h2d, "d2h": d2h, "tokens": tokens}
+    return res
+
+
+def cpu_units(n_units, seed=0):
+    """Oracle-side cache state of n_units (sequence, KV head) units of the
+    workload at context 8193: the oracle's own packed K/V and 4 queries."""
+    import oracle
+    import workloads as W
+    T = CTX + 1
+    g = W.rng(seed + 77)
+    ch = W.outlier_channels(g)
+    units = []
+    for _ in range(n_units):
+        kh = W.finish(W.keys(g, (T, D), ch), "bf16")
+        vh = W.finish(W.normal(g, (T, D)), "bf16")
+        q = W.finish(W.normal(g, (4, D)), "bf16")
+        units.append((oracle.quantize_tokens(kh, 128, 128, 4), oracle.quantize_tokens(vh, 0, 128, 4), q))
+    return units
+
+
+def cpu_time(units, budget_s):
+    """The oracle (float64, one thread) on whole units, cycling through them
+    until budget_s of work: dequantize the unit's packed K and V, rotate the
+    queries and attend. Returns (GB/s of packed bytes, units done, seconds)."""
+    import oracle
+    done, t_used, nbytes = 0, 0.0, 0
+    while done == 0 or t_used < budget_s:
+        (kc, ksz), (vc, vsz), q = units[done % len(units)]
+        t0 = time.perf_counter()
+        kd = oracle.dequant_tokens(kc, ksz, 128, 4)
+        vd = oracle.dequant_tokens(vc, vsz, 128, 4)
+        oracle.decode_attention_gqa(q, kd[None], vd[None], 1.0 / math.sqrt(D), rotate_q_block=128)
+        t_used += time.perf_counter() - t0
+        done += 1
+        nbytes += kc.shape[0] * BYTES_PER_TOKEN_HEAD
+    return nbytes / t_used / 1e9, done, t_used
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=640)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # The reference arm is the CPU oracle as it stands (the pages ship no
+        # code); rank 0 alone runs it.
+        if rank != 0:
+            return
+        units = cpu_units(8)
+        for _ in range(args.warmup):
+            cpu_time(units, 0.0)
+        vals, n_units, secs = [], 0, 0.0
+        for _ in range(args.steps):
+            gbs, u, t = cpu_time(units, 0.0)     # one unit per step
+            vals.append(gbs)
+            n_units += u
+            secs += t
+        value = statistics.median(vals)
+        cores = 1
+        sample = ("one (sequence, KV head) unit of the decode step at context 8193 per step, "
+                  "%d steps (%.1f s of oracle work): float64 dequantize + attention, one thread"
+                  % (n_units, secs))
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": WORKLOAD},
+                "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, rank, world, local_rank)
+
+    # max over ranks of the device time; bytes summed over ranks
+    total_ms, total_bytes, e2e_s, e2e_bytes = res["total_ms"], res["bytes"], res["e2e_s"], res["e2e_bytes"]
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_s], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        b = torch.tensor([float(total_bytes), float(e2e_bytes)], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(b, op=torch.distributed.ReduceOp.SUM)
+        total_ms, e2e_s = float(t[0]), float(t[1])
+        total_bytes, e2e_bytes = float(b[0]), float(b[1])
+    if rank == 0:
+        hbm_peak, peak_kind = peaks()
+        value = total_bytes / (total_ms * 1e-3) / 1e9
+        split_mean_ms = statistics.mean(res["split_ms"])
+        bytes_per_launch = res["bytes"] / args.steps
+        achieved = bytes_per_launch / (split_mean_ms * 1e-3) / 1e9
+        traffic = traffic_per_launch()
+        cpu_gbs, cpu_done, cpu_s = cpu_time(cpu_units(16), args.cpu_budget)
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int4 packed K/V, fp32 math", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": BATCH * world, "seq_len": CTX,
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "flushed between steps (256 MiB write)",
+                       "pct_of_8TBs": 100.0 * value / NOMINAL_HBM_GBS},
+            "roofline": {"kernel": "decode_splitk_kernel", "bound": "hbm", "achieved": achieved,
+                         "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": traffic,
+                         "bytes_per_launch": bytes_per_launch, "ms_per_launch": split_mean_ms},
+            "breakdown_ms": {"append": statistics.mean(res["append1_ms"]), "splitk": split_mean_ms,
+                             "merge": statistics.mean(res["merge_ms"])},
+            "append": res["append"],
+            "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": "%d (sequence, KV head) units of the decode step at "
+                                       "context 8193, cycling over 16 (%.1f s): float64 dequantize "
+                                       "+ attention, one thread" % (cpu_done, cpu_s)},
+            "e2e": {"value": e2e_bytes / e2e_s / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+            "gpu_launches": 4 * args.steps,
+            "clocks": res["clocks"],
+        }
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

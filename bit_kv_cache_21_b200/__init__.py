@@ -1,0 +1,17 @@
+"""B200 (sm_100a) low-bit KV cache: INT4/INT2 quantize-append with Hadamard
+rotation, split-K decode attention over the packed cache, and XQuant-style
+K/V rematerialization on the tensor cores.
+
+The compute lives in libkvq.so (C ABI, include/kvq.h); this package is its
+ctypes binding plus helpers that allocate the cache buffers with torch.
+"""
+from ._binding import (  # noqa: F401
+    BF16, FP16, FP32, PER_TOKEN, PER_CHANNEL,
+    DEV_CAPACITY, DEV_TIMEOUT, DEV_SEQLEN,
+    DEBUG_WAIT_TIMEOUT_NS, DEBUG_SKIP_TILE,
+    OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_TIMEOUT, ERR_CUDA,
+    CacheDesc, KvqError, lib, header_symbols, status_string, check,
+    quantize_append, decode_workspace_size, decode_attention, decode_splitk, decode_merge,
+    remat_kv, rope_tables, debug_set, version,
+)
+from .cache import CacheSpec, KVCache  # noqa: F401

@@ -1,0 +1,143 @@
+// kvq_common.cuh -- device helpers shared by the sm_100a kernels: bounded
+// mbarrier waits, 1-D bulk copies (TMA engine), status reporting, number
+// conversions. Internal header, not part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------------------
+// Host-side launch settings shared by the translation units.
+// ---------------------------------------------------------------------------
+struct DebugHooks {
+    int64_t wait_timeout_ns;
+    int32_t skip_tile;
+};
+DebugHooks &debug_hooks();
+
+// ---------------------------------------------------------------------------
+// Status word
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void status_or(int32_t *st, int32_t bits) {
+    if (st != nullptr) atomicOr(st, bits);
+}
+
+// ---------------------------------------------------------------------------
+// Timers and mbarriers (PTX). Every wait is bounded by a %globaltimer limit.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make mbarrier initialisation visible to the async proxy (bulk copies).
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
+        "r"(bytes)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait until the phase of `bar` with the given parity has completed, or until
+// `timeout_ns` passes (then OR KVQ_DEV_TIMEOUT into *status and raise the
+// CTA's abort flag), or until another thread raised the abort flag.
+// Returns true when the phase completed.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  int64_t timeout_ns, int32_t *status,
+                                                  volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (static_cast<int64_t>(global_timer_ns() - t0) > timeout_ns) {
+            status_or(status, KVQ_DEV_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// 1-D bulk copy global -> shared through the TMA engine, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16. No multicast.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Named barrier among `nthreads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Number conversions
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) {
+    return __uint_as_float(b16 << 16);
+}
+
+// Small unsigned integer (< 2^23) to float exactly: place it in the
+// mantissa of 2^23 and subtract 2^23.
+__device__ __forceinline__ float small_uint_to_float(uint32_t c) {
+    return __fsub_rn(__uint_as_float(0x4B000000u | c), 8388608.0f);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+}  // namespace kvq

@@ -1,0 +1,48 @@
+// kvq_internal.h -- host-side launchers shared between the translation units
+// of libkvq.so. Internal; the public interface is include/kvq.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// Rotation scale fp32(1/sqrt(block)) for a power-of-two block, 0 for none.
+float hadamard_scale(int block);
+
+// Quantized-residual split: tokens [0, R*floor((T-1)/R)) are quantized.
+__host__ __device__ inline int quantized_len(int T, int R) { return (R <= 0) ? T : (T <= 0 ? 0 : R * ((T - 1) / R)); }
+
+kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void *v_new,
+                         kvq_dtype dtype, const int32_t *cu_new, int32_t *seq_lens,
+                         int num_seqs, int total_new, cudaStream_t stream);
+
+// Decode attention geometry chosen on the host from the sizes alone.
+struct DecodePlan {
+    int chunk;      // tokens per split (multiple of the tile)
+    int n_split;    // splits per (sequence, KV head)
+    size_t ws_part; // bytes of partial outputs
+    size_t ws_ml;   // bytes of (m, l) pairs
+    size_t ws_total;
+};
+bool plan_decode(const kvq_cache_desc &d, int num_seqs, int num_q_heads, int max_seq_len,
+                 DecodePlan *plan);
+
+kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan, const void *q,
+                                kvq_dtype q_dtype, int num_q_heads, const int32_t *seq_lens,
+                                int num_seqs, int max_seq_len, float softmax_scale,
+                                void *workspace, cudaStream_t stream);
+kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, int num_q_heads,
+                               const int32_t *seq_lens, int num_seqs, int max_seq_len,
+                               float *out, const void *workspace, cudaStream_t stream);
+
+kvq_status launch_remat(const kvq_cache_desc &x, const void *w_kv, int n_kv_heads,
+                        const float *rope_cos, const float *rope_sin, int batch, int ctx_len,
+                        void *k_out, void *v_out, cudaStream_t stream);
+kvq_status launch_rope_tables(float *c, float *s, int n_pos, int head_dim, double theta,
+                              cudaStream_t stream);
+
+}  // namespace kvq
