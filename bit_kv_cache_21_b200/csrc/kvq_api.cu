@@ -107,9 +107,9 @@ kvq_status kvq_quantize_append(const kvq_cache_desc *desc, const void *k_new, co
     if (!dtype_ok(dtype) || cu_new == nullptr || seq_lens == nullptr) return KVQ_ERR_INVALID_ARG;
     if (num_seqs <= 0 || total_new_tokens < 0) return KVQ_ERR_INVALID_ARG;
     if (!desc->paged && num_seqs > desc->num_seqs) return KVQ_ERR_INVALID_ARG;
+    if (total_new_tokens == 0) return KVQ_OK;  // nothing to write, lengths unchanged
     if ((v_new != nullptr) != need_v) return KVQ_ERR_INVALID_ARG;
-    if (total_new_tokens > 0 && (k_new == nullptr || !aligned16(k_new) ||
-                                 (need_v && !aligned16(v_new))))
+    if (k_new == nullptr || !aligned16(k_new) || (need_v && !aligned16(v_new)))
         return KVQ_ERR_INVALID_ARG;
     if (desc->residual_len > 0 && dtype != KVQ_BF16) return KVQ_ERR_UNSUPPORTED;
     return launch_append(*desc, k_new, v_new, dtype, cu_new, seq_lens, num_seqs, total_new_tokens,

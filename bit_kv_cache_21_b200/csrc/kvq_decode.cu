@@ -10,16 +10,25 @@
 // the keys' orthogonal transform, so q~ . k~ = q . k.
 //
 // CTA = one (split, KV head, sequence): 4 consumer warps and 1 producer warp.
-// The producer's elected lane stages each 64-token tile (K codes, K scale/zero,
-// V codes, V scale/zero) into a shared-memory ring with 1-D bulk copies (TMA
-// engine, mbarrier complete_tx); page-table indirection is resolved per page.
-// Each consumer warp owns 16 of a tile's 64 tokens with its own online-softmax
-// state, so tiles need no cross-warp synchronisation:
-//   scores: 8 lanes per token, 16 channels per lane, all GQA heads at once;
-//           a reduce-scatter over the 8 lanes leaves one head's score per lane
-//           pair;
-//   values: 16 lanes cover the 128 channels (8 each) for all GQA heads, the
-//           two half-warps take alternate tokens.
+// The producer's elected lane stages each tile (K codes, K scale/zero, V
+// codes, V scale/zero; or bf16 rows of the recent-token window) into a
+// shared-memory ring with 1-D bulk copies (TMA engine, mbarrier complete_tx),
+// resolving page-table indirection per page.
+//
+// Inner loop. The path is bound by the FP32 FMA pipe, not by the tensor
+// cores: every cached element meets GQA query heads, one multiply-add each.
+// So the loop is built to spend as few issue slots as possible besides those
+// multiply-adds:
+//   * multiply-adds are packed f32x2 FMAs (two lanes of work per issue);
+//   * a 4-bit or 2-bit code c becomes the float 0.5 + c/256 with ONE byte
+//     permute (the code lands in mantissa bits 16..19 of 0.5); the constant
+//     0.5 is folded into the per-group zero-point terms, exactly;
+//   * each consumer warp owns a quarter of every tile with its own
+//     online-softmax state, so tiles need no cross-warp synchronisation;
+//   * scores: 8 lanes per token, 16 channels per lane, all GQA heads at once,
+//     a reduce-scatter over the 8 lanes leaves one head's score per lane pair;
+//   * values: 16 lanes cover the 128 channels (8 each) for all GQA heads; the
+//     two half-warps take alternate tokens.
 // The four warps' states are merged once per split; the merge kernel combines
 // the splits.
 #include <algorithm>
@@ -31,7 +40,8 @@ namespace kvq {
 
 namespace {
 
-constexpr int kTile = 64;
+constexpr int kTile = 64;          // tokens per quantized tile
+constexpr int kWinTile = 16;       // tokens per bf16 window tile (quantized caches)
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
@@ -61,6 +71,7 @@ struct DecodeParams {
     int q_dtype;
     // shared-memory stage layout (bytes)
     int stage_bytes, off_ksz, off_vc, off_vsz;
+    int bf_tile, bf_off_v;  // bf16 tiles: tokens per tile, offset of the V rows
     int64_t timeout_ns;
     int skip_tile;
 };
@@ -74,111 +85,164 @@ struct VRow {
     static constexpr int bytes = (VM == V_BF16) ? kHeadDim * 2 : kHeadDim * VBITS / 8;
 };
 
-__device__ __forceinline__ float load_q_elem(const void *q, int64_t idx, int dt) {
-    if (dt == KVQ_FP32) return static_cast<const float *>(q)[idx];
-    const uint16_t b = static_cast<const uint16_t *>(q)[idx];
-    if (dt == KVQ_BF16) return bf16_bits_to_float(b);
-    return __half2float(__ushort_as_half(b));
+// ---- packed f32x2 arithmetic (sm_100) --------------------------------------
+__device__ __forceinline__ unsigned long long as_u64(float2 v) {
+    return *reinterpret_cast<unsigned long long *>(&v);
+}
+__device__ __forceinline__ float2 as_f2(unsigned long long v) {
+    return *reinterpret_cast<float2 *>(&v);
+}
+// d = a * b + d, two lanes
+__device__ __forceinline__ void ffma2(float2 &d, float2 a, float2 b) {
+    unsigned long long r = as_u64(d);
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(r) : "l"(as_u64(a)), "l"(as_u64(b)));
+    d = as_f2(r);
 }
 
-// Codes of 16 channels -> floats (exact small integers).
-template <int BITS>
-__device__ __forceinline__ void k_codes16(const uint8_t *row, int part, float c[16]) {
-    if constexpr (BITS == 4) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(row + part * 8);
+// ---- shared-memory loads ----------------------------------------------------
+__device__ __forceinline__ uint32_t lds32(const void *p) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16(const void *p) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_addr(p)));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(const void *p) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr(p)));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(const void *p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_addr(p)));
+    return v;
+}
+__device__ __forceinline__ float2 half2_lds(const void *p) {
+    const uint32_t u = lds32(p);
+    return __half22float2(*reinterpret_cast<const __half2 *>(&u));
+}
+
+// ---- code -> float ----------------------------------------------------------
+// Byte k of `b` holds a code in its low bits; the result is the float
+// 0.5 + code/256 (the byte becomes mantissa bits 16..23 of 0.5). One PRMT.
+__device__ __forceinline__ float code_f(uint32_t b, int k) {
+    return __uint_as_float(__byte_perm(b, 0x3F000000u, 0x7054u | (static_cast<uint32_t>(k) << 8)));
+}
+
+// 16 key channels [16*part, 16*part + 16) as 8 (even, odd) pairs.
+template <int KM, int KBITS>
+__device__ __forceinline__ void key_pairs(const uint8_t *row, int part, float2 f[8]) {
+    if constexpr (KM == K_BF16) {
+        const uint4 a = lds128(row + part * 32), b = lds128(row + part * 32 + 16);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            c[j] = small_uint_to_float((w.x >> (4 * j)) & 0xFu);
-            c[8 + j] = small_uint_to_float((w.y >> (4 * j)) & 0xFu);
+        for (int j = 0; j < 8; ++j) f[j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+    } else if constexpr (KBITS == 4) {
+        const uint2 w = lds64(row + part * 8);
+        const uint32_t a0 = w.x & 0x0F0F0F0Fu, b0 = (w.x >> 4) & 0x0F0F0F0Fu;
+        const uint32_t a1 = w.y & 0x0F0F0F0Fu, b1 = (w.y >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            f[k] = make_float2(code_f(a0, k), code_f(b0, k));
+            f[4 + k] = make_float2(code_f(a1, k), code_f(b1, k));
         }
     } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(row + part * 4);
+        const uint32_t w = lds32(row + part * 4);
+        const uint32_t a = w & 0x03030303u, b = (w >> 2) & 0x03030303u;
+        const uint32_t c = (w >> 4) & 0x03030303u, d = (w >> 6) & 0x03030303u;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) c[j] = small_uint_to_float((w >> (2 * j)) & 0x3u);
+        for (int k = 0; k < 4; ++k) {
+            f[2 * k] = make_float2(code_f(a, k), code_f(b, k));
+            f[2 * k + 1] = make_float2(code_f(c, k), code_f(d, k));
+        }
     }
 }
 
-__device__ __forceinline__ void bf16_16(const uint8_t *row, int part, float c[16]) {
-    const uint4 *p = reinterpret_cast<const uint4 *>(row + part * 32);
-    const uint4 a = p[0], b = p[1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        c[2 * j] = __uint_as_float(w[j] << 16);
-        c[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-}
-
-// Eight value channels [8*slice, 8*slice + 8) of one token row.
+// 8 value channels [8*slice, 8*slice + 8) as 4 pairs.
 template <int VM, int VBITS>
-__device__ __forceinline__ void v_vals8(const uint8_t *row, int slice, float c[8]) {
+__device__ __forceinline__ void value_pairs(const uint8_t *row, int slice, float2 f[4]) {
     if constexpr (VM == V_BF16) {
-        const uint4 a = *reinterpret_cast<const uint4 *>(row + slice * 16);
+        const uint4 a = lds128(row + slice * 16);
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            c[2 * j] = __uint_as_float(w[j] << 16);
-            c[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
+        for (int j = 0; j < 4; ++j) f[j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
     } else if constexpr (VBITS == 4) {
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(row + slice * 4);
+        const uint32_t w = lds32(row + slice * 4);
+        const uint32_t a = w & 0x0F0F0F0Fu, b = (w >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) c[j] = small_uint_to_float((w >> (4 * j)) & 0xFu);
+        for (int k = 0; k < 4; ++k) f[k] = make_float2(code_f(a, k), code_f(b, k));
     } else {
-        const uint32_t w = *reinterpret_cast<const uint16_t *>(row + slice * 2);
+        const uint32_t w = lds16(row + slice * 2);
+        const uint32_t a = w & 0x0303u, b = (w >> 2) & 0x0303u;
+        const uint32_t c = (w >> 4) & 0x0303u, d = (w >> 6) & 0x0303u;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) c[j] = small_uint_to_float((w >> (2 * j)) & 0x3u);
+        for (int k = 0; k < 2; ++k) {
+            f[2 * k] = make_float2(code_f(a, k), code_f(b, k));
+            f[2 * k + 1] = make_float2(code_f(c, k), code_f(d, k));
+        }
     }
 }
 
 // Per-warp decode state.
 template <int GQA>
 struct WarpState {
-    float m_own;     // running max (log2 domain) of this lane's head
-    float l_own;     // running sum of this lane's tokens' weights (own head)
-    float zs[8];     // running sum of p * zero per value group (own head)
-    float o[GQA][8]; // value accumulators: 8 channels x GQA heads
+    float m_own;      // running max (log2 domain) of this lane's head
+    float l_own;      // running sum of the weights of this lane's tokens (own head)
+    float corr[4];    // value-group correction terms owned by this lane (own head)
+    float2 o[GQA][4]; // value accumulators: 8 channels (4 pairs) x GQA heads
 };
 
-// One tile of up to 64 tokens: rows at kc / ks / vc / vs (generic pointers,
-// shared or global memory), `n` valid tokens. qk/qc hold the lane's query
-// (already scaled) in the layout the key mode needs.
-template <int GQA, int KM, int VM, int KBITS, int VBITS>
-__device__ __forceinline__ void process_tile(const uint8_t *kc, const __half2 *ks,
-                                             const uint8_t *vc, const __half2 *vs, int n,
-                                             int group_k, int group_v, const float (&qk)[GQA][16],
+template <int GQA>
+struct LaneMap {
+    static constexpr int kPerHead = 8 / GQA;                 // lanes of a token per head
+    static constexpr int kOwnShift = (GQA == 4) ? 1 : (GQA == 2 ? 2 : 3);
+};
+
+// One tile: rows at kc / ks / vc / vs (shared memory), `n` valid tokens, TPW
+// tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)).
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW>
+__device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
+                                             const uint8_t *vc, const uint8_t *vs, int n,
+                                             int group_k, int group_v, const float2 (&qk)[GQA][8],
                                              const float (&qc)[GQA], WarpState<GQA> &st,
                                              float *wsm, int warp, int lane) {
     constexpr int KROW = KRow<KM, KBITS>::bytes;
     constexpr int VROW = VRow<VM, VBITS>::bytes;
+    constexpr int PASSES = TPW / 4;
+    constexpr int kPerHead = LaneMap<GQA>::kPerHead;
+    constexpr int kOwnShift = LaneMap<GQA>::kOwnShift;
     const int i = lane >> 3, part = lane & 7;
+    const int h_own = part >> kOwnShift;
+    const int r_own = part & (kPerHead - 1);  // rank of this lane among its head's lanes
     const int n_vg = (VM == V_BF16) ? 1 : kHeadDim / group_v;
     const int ngk = (KM == K_TOKEN) ? kHeadDim / group_k : 0;
-    constexpr int kOwnShift = (GQA == 4) ? 1 : (GQA == 2 ? 2 : 3);
-    const int h_own = part >> kOwnShift;
+    const int t_warp = warp * TPW;
 
     // ---- scores ----
-    float sc[4];
+    float sc[PASSES];
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-        const int tt = pass * 16 + warp * 4 + i;
-        const int tr = tt < n ? tt : 0;  // masked tokens read row 0 (always staged)
-        float c[16];
-        const uint8_t *row = kc + static_cast<size_t>(tr) * KROW;
-        if constexpr (KM == K_BF16) bf16_16(row, part, c);
-        else k_codes16<KBITS>(row, part, c);
+    for (int pass = 0; pass < PASSES; ++pass) {
+        const int tt = t_warp + pass * 4 + i;
+        float2 f[8];
+        key_pairs<KM, KBITS>(kc + tt * KROW, part, f);
         float acc[GQA];
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
-            float a = 0.0f;
+            float2 a = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) a = fmaf(qk[g][j], c[j], a);
-            acc[g] = a;
+            for (int j = 0; j < 8; ++j) ffma2(a, qk[g][j], f[j]);
+            acc[g] = a.x + a.y;
         }
         if constexpr (KM == K_TOKEN) {
-            const float2 szf = __half22float2(ks[tr * ngk + (part * 16) / group_k]);
+            const float2 szf = half2_lds(ks + (tt * ngk + (part * 16) / group_k) * 4);
+            const float zc = fmaf(-128.0f, szf.x, szf.y);  // z - 128 s
 #pragma unroll
-            for (int g = 0; g < GQA; ++g) acc[g] = fmaf(szf.x, acc[g], szf.y * qc[g]);
+            for (int g = 0; g < GQA; ++g) acc[g] = fmaf(szf.x, acc[g], zc * qc[g]);
         } else if constexpr (KM == K_CHANNEL) {
 #pragma unroll
             for (int g = 0; g < GQA; ++g) acc[g] += qc[g];
@@ -209,42 +273,51 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const __half2 *k
     }
 
     // ---- online softmax (per warp, per head) ----
-    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    float mx = sc[0];
+#pragma unroll
+    for (int pass = 1; pass < PASSES; ++pass) mx = fmaxf(mx, sc[pass]);
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     const float m_new = fmaxf(st.m_own, mx);
-    float alpha, p[4];
+    float alpha, p[PASSES];
     if (m_new == -INFINITY) {
         alpha = 1.0f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) p[k] = 0.0f;
+        for (int k = 0; k < PASSES; ++k) p[k] = 0.0f;
     } else {
         alpha = fast_exp2(st.m_own - m_new);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) p[k] = fast_exp2(sc[k] - m_new);
+        for (int k = 0; k < PASSES; ++k) p[k] = fast_exp2(sc[k] - m_new);
     }
     st.m_own = m_new;
-    st.l_own = st.l_own * alpha + (p[0] + p[1]) + (p[2] + p[3]);
-    const bool writer = (part & ((8 / GQA) - 1)) == 0;
+    float psum = p[0];
 #pragma unroll
-    for (int gv = 0; gv < 8; ++gv) st.zs[gv] *= alpha;
+    for (int k = 1; k < PASSES; ++k) psum += p[k];
+    st.l_own = fmaf(st.l_own, alpha, psum);
+    // Value weights: w = 256 * p * s per (token, value group), duplicated as a
+    // pair; the owner lanes of a head split the groups between them.
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
+    for (int c = 0; c < 4; ++c) st.corr[c] *= alpha;
+#pragma unroll
+    for (int pass = 0; pass < PASSES; ++pass) {
         const int j = pass * 4 + i;  // warp-local token index
-        const int tt = pass * 16 + warp * 4 + i;
-        const int tr = tt < n ? tt : 0;
-        float *wrow = wsm + (j * n_vg) * GQA;
+        const int tt = t_warp + j;
+        float2 *wrow = reinterpret_cast<float2 *>(wsm) + j * n_vg * GQA;
         if constexpr (VM == V_BF16) {
-            if (writer) wrow[h_own] = p[pass];
+            if (r_own == 0) wrow[h_own] = make_float2(p[pass], p[pass]);
         } else {
-            for (int gv = 0; gv < n_vg; ++gv) {
-                const float2 szf = __half22float2(vs[tr * n_vg + gv]);
-                st.zs[gv] = fmaf(p[pass], szf.y, st.zs[gv]);
-                if (writer) wrow[gv * GQA + h_own] = p[pass] * szf.x;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int gv = r_own + c * kPerHead;
+                if (gv < n_vg) {
+                    const float2 szf = half2_lds(vs + (tt * n_vg + gv) * 4);
+                    const float w = 256.0f * p[pass] * szf.x;
+                    st.corr[c] = fmaf(p[pass], fmaf(-128.0f, szf.x, szf.y), st.corr[c]);
+                    wrow[gv * GQA + h_own] = make_float2(w, w);
+                }
             }
         }
     }
-    // alpha of every head, from the lane pair that owns it (token slot 0)
     float alpha_g[GQA];
 #pragma unroll
     for (int g = 0; g < GQA; ++g) alpha_g[g] = __shfl_sync(0xffffffffu, alpha, g << kOwnShift);
@@ -259,44 +332,42 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const __half2 *k
 #pragma unroll
         for (int g = 0; g < GQA; ++g)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) st.o[g][c] *= alpha_g[g];
+            for (int c = 0; c < 4; ++c) {
+                st.o[g][c].x *= alpha_g[g];
+                st.o[g][c].y *= alpha_g[g];
+            }
     }
     const int gv_lane = (VM == V_BF16) ? 0 : (8 * slice) / group_v;
-#pragma unroll 2
-    for (int k = 0; k < 8; ++k) {
-        const int j = 2 * k + parity;
-        const int tt = (j >> 2) * 16 + warp * 4 + (j & 3);
-        if (tt >= n) continue;
-        float c[8];
-        v_vals8<VM, VBITS>(vc + static_cast<size_t>(tt) * VROW, slice, c);
-        const float *wrow = wsm + (j * n_vg + gv_lane) * GQA;
-        float w[GQA];
-        if constexpr (GQA == 4) {
-            const float4 w4 = *reinterpret_cast<const float4 *>(wrow);
-            w[0] = w4.x; w[1] = w4.y; w[2] = w4.z; w[3] = w4.w;
-        } else {
 #pragma unroll
-            for (int g = 0; g < GQA; ++g) w[g] = wrow[g];
+    for (int k = 0; k < TPW / 2; ++k) {
+        const int j = 2 * k + parity;
+        const int tt = t_warp + j;
+        if (VM == V_BF16 && tt >= n) continue;  // stale bf16 rows may be NaN
+        float2 f[4];
+        value_pairs<VM, VBITS>(vc + tt * VROW, slice, f);
+        const float2 *wrow = reinterpret_cast<const float2 *>(wsm) + (j * n_vg + gv_lane) * GQA;
+        float2 w[GQA];
+        if constexpr (GQA >= 2) {
+#pragma unroll
+            for (int g = 0; g < GQA; g += 2) {
+                const uint4 u = lds128(wrow + g);
+                w[g] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+                w[g + 1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+            }
+        } else {
+            const uint2 u = lds64(wrow);
+            w[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
         }
 #pragma unroll
         for (int g = 0; g < GQA; ++g)
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) st.o[g][cc] = fmaf(w[g], c[cc], st.o[g][cc]);
+            for (int c = 0; c < 4; ++c) ffma2(st.o[g][c], w[g], f[c]);
     }
     __syncwarp();
 }
 
-struct SmemLayout {
-    // after the NS stages:
-    float *qs;      // [GQA][128]
-    float *wsm;     // [4 warps][16 tokens][8 groups][GQA]
-    float *red;     // [4 warps][GQA][130]
-    uint64_t *full, *empty;
-    int *abort_flag;
-};
-
 template <int GQA, int KM, int VM, int KBITS, int VBITS, int NS>
-__global__ void __launch_bounds__(kThreads) decode_splitk_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const DecodeParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int split = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -311,14 +382,16 @@ __global__ void __launch_bounds__(kThreads) decode_splitk_kernel(const DecodePar
     const int t_end = min(T, t_begin + p.chunk);
     const int Tq = quantized_len(T, p.R);
     const int q_end = min(t_end, Tq);                // quantized tokens [t_begin, q_end)
-    const int n_tiles = q_end > t_begin ? (q_end - t_begin + kTile - 1) / kTile : 0;
-    const int w_begin = max(t_begin, Tq);            // window tokens [w_begin, t_end)
+    const int n_qt = q_end > t_begin ? (q_end - t_begin + kTile - 1) / kTile : 0;
+    const int w_begin = max(t_begin, Tq);            // bf16 window tokens [w_begin, t_end)
+    const int n_wt = t_end > w_begin ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
+    const int n_tiles = n_qt + n_wt;
 
     uint8_t *stages = smem;
     uint8_t *tail = smem + static_cast<size_t>(NS) * p.stage_bytes;
     float *qs = reinterpret_cast<float *>(tail);
     float *wsm_all = qs + GQA * kHeadDim;
-    float *red = wsm_all + kConsumerWarps * 16 * 8 * GQA;
+    float *red = wsm_all + kConsumerWarps * 16 * 8 * GQA * 2;
     uint64_t *full = reinterpret_cast<uint64_t *>(red + kConsumerWarps * GQA * 130);
     uint64_t *empty = full + NS;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + NS);
@@ -350,14 +423,22 @@ __global__ void __launch_bounds__(kThreads) decode_splitk_kernel(const DecodePar
                 break;
             issued = it + 1;
             if (it == p.skip_tile) continue;  // test hook: never arrive
-            const int t0 = t_begin + it * kTile;
-            const int n = min(kTile, q_end - t0);
             uint8_t *st = stages + static_cast<size_t>(s) * p.stage_bytes;
             // Collect the copies, sum their bytes, arm the barrier, then issue.
-            const uint8_t *src[4 * 8];
-            uint32_t off[4 * 8], len[4 * 8];
+            const uint8_t *src[16];
+            uint32_t off[16], len[16];
             int nc = 0;
-            if (!p.paged) {
+            if (it >= n_qt) {  // bf16 window rows
+                const int t0 = w_begin + (it - n_qt) * p.bf_tile;
+                const int n = min(p.bf_tile, t_end - t0);
+                const int64_t slot = sh * p.R + (t0 - Tq);
+                src[nc] = reinterpret_cast<const uint8_t *>(p.k_res + slot * kHeadDim);
+                off[nc] = 0; len[nc++] = n * kHeadDim * 2;
+                src[nc] = reinterpret_cast<const uint8_t *>(p.v_res + slot * kHeadDim);
+                off[nc] = p.bf_off_v; len[nc++] = n * kHeadDim * 2;
+            } else if (!p.paged) {
+                const int t0 = t_begin + it * kTile;
+                const int n = min(kTile, q_end - t0);
                 const int64_t row = sh * p.cap + t0;
                 src[nc] = p.k_codes + row * KROW; off[nc] = 0; len[nc++] = n * KROW;
                 if (KM == K_TOKEN) {
@@ -374,6 +455,8 @@ __global__ void __launch_bounds__(kThreads) decode_splitk_kernel(const DecodePar
                     off[nc] = p.off_vsz; len[nc++] = (n * ngv * 4 + 15) & ~15;
                 }
             } else {
+                const int t0 = t_begin + it * kTile;
+                const int n = min(kTile, q_end - t0);
                 const int ps = p.page_size;
                 const int span = ps < kTile ? ps : kTile;  // tokens per copy
                 for (int tp = t0; tp < t0 + n; tp += span) {
@@ -405,7 +488,7 @@ __global__ void __launch_bounds__(kThreads) decode_splitk_kernel(const DecodePar
         for (int it = max(0, issued - NS); it < issued; ++it) {
             if (it == p.skip_tile) continue;
             const int s = it % NS, r = it / NS;
-            uint64_t t0 = global_timer_ns();
+            const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(&full[s], r & 1)) {
                 if (static_cast<int64_t>(global_timer_ns() - t0) > p.timeout_ns) {
                     status_or(p.status, KVQ_DEV_TIMEOUT);
@@ -418,13 +501,28 @@ __global__ void __launch_bounds__(kThreads) decode_splitk_kernel(const DecodePar
 
     // --------------------------- consumers ---------------------------
     // Query: warp g < GQA loads head kvh*GQA + g, 4 channels per lane, and
-    // rotates it like the keys.
+    // rotates it like the keys; then scales by softmax_scale * log2(e).
     if (warp < GQA) {
         const int hq = kvh * GQA + warp;
         const int64_t base = (static_cast<int64_t>(seq) * p.Hq + hq) * kHeadDim + 4 * lane;
         float x[4];
+        if (p.q_dtype == KVQ_FP32) {
+            const float4 v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + base);
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+        } else {
+            const uint2 v = *reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.q) + base);
+            const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) x[j] = load_q_elem(p.q, base + j, p.q_dtype);
+            for (int j = 0; j < 2; ++j) {
+                if (p.q_dtype == KVQ_BF16) {
+                    x[2 * j] = bf16_bits_to_float(w[j] & 0xFFFFu);
+                    x[2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
+                } else {
+                    x[2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] & 0xFFFFu)));
+                    x[2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] >> 16)));
+                }
+            }
+        }
         if (p.hb > 0) {
             if (p.hb > 1) { float a = x[0], b = x[1]; x[0] = a + b; x[1] = a - b;
                             a = x[2]; b = x[3]; x[2] = a + b; x[3] = a - b; }
@@ -447,120 +545,128 @@ __global__ void __launch_bounds__(kThreads) decode_splitk_kernel(const DecodePar
     named_sync(1, kConsumers);
 
     const int part = lane & 7;
-    float qk[GQA][16];
+    // Query registers in the layout of the key mode (see the header comment):
+    // token-wise codes: 256 q, with qc = sum of the lane's q (zero-point term);
+    // channel-wise codes: set per block below; bf16 keys: q itself.
+    float2 qk[GQA][8];
     float qc[GQA];
+    auto load_plain_q = [&](float scale_q) {
 #pragma unroll
-    for (int g = 0; g < GQA; ++g) {
-        float s = 0.0f;
+        for (int g = 0; g < GQA; ++g) {
+            float s = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            qk[g][j] = qs[g * kHeadDim + part * 16 + j];
-            s += qk[g][j];
+            for (int j = 0; j < 8; ++j) {
+                const float a = qs[g * kHeadDim + part * 16 + 2 * j];
+                const float b = qs[g * kHeadDim + part * 16 + 2 * j + 1];
+                qk[g][j] = make_float2(a * scale_q, b * scale_q);
+                s += a + b;
+            }
+            qc[g] = s;
         }
-        qc[g] = (KM == K_TOKEN) ? s : 0.0f;
-    }
+    };
+    load_plain_q(KM == K_TOKEN ? 256.0f : 1.0f);
 
     WarpState<GQA> st;
     st.m_own = -INFINITY;
     st.l_own = 0.0f;
 #pragma unroll
-    for (int gv = 0; gv < 8; ++gv) st.zs[gv] = 0.0f;
+    for (int c = 0; c < 4; ++c) st.corr[c] = 0.0f;
 #pragma unroll
     for (int g = 0; g < GQA; ++g)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) st.o[g][c] = 0.0f;
-    float *wsm = wsm_all + warp * 16 * 8 * GQA;
+        for (int c = 0; c < 4; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
+    float *wsm = wsm_all + warp * 16 * 8 * GQA * 2;
 
     int cur_block = -1;
     for (int it = 0; it < n_tiles; ++it) {
         const int s = it % NS, r = it / NS;
         if (!mbar_wait_bounded(&full[s], r & 1, p.timeout_ns, p.status, abort_flag)) break;
-        const uint8_t *st_base = stages + static_cast<size_t>(s) * p.stage_bytes;
-        const int t0 = t_begin + it * kTile;
-        const int n = min(kTile, q_end - t0);
-        if constexpr (KM == K_CHANNEL) {
-            const int blk = t0 / p.R;
-            if (blk != cur_block) {  // fold this block's channel scales into q
-                cur_block = blk;
-                const __half2 *ksz = reinterpret_cast<const __half2 *>(st_base + p.off_ksz);
+        const uint8_t *sb = stages + static_cast<size_t>(s) * p.stage_bytes;
+        if (it < n_qt) {
+            const int t0 = t_begin + it * kTile;
+            const int n = min(kTile, q_end - t0);
+            if constexpr (KM == K_CHANNEL) {
+                const int blk = t0 / p.R;
+                if (blk != cur_block) {  // fold this block's channel scales into q
+                    cur_block = blk;
 #pragma unroll
-                for (int g = 0; g < GQA; ++g) {
-                    float c = 0.0f;
+                    for (int g = 0; g < GQA; ++g) {
+                        float c = 0.0f;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float2 szf = __half22float2(ksz[part * 16 + j]);
-                        const float qv = qs[g * kHeadDim + part * 16 + j];
-                        qk[g][j] = qv * szf.x;
-                        c = fmaf(qv, szf.y, c);
+                        for (int j = 0; j < 8; ++j) {
+                            const int ch = part * 16 + 2 * j;
+                            const float2 s0 = half2_lds(sb + p.off_ksz + ch * 4);
+                            const float2 s1 = half2_lds(sb + p.off_ksz + (ch + 1) * 4);
+                            const float qa = qs[g * kHeadDim + ch], qb = qs[g * kHeadDim + ch + 1];
+                            qk[g][j] = make_float2(256.0f * qa * s0.x, 256.0f * qb * s1.x);
+                            c = fmaf(qa, fmaf(-128.0f, s0.x, s0.y), c);
+                            c = fmaf(qb, fmaf(-128.0f, s1.x, s1.y), c);
+                        }
+                        qc[g] = c;
                     }
-                    qc[g] = c;
                 }
             }
+            process_tile<GQA, KM, VM, KBITS, VBITS, kTile / kConsumerWarps>(
+                sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, n, p.group_k, p.group_v, qk, qc,
+                st, wsm, warp, lane);
+        } else {
+            if (it == n_qt && KM != K_BF16) {
+                load_plain_q(1.0f);
+#pragma unroll
+                for (int g = 0; g < GQA; ++g) qc[g] = 0.0f;
+            }
+            const int t0 = w_begin + (it - n_qt) * p.bf_tile;
+            const int n = min(p.bf_tile, t_end - t0);
+            if constexpr (KM == K_BF16) {
+                process_tile<GQA, K_BF16, V_BF16, 16, 16, kTile / kConsumerWarps>(
+                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, qk, qc, st, wsm, warp, lane);
+            } else {
+                process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps>(
+                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, qk, qc, st, wsm, warp, lane);
+            }
         }
-        process_tile<GQA, KM, VM, KBITS, VBITS>(
-            st_base, reinterpret_cast<const __half2 *>(st_base + p.off_ksz), st_base + p.off_vc,
-            reinterpret_cast<const __half2 *>(st_base + p.off_vsz), n, p.group_k, p.group_v, qk, qc,
-            st, wsm, warp, lane);
         if (lane == 0) mbar_arrive(&empty[s]);
     }
-
     const bool aborted = *abort_flag != 0;
-    // bf16 window tokens [w_begin, t_end), read straight from global memory.
-    if (!aborted && w_begin < t_end) {
-#pragma unroll
-        for (int g = 0; g < GQA; ++g) {
-            float s = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                qk[g][j] = qs[g * kHeadDim + part * 16 + j];
-                s += qk[g][j];
-            }
-            qc[g] = 0.0f;
-            (void)s;
-        }
-        const int Tq_base = Tq;
-        for (int t0 = w_begin; t0 < t_end; t0 += kTile) {
-            const int n = min(kTile, t_end - t0);
-            const int64_t slot = sh * p.R + (t0 - Tq_base);
-            const uint8_t *kw = reinterpret_cast<const uint8_t *>(p.k_res + slot * kHeadDim);
-            const uint8_t *vw = reinterpret_cast<const uint8_t *>(p.v_res + slot * kHeadDim);
-            process_tile<GQA, K_BF16, V_BF16, 16, 16>(kw, nullptr, vw, nullptr, n, 128, 128, qk, qc,
-                                                       st, wsm, warp, lane);
-        }
-    }
 
     // ---- merge the four warps ----
-    constexpr int kOwnShift = (GQA == 4) ? 1 : (GQA == 2 ? 2 : 3);
-    const int i_tok = lane >> 3;
-    (void)i_tok;
+    constexpr int kPerHead = LaneMap<GQA>::kPerHead;
+    constexpr int kOwnShift = LaneMap<GQA>::kOwnShift;
     float l_own = st.l_own;
     l_own += __shfl_xor_sync(0xffffffffu, l_own, 8);
     l_own += __shfl_xor_sync(0xffffffffu, l_own, 16);
-    float zs[8];
+    float corr[4];
 #pragma unroll
-    for (int gv = 0; gv < 8; ++gv) {
-        zs[gv] = st.zs[gv];
-        zs[gv] += __shfl_xor_sync(0xffffffffu, zs[gv], 8);
-        zs[gv] += __shfl_xor_sync(0xffffffffu, zs[gv], 16);
+    for (int c = 0; c < 4; ++c) {
+        corr[c] = st.corr[c];
+        corr[c] += __shfl_xor_sync(0xffffffffu, corr[c], 8);
+        corr[c] += __shfl_xor_sync(0xffffffffu, corr[c], 16);
     }
     const int slice = lane & 15;
     const int gv_lane = (VM == V_BF16) ? 0 : (8 * slice) / p.group_v;
 #pragma unroll
     for (int g = 0; g < GQA; ++g) {
-        const int src = g << kOwnShift;
+        // group gv of head g lives in lane (g << kOwnShift) + gv % kPerHead, slot gv / kPerHead
         float zg = 0.0f;
 #pragma unroll
-        for (int gv = 0; gv < 8; ++gv) {
-            const float z = __shfl_sync(0xffffffffu, zs[gv], src);
-            if (gv == gv_lane) zg = z;
-        }
-        const float mg = __shfl_sync(0xffffffffu, st.m_own, src);
-        const float lg = __shfl_sync(0xffffffffu, l_own, src);
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float v = st.o[g][c] + __shfl_xor_sync(0xffffffffu, st.o[g][c], 16);
-            if (VM == V_TOKEN) v += zg;
-            if (lane < 16) red[(warp * GQA + g) * 130 + 8 * slice + c] = v;
+            for (int r = 0; r < kPerHead; ++r) {
+                const float z = __shfl_sync(0xffffffffu, corr[c], (g << kOwnShift) + r);
+                if (VM == V_TOKEN && gv_lane == r + c * kPerHead) zg = z;
+            }
+        }
+        const float mg = __shfl_sync(0xffffffffu, st.m_own, g << kOwnShift);
+        const float lg = __shfl_sync(0xffffffffu, l_own, g << kOwnShift);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float2 v = st.o[g][c];
+            v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
+            v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
+            if (lane < 16) {
+                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c] = v.x + zg;
+                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c + 1] = v.y + zg;
+            }
         }
         if (lane == 0) {
             red[(warp * GQA + g) * 130 + 128] = mg;
@@ -614,28 +720,38 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *o_part, 
 // Host side
 // ---------------------------------------------------------------------------
 struct StageLayout {
-    int bytes, off_ksz, off_vc, off_vsz;
+    int bytes, off_ksz, off_vc, off_vsz, bf_tile, bf_off_v;
 };
 
 inline int round16(int x) { return (x + 15) & ~15; }
 
 StageLayout stage_layout(const kvq_cache_desc &d) {
-    const int krow = d.bits_k == 16 ? 256 : 128 * d.bits_k / 8;
-    const int vrow = d.bits_v == 16 ? 256 : 128 * d.bits_v / 8;
-    int ksz = 0, vsz = 0;
-    if (d.bits_k != 16) ksz = (d.axis_k == KVQ_PER_CHANNEL) ? 128 * 4 : kTile * (128 / d.group_k) * 4;
-    if (d.bits_v != 16) vsz = kTile * (128 / d.group_v) * 4;
-    StageLayout L;
+    StageLayout L{};
+    if (d.bits_k == 16) {  // every tile is bf16 rows: K at 0, V after it
+        L.bf_tile = kTile;
+        L.bf_off_v = kTile * 256;
+        L.off_vc = L.bf_off_v;
+        L.bytes = 2 * kTile * 256;
+        return L;
+    }
+    const int krow = 128 * d.bits_k / 8;
+    const int vrow = 128 * d.bits_v / 8;
+    const int ksz = (d.axis_k == KVQ_PER_CHANNEL) ? 128 * 4 : kTile * (128 / d.group_k) * 4;
+    const int vsz = kTile * (128 / d.group_v) * 4;
     L.off_ksz = round16(kTile * krow);
     L.off_vc = L.off_ksz + round16(ksz);
     L.off_vsz = L.off_vc + round16(kTile * vrow);
-    L.bytes = (L.off_vsz + round16(vsz) + 127) & ~127;
+    L.bytes = L.off_vsz + round16(vsz);
+    L.bf_tile = kWinTile;
+    L.bf_off_v = kWinTile * 256;
+    if (d.residual_len > 0) L.bytes = std::max(L.bytes, 2 * kWinTile * 256);
+    L.bytes = (L.bytes + 127) & ~127;
     return L;
 }
 
 template <int GQA>
 size_t tail_bytes(int NS) {
-    return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * 16 * 8 * GQA + kConsumerWarps * GQA * 130) +
+    return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * 16 * 8 * GQA * 2 + kConsumerWarps * GQA * 130) +
            sizeof(uint64_t) * 2 * NS + 16;
 }
 
@@ -730,6 +846,8 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.off_ksz = L.off_ksz;
     p.off_vc = L.off_vc;
     p.off_vsz = L.off_vsz;
+    p.bf_tile = L.bf_tile;
+    p.bf_off_v = L.bf_off_v;
     p.timeout_ns = debug_hooks().wait_timeout_ns;
     p.skip_tile = debug_hooks().skip_tile;
     const dim3 grid(plan.n_split, d.num_kv_heads, num_seqs);

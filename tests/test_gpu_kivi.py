@@ -13,14 +13,16 @@ from gpu_common import (D, SCALE, append, assert_close, dev, lens_tensor, oracle
 pytestmark = pytest.mark.gpu
 
 
-def _spec(S, H, cap, bits=2, G_v=32, R=128):
-    return K.CacheSpec(S, H, bits_k=bits, bits_v=bits, group_k=R, group_v=G_v, per_channel_k=True,
-                       residual_len=R, capacity_tokens=cap)
+def _spec(S, H, cap, bits=2, G_v=32, R=128, per_channel=True):
+    return K.CacheSpec(S, H, bits_k=bits, bits_v=bits, group_k=R if per_channel else 128,
+                       group_v=G_v, per_channel_k=per_channel, residual_len=R, capacity_tokens=cap)
 
 
 def _check_state(cache, k, v, T, s, h):
     sp = cache.spec
     R = sp.residual_len
+    if not sp.per_channel_k:
+        return _check_state_token_keys(cache, k, v, T, s, h)
     want = oracle.quantize_kivi_sequence(np.ascontiguousarray(k[:T, h]), np.ascontiguousarray(v[:T, h]),
                                          R, sp.bits_k, sp.bits_v, sp.group_v)
     Tq = want["Tq"]
@@ -39,15 +41,46 @@ def _check_state(cache, k, v, T, s, h):
     assert np.array_equal(kw, want["k_win"]) and np.array_equal(vw, want["v_win"])
 
 
-@pytest.mark.parametrize("bits,G_v", [(2, 32), (4, 128), (2, 16)])
-def test_window_flush_and_attention(bits, G_v):
+def _check_state_token_keys(cache, k, v, T, s, h):
+    # residual window with token-wise key groups: blocks quantized per token
+    sp = cache.spec
+    R = sp.residual_len
+    Tq = oracle.kivi_split(T, R)
+    for which, x, G, bits in (("k", k, sp.group_k, sp.bits_k), ("v", v, sp.group_v, sp.bits_v)):
+        ec, ez = oracle.quantize_tokens(np.ascontiguousarray(x[:Tq, h]), 0, G, bits)
+        assert np.array_equal(cache.codes_view(which)[s, h, :Tq].cpu().numpy(), ec)
+        assert np.array_equal(cache.sz_view(which)[s, h, :Tq].cpu().numpy().view(np.uint16), ez)
+    S, H = sp.num_seqs, sp.num_kv_heads
+    kw = cache.k_res.view(S, H, R, D)[s, h, :T - Tq].float().cpu().numpy()
+    assert np.array_equal(kw, k[Tq:T, h])
+
+
+def _oracle_decode(k, v, q, spec):
+    if spec.per_channel_k:
+        return oracle_decode_kivi(k, v, q, spec)
+    H, T = k.shape[1], k.shape[0]
+    R = spec.residual_len
+    Tq = oracle.kivi_split(T, R)
+    kh = np.zeros((H, T, D))
+    vh = np.zeros((H, T, D))
+    for h in range(H):
+        for dst, x, G, bits in ((kh, k, spec.group_k, spec.bits_k), (vh, v, spec.group_v, spec.bits_v)):
+            c, z = oracle.quantize_tokens(np.ascontiguousarray(x[:Tq, h]), 0, G, bits)
+            dst[h, :Tq] = oracle.dequant_tokens(c, z, G, bits) if Tq else 0
+            dst[h, Tq:] = x[Tq:, h]
+    return oracle.decode_attention_gqa(q, kh, vh, SCALE)
+
+
+@pytest.mark.parametrize("bits,G_v,per_channel", [(2, 32, True), (4, 128, True), (2, 16, True),
+                                                   (4, 32, False)])
+def test_window_flush_and_attention(bits, G_v, per_channel):
     H, Hq, S = 2, 8, 3
     total = [702, 141, 130]
     g = np.random.default_rng(bits + G_v)
     ch = W.outlier_channels(g)
     ks = [W.finish(W.keys(g, (t, H, D), ch), "bf16") for t in total]
     vs = [W.finish(W.normal(g, (t, H, D)), "bf16") for t in total]
-    cache = K.KVCache(_spec(S, H, 768, bits, G_v))
+    cache = K.KVCache(_spec(S, H, 768, bits, G_v, per_channel=per_channel))
     sl = lens_tensor([0] * S)
     # bulk chunk, then single tokens across flush boundaries, then another chunk
     plan = [[300, 5, 127]] + [[1, 1, 1]] * 3 + [[0, 130, 0]] + [[1, 1, 0]] * 2 + [[397, 1, 0]]
@@ -64,7 +97,7 @@ def test_window_flush_and_attention(bits, G_v):
     assert cache.device_status() == 0
     out = K.decode_attention(cache.desc, dev(qs, "bf16"), sl, 768, SCALE).cpu().numpy()
     for s in range(S):
-        assert_close(out[s], oracle_decode_kivi(ks[s][:pos[s]], vs[s][:pos[s]], qs[s], cache.spec),
+        assert_close(out[s], _oracle_decode(ks[s][:pos[s]], vs[s][:pos[s]], qs[s], cache.spec),
                      "seq %d" % s)
 
 

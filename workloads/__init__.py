@@ -96,8 +96,18 @@ def keys(g: np.random.Generator, shape, channels: np.ndarray, factor: float = 20
     return k
 
 
+def to_fp16_values(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest fp16 (input preparation only)."""
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).astype(np.float32)
+
+
 def finish(x: np.ndarray, dtype: str) -> np.ndarray:
-    return to_bf16_values(x) if dtype == "bf16" else np.ascontiguousarray(x, np.float32)
+    """Values of the workload's input dtype ("bf16", "fp16" or "fp32") as float32."""
+    if dtype == "bf16":
+        return to_bf16_values(x)
+    if dtype == "fp16":
+        return to_fp16_values(x)
+    return np.ascontiguousarray(x, np.float32)
 
 
 def paged_lengths(seed: int, n: int = 64, median: int = 4096, sigma: float = 1.0,
