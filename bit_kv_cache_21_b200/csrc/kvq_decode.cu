@@ -46,6 +46,9 @@ constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kLog2e = 1.4426950408889634f;
+#ifndef KVQ_DECODE_MIN_BLOCKS
+#define KVQ_DECODE_MIN_BLOCKS 2  // resident CTAs per SM the register budget targets
+#endif
 
 enum KMode { K_TOKEN = 0, K_CHANNEL = 1, K_BF16 = 2 };
 enum VMode { V_TOKEN = 0, V_BF16 = 2 };
@@ -100,27 +103,20 @@ __device__ __forceinline__ void ffma2(float2 &d, float2 a, float2 b) {
 }
 
 // ---- shared-memory loads ----------------------------------------------------
+// Plain typed loads: the compiler sees their dependence on the stores and on
+// the mbarrier waits (asm with a memory clobber) and keeps them in order; the
+// pointers all derive from the kernel's shared array.
 __device__ __forceinline__ uint32_t lds32(const void *p) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)));
-    return v;
+    return *static_cast<const uint32_t *>(p);
 }
 __device__ __forceinline__ uint32_t lds16(const void *p) {
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_addr(p)));
-    return v;
+    return *static_cast<const uint16_t *>(p);
 }
 __device__ __forceinline__ uint2 lds64(const void *p) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr(p)));
-    return v;
+    return *static_cast<const uint2 *>(p);
 }
 __device__ __forceinline__ uint4 lds128(const void *p) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(smem_addr(p)));
-    return v;
+    return *static_cast<const uint4 *>(p);
 }
 __device__ __forceinline__ float2 half2_lds(const void *p) {
     const uint32_t u = lds32(p);
@@ -128,13 +124,23 @@ __device__ __forceinline__ float2 half2_lds(const void *p) {
 }
 
 // ---- code -> float ----------------------------------------------------------
-// Byte k of `b` holds a code in its low bits; the result is the float
-// 0.5 + code/256 (the byte becomes mantissa bits 16..23 of 0.5). One PRMT.
-__device__ __forceinline__ float code_f(uint32_t b, int k) {
+// A byte value X < 128 placed into bits 16..22 of 0.5 gives the float
+// 0.5 + X/256 exactly (bit 23, the exponent's low bit, stays 0). One PRMT.
+// Every encoded byte below is < 128: INT4 codes are split into their low and
+// high nibble planes; INT2 codes use the planes
+//   X0 = c0, X1 = c0 + 4c1, X2 = c0 + 4c1 + 16c2, X3 = c1 + 4c2 + 16c3
+// (three masks and one shift of the packed word), all < 64. The floats are
+// linear in the codes; the query is transformed once per CTA so that its dot
+// product with them is the dot product with the codes (query_coeffs), and the
+// value accumulators are untangled once per split (value_channels).
+__device__ __forceinline__ float byte_f(uint32_t b, int k) {
     return __uint_as_float(__byte_perm(b, 0x3F000000u, 0x7054u | (static_cast<uint32_t>(k) << 8)));
 }
 
-// 16 key channels [16*part, 16*part + 16) as 8 (even, odd) pairs.
+// 16 key channels [16*part, 16*part + 16) as 8 float pairs.
+//   INT4 byte k (channels lo, hi): {f(lo), f(hi)}
+//   INT2 byte k (channels c0..c3): {f(X0), f(X1)}, {f(X2), f(X3)}
+//   bf16: the channel values themselves.
 template <int KM, int KBITS>
 __device__ __forceinline__ void key_pairs(const uint8_t *row, int part, float2 f[8]) {
     if constexpr (KM == K_BF16) {
@@ -148,22 +154,22 @@ __device__ __forceinline__ void key_pairs(const uint8_t *row, int part, float2 f
         const uint32_t a1 = w.y & 0x0F0F0F0Fu, b1 = (w.y >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            f[k] = make_float2(code_f(a0, k), code_f(b0, k));
-            f[4 + k] = make_float2(code_f(a1, k), code_f(b1, k));
+            f[k] = make_float2(byte_f(a0, k), byte_f(b0, k));
+            f[4 + k] = make_float2(byte_f(a1, k), byte_f(b1, k));
         }
     } else {
         const uint32_t w = lds32(row + part * 4);
-        const uint32_t a = w & 0x03030303u, b = (w >> 2) & 0x03030303u;
-        const uint32_t c = (w >> 4) & 0x03030303u, d = (w >> 6) & 0x03030303u;
+        const uint32_t x0 = w & 0x03030303u, x1 = w & 0x0F0F0F0Fu, x2 = w & 0x3F3F3F3Fu;
+        const uint32_t x3 = (w >> 2) & 0x3F3F3F3Fu;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            f[2 * k] = make_float2(code_f(a, k), code_f(b, k));
-            f[2 * k + 1] = make_float2(code_f(c, k), code_f(d, k));
+            f[2 * k] = make_float2(byte_f(x0, k), byte_f(x1, k));
+            f[2 * k + 1] = make_float2(byte_f(x2, k), byte_f(x3, k));
         }
     }
 }
 
-// 8 value channels [8*slice, 8*slice + 8) as 4 pairs.
+// 8 value channels [8*slice, 8*slice + 8) as 4 float pairs, same encoding.
 template <int VM, int VBITS>
 __device__ __forceinline__ void value_pairs(const uint8_t *row, int slice, float2 f[4]) {
     if constexpr (VM == V_BF16) {
@@ -175,41 +181,100 @@ __device__ __forceinline__ void value_pairs(const uint8_t *row, int slice, float
         const uint32_t w = lds32(row + slice * 4);
         const uint32_t a = w & 0x0F0F0F0Fu, b = (w >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) f[k] = make_float2(code_f(a, k), code_f(b, k));
+        for (int k = 0; k < 4; ++k) f[k] = make_float2(byte_f(a, k), byte_f(b, k));
     } else {
         const uint32_t w = lds16(row + slice * 2);
-        const uint32_t a = w & 0x0303u, b = (w >> 2) & 0x0303u;
-        const uint32_t c = (w >> 4) & 0x0303u, d = (w >> 6) & 0x0303u;
+        const uint32_t x0 = w & 0x0303u, x1 = w & 0x0F0Fu, x2 = w & 0x3F3Fu, x3 = (w >> 2) & 0x3F3Fu;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-            f[2 * k] = make_float2(code_f(a, k), code_f(b, k));
-            f[2 * k + 1] = make_float2(code_f(c, k), code_f(d, k));
+            f[2 * k] = make_float2(byte_f(x0, k), byte_f(x1, k));
+            f[2 * k + 1] = make_float2(byte_f(x2, k), byte_f(x3, k));
         }
     }
 }
 
-// Per-warp decode state.
+// Query coefficients for 16 channels x[0..15] of one head, in the pair
+// layout of key_pairs and times 256, such that
+//   sum_j qk[j] . f[j] = 128 * first + sum_i x_i c_i,
+// `first` being the sum of the (unscaled) coefficients.
+template <int KM, int KBITS>
+__device__ __forceinline__ void query_coeffs(const float x[16], float2 qk[8], float &first) {
+    first = 0.0f;
+    if constexpr (KM == K_BF16) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qk[j] = make_float2(x[2 * j], x[2 * j + 1]);
+    } else if constexpr (KBITS == 4) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            qk[j] = make_float2(256.0f * x[2 * j], 256.0f * x[2 * j + 1]);
+            first += x[2 * j] + x[2 * j + 1];
+        }
+    } else {
+        // a0 X0 + a1 X1 + a2 X2 + a3 X3 = q0 c0 + q1 c1 + q2 c2 + q3 c3
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float q0 = x[4 * k], q1 = x[4 * k + 1], q2 = x[4 * k + 2], q3 = x[4 * k + 3];
+            const float a3 = q3 * 0.0625f;
+            const float a2 = (q2 - 4.0f * a3) * 0.0625f;
+            const float a1 = (q1 - 4.0f * a2 - a3) * 0.25f;
+            const float a0 = q0 - a1 - a2;
+            qk[2 * k] = make_float2(256.0f * a0, 256.0f * a1);
+            qk[2 * k + 1] = make_float2(256.0f * a2, 256.0f * a3);
+            first += (a0 + a1) + (a2 + a3);
+        }
+    }
+}
+
 template <int GQA>
+__device__ __forceinline__ void load_sums(const float *p, float v[GQA]) {
+    if constexpr (GQA == 4) {
+        const uint4 u = lds128(p);
+        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+    } else {
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) v[g] = __uint_as_float(lds32(p + g));
+    }
+}
+
+// Per-warp decode state. VSLOTS: value groups a lane accumulates terms for
+// (1 when each head's groups fit one per lane, else 4).
+template <int GQA, int VSLOTS>
 struct WarpState {
-    float m_own;      // running max (log2 domain) of this lane's head
-    float l_own;      // running sum of the weights of this lane's tokens (own head)
-    float corr[4];    // value-group correction terms owned by this lane (own head)
-    float2 o[GQA][4]; // value accumulators: 8 channels (4 pairs) x GQA heads
+    float m_own;           // running max (log2 domain) used for this lane's head
+    float l_own;           // running sum of the weights of this lane's tokens (own head)
+    float wsum[VSLOTS];    // value groups owned by this lane: sum of p*s (own head)
+    float zsum[VSLOTS];    //                                   sum of p*z
+    float2 o[GQA][4];      // value accumulators: 8 channels (4 pairs) x GQA heads
 };
 
 template <int GQA>
 struct LaneMap {
-    static constexpr int kPerHead = 8 / GQA;                 // lanes of a token per head
+    static constexpr int kPerHead = 8 / GQA;  // lanes of a token per head
     static constexpr int kOwnShift = (GQA == 4) ? 1 : (GQA == 2 ? 2 : 3);
+};
+
+// Scores are kept in log2 units; a new tile maximum only moves the reference
+// when it exceeds the old one by more than this (weights then stay <= 2^8).
+constexpr float kRescaleSlack = 8.0f;
+
+// Per-lane query data for the key pass. Per-lane sums the inner loop needs
+// once per pass live in shared memory (qsum, [8 parts][3][GQA] floats, head
+// order as in qk): [0] sum of q, [1] sum over first-of-byte channels,
+// [2] channel-wise groups: sum q z - 128 sum first-of-byte q s.
+template <int GQA>
+struct QueryRegs {
+    float2 qk[GQA][8];     // coefficients, head order permuted for the reduce-scatter
+    float qa_own, qe_own;  // groups of 128: whole-head sums of the lane's own head
 };
 
 // One tile: rows at kc / ks / vc / vs (shared memory), `n` valid tokens, TPW
 // tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)).
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW>
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW, int VSLOTS>
 __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
                                              const uint8_t *vc, const uint8_t *vs, int n,
-                                             int group_k, int group_v, const float2 (&qk)[GQA][8],
-                                             const float (&qc)[GQA], WarpState<GQA> &st,
+                                             int group_k, int group_v, const QueryRegs<GQA> &Q,
+                                             const float *qsum, WarpState<GQA, VSLOTS> &st,
                                              float *wsm, int warp, int lane) {
     constexpr int KROW = KRow<KM, KBITS>::bytes;
     constexpr int VROW = VRow<VM, VBITS>::bytes;
@@ -221,6 +286,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     const int r_own = part & (kPerHead - 1);  // rank of this lane among its head's lanes
     const int n_vg = (VM == V_BF16) ? 1 : kHeadDim / group_v;
     const int ngk = (KM == K_TOKEN) ? kHeadDim / group_k : 0;
+    const bool post_scale = (KM == K_TOKEN) && group_k == kHeadDim;
     const int t_warp = warp * TPW;
 
     // ---- scores ----
@@ -228,35 +294,40 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 #pragma unroll
     for (int pass = 0; pass < PASSES; ++pass) {
         const int tt = t_warp + pass * 4 + i;
+        const int tr = tt < n ? tt : 0;  // masked tokens read row 0 (always staged)
         float2 f[8];
-        key_pairs<KM, KBITS>(kc + tt * KROW, part, f);
+        key_pairs<KM, KBITS>(kc + tr * KROW, part, f);
         float acc[GQA];
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
             float2 a = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) ffma2(a, qk[g][j], f[j]);
+            for (int j = 0; j < 8; ++j) ffma2(a, Q.qk[g][j], f[j]);
             acc[g] = a.x + a.y;
         }
+        float2 szf = make_float2(0.0f, 0.0f);
         if constexpr (KM == K_TOKEN) {
-            const float2 szf = half2_lds(ks + (tt * ngk + (part * 16) / group_k) * 4);
-            const float zc = fmaf(-128.0f, szf.x, szf.y);  // z - 128 s
+            szf = half2_lds(ks + (tr * ngk + (post_scale ? 0 : (part * 16) / group_k)) * 4);
+            if (!post_scale) {
+                float qa[GQA], qe[GQA];
+                load_sums<GQA>(qsum + (part * 3 + 0) * GQA, qa);
+                load_sums<GQA>(qsum + (part * 3 + 1) * GQA, qe);
 #pragma unroll
-            for (int g = 0; g < GQA; ++g) acc[g] = fmaf(szf.x, acc[g], zc * qc[g]);
+                for (int g = 0; g < GQA; ++g)
+                    acc[g] = fmaf(szf.x, fmaf(-128.0f, qe[g], acc[g]), szf.y * qa[g]);
+            }
         } else if constexpr (KM == K_CHANNEL) {
+            float qc[GQA];
+            load_sums<GQA>(qsum + (part * 3 + 2) * GQA, qc);
 #pragma unroll
             for (int g = 0; g < GQA; ++g) acc[g] += qc[g];
         }
         float val;
         if constexpr (GQA == 4) {
-            const bool b2 = (part & 4) != 0, b1 = (part & 2) != 0;
-            const float s0 = b2 ? acc[0] : acc[2], s1 = b2 ? acc[1] : acc[3];
-            const float r0 = __shfl_xor_sync(0xffffffffu, s0, 4);
-            const float r1 = __shfl_xor_sync(0xffffffffu, s1, 4);
-            const float ka = (b2 ? acc[2] : acc[0]) + r0;
-            const float kb = (b2 ? acc[3] : acc[1]) + r1;
-            const float r2 = __shfl_xor_sync(0xffffffffu, b1 ? ka : kb, 2);
-            val = (b1 ? kb : ka) + r2;
+            // heads are held in the order g ^ (2*b2 + b1), so no selects
+            const float ka = acc[0] + __shfl_xor_sync(0xffffffffu, acc[2], 4);
+            const float kb = acc[1] + __shfl_xor_sync(0xffffffffu, acc[3], 4);
+            val = ka + __shfl_xor_sync(0xffffffffu, kb, 2);
             val += __shfl_xor_sync(0xffffffffu, val, 1);
         } else {
 #pragma unroll
@@ -269,65 +340,72 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
             for (int g = 1; g < GQA; ++g)
                 if (h_own == g) val = acc[g];
         }
+        if constexpr (KM == K_TOKEN) {
+            if (post_scale) val = fmaf(szf.x, val, fmaf(szf.y, Q.qa_own, -128.0f * szf.x * Q.qe_own));
+        }
         sc[pass] = tt < n ? val : -INFINITY;
     }
 
-    // ---- online softmax (per warp, per head) ----
+    // ---- online softmax (per warp, per head), lazy rescaling ----
     float mx = sc[0];
 #pragma unroll
     for (int pass = 1; pass < PASSES; ++pass) mx = fmaxf(mx, sc[pass]);
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    const float m_new = fmaxf(st.m_own, mx);
-    float alpha, p[PASSES];
-    if (m_new == -INFINITY) {
-        alpha = 1.0f;
-#pragma unroll
-        for (int k = 0; k < PASSES; ++k) p[k] = 0.0f;
-    } else {
-        alpha = fast_exp2(st.m_own - m_new);
-#pragma unroll
-        for (int k = 0; k < PASSES; ++k) p[k] = fast_exp2(sc[k] - m_new);
+    float alpha = 1.0f;
+    if (mx > st.m_own + kRescaleSlack) {   // also true the first time (m_own = -inf)
+        alpha = fast_exp2(st.m_own - mx);  // 0 when m_own = -inf
+        st.m_own = mx;
     }
-    st.m_own = m_new;
+    // reference 0 while no token of this warp has been seen (all sc = -inf)
+    const float mref = (st.m_own == -INFINITY) ? 0.0f : st.m_own;
+    float p[PASSES];
+#pragma unroll
+    for (int k = 0; k < PASSES; ++k) p[k] = fast_exp2(sc[k] - mref);  // 0 for masked
     float psum = p[0];
 #pragma unroll
     for (int k = 1; k < PASSES; ++k) psum += p[k];
     st.l_own = fmaf(st.l_own, alpha, psum);
-    // Value weights: w = 256 * p * s per (token, value group), duplicated as a
-    // pair; the owner lanes of a head split the groups between them.
 #pragma unroll
-    for (int c = 0; c < 4; ++c) st.corr[c] *= alpha;
+    for (int c = 0; c < VSLOTS; ++c) {
+        st.wsum[c] *= alpha;
+        st.zsum[c] *= alpha;
+    }
+    // Value weights w = p * s per (token, value group), stored as a pair; the
+    // lanes of a head split the groups between them.
 #pragma unroll
     for (int pass = 0; pass < PASSES; ++pass) {
         const int j = pass * 4 + i;  // warp-local token index
         const int tt = t_warp + j;
+        const int tr = tt < n ? tt : 0;
         float2 *wrow = reinterpret_cast<float2 *>(wsm) + j * n_vg * GQA;
         if constexpr (VM == V_BF16) {
             if (r_own == 0) wrow[h_own] = make_float2(p[pass], p[pass]);
         } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < VSLOTS; ++c) {
                 const int gv = r_own + c * kPerHead;
                 if (gv < n_vg) {
-                    const float2 szf = half2_lds(vs + (tt * n_vg + gv) * 4);
-                    const float w = 256.0f * p[pass] * szf.x;
-                    st.corr[c] = fmaf(p[pass], fmaf(-128.0f, szf.x, szf.y), st.corr[c]);
+                    const float2 szf = half2_lds(vs + (tr * n_vg + gv) * 4);
+                    const float w = p[pass] * szf.x;
+                    st.wsum[c] += w;
+                    st.zsum[c] = fmaf(p[pass], szf.y, st.zsum[c]);
                     wrow[gv * GQA + h_own] = make_float2(w, w);
                 }
             }
         }
     }
     float alpha_g[GQA];
+    bool rescale = false;
 #pragma unroll
-    for (int g = 0; g < GQA; ++g) alpha_g[g] = __shfl_sync(0xffffffffu, alpha, g << kOwnShift);
+    for (int g = 0; g < GQA; ++g) {
+        alpha_g[g] = __shfl_sync(0xffffffffu, alpha, g << kOwnShift);
+        rescale |= alpha_g[g] != 1.0f;
+    }
     __syncwarp();
 
     // ---- values ----
     const int slice = lane & 15, parity = lane >> 4;
-    bool rescale = false;
-#pragma unroll
-    for (int g = 0; g < GQA; ++g) rescale |= alpha_g[g] != 1.0f;
     if (rescale) {
 #pragma unroll
         for (int g = 0; g < GQA; ++g)
@@ -366,8 +444,35 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     __syncwarp();
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int NS>
-__global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const DecodeParams p) {
+// Untangle one slice's value accumulators into its 8 channel sums
+// sum_t w_t c_t (without the zero-point term); W = sum_t w_t of its group.
+template <int VM, int VBITS>
+__device__ __forceinline__ void value_channels(const float2 o[4], float W, float out[8]) {
+    if constexpr (VM == V_BF16) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { out[2 * c] = o[c].x; out[2 * c + 1] = o[c].y; }
+    } else if constexpr (VBITS == 4) {
+        // acc = sum w (0.5 + c/256)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            out[2 * c] = fmaf(256.0f, o[c].x, -128.0f * W);
+            out[2 * c + 1] = fmaf(256.0f, o[c].y, -128.0f * W);
+        }
+    } else {
+        // acc_i = sum w (0.5 + X_i/256) with the X planes of value_pairs
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const float2 a = o[2 * b], c = o[2 * b + 1];
+            out[4 * b] = fmaf(256.0f, a.x, -128.0f * W);
+            out[4 * b + 1] = 64.0f * (a.y - a.x);
+            out[4 * b + 2] = 16.0f * (c.x - a.y);
+            out[4 * b + 3] = fmaf(16.0f, c.y, -8.0f * W) - 4.0f * (c.x - a.x);
+        }
+    }
+}
+
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int NS, int VSLOTS>
+__global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk_kernel(const DecodeParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int split = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -392,7 +497,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const Decode
     float *qs = reinterpret_cast<float *>(tail);
     float *wsm_all = qs + GQA * kHeadDim;
     float *red = wsm_all + kConsumerWarps * 16 * 8 * GQA * 2;
-    uint64_t *full = reinterpret_cast<uint64_t *>(red + kConsumerWarps * GQA * 130);
+    float *qsum_all = red + kConsumerWarps * GQA * 130;           // [4 warps][8][3][GQA]
+    uint64_t *full = reinterpret_cast<uint64_t *>(qsum_all + kConsumerWarps * 8 * 3 * GQA);
     uint64_t *empty = full + NS;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + NS);
 
@@ -424,64 +530,57 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const Decode
             issued = it + 1;
             if (it == p.skip_tile) continue;  // test hook: never arrive
             uint8_t *st = stages + static_cast<size_t>(s) * p.stage_bytes;
-            // Collect the copies, sum their bytes, arm the barrier, then issue.
-            const uint8_t *src[16];
-            uint32_t off[16], len[16];
-            int nc = 0;
+            uint64_t *bar = &full[s];
             if (it >= n_qt) {  // bf16 window rows
                 const int t0 = w_begin + (it - n_qt) * p.bf_tile;
-                const int n = min(p.bf_tile, t_end - t0);
+                const uint32_t bytes = min(p.bf_tile, t_end - t0) * kHeadDim * 2;
                 const int64_t slot = sh * p.R + (t0 - Tq);
-                src[nc] = reinterpret_cast<const uint8_t *>(p.k_res + slot * kHeadDim);
-                off[nc] = 0; len[nc++] = n * kHeadDim * 2;
-                src[nc] = reinterpret_cast<const uint8_t *>(p.v_res + slot * kHeadDim);
-                off[nc] = p.bf_off_v; len[nc++] = n * kHeadDim * 2;
+                mbar_arrive_expect_tx(bar, 2 * bytes);
+                bulk_g2s(st, p.k_res + slot * kHeadDim, bytes, bar);
+                bulk_g2s(st + p.bf_off_v, p.v_res + slot * kHeadDim, bytes, bar);
             } else if (!p.paged) {
                 const int t0 = t_begin + it * kTile;
                 const int n = min(kTile, q_end - t0);
                 const int64_t row = sh * p.cap + t0;
-                src[nc] = p.k_codes + row * KROW; off[nc] = 0; len[nc++] = n * KROW;
-                if (KM == K_TOKEN) {
-                    src[nc] = reinterpret_cast<const uint8_t *>(p.k_sz + row * ngk);
-                    off[nc] = p.off_ksz; len[nc++] = (n * ngk * 4 + 15) & ~15;
-                } else if (KM == K_CHANNEL) {
-                    src[nc] = reinterpret_cast<const uint8_t *>(
-                        p.k_sz + (sh * (p.cap / p.R) + t0 / p.R) * kHeadDim);
-                    off[nc] = p.off_ksz; len[nc++] = kHeadDim * 4;
-                }
-                src[nc] = p.v_codes + row * VROW; off[nc] = p.off_vc; len[nc++] = n * VROW;
-                if (VM == V_TOKEN) {
-                    src[nc] = reinterpret_cast<const uint8_t *>(p.v_sz + row * ngv);
-                    off[nc] = p.off_vsz; len[nc++] = (n * ngv * 4 + 15) & ~15;
-                }
+                const uint32_t kb = n * KROW, vb = n * VROW;
+                const uint32_t kzb = (KM == K_TOKEN) ? ((n * ngk * 4 + 15) & ~15)
+                                                     : (KM == K_CHANNEL ? kHeadDim * 4 : 0);
+                const uint32_t vzb = (VM == V_TOKEN) ? ((n * ngv * 4 + 15) & ~15) : 0;
+                mbar_arrive_expect_tx(bar, kb + vb + kzb + vzb);
+                bulk_g2s(st, p.k_codes + row * KROW, kb, bar);
+                bulk_g2s(st + p.off_vc, p.v_codes + row * VROW, vb, bar);
+                if (KM == K_TOKEN) bulk_g2s(st + p.off_ksz, p.k_sz + row * ngk, kzb, bar);
+                if (KM == K_CHANNEL)
+                    bulk_g2s(st + p.off_ksz, p.k_sz + (sh * (p.cap / p.R) + t0 / p.R) * kHeadDim, kzb, bar);
+                if (VM == V_TOKEN) bulk_g2s(st + p.off_vsz, p.v_sz + row * ngv, vzb, bar);
             } else {
+                // Paged (token-wise groups only): one copy of each part per page.
                 const int t0 = t_begin + it * kTile;
                 const int n = min(kTile, q_end - t0);
                 const int ps = p.page_size;
                 const int span = ps < kTile ? ps : kTile;  // tokens per copy
+                const uint32_t per_copy = span * (KROW + VROW + 4 * ngk + 4 * ngv);
+                const int32_t *bt = p.block_table + static_cast<int64_t>(seq) * p.max_pages;
+                uint32_t bytes = 0;
                 for (int tp = t0; tp < t0 + n; tp += span) {
                     const int pi = tp / ps;
-                    const int page = (pi < p.max_pages)
-                                         ? __ldg(p.block_table + static_cast<int64_t>(seq) * p.max_pages + pi)
-                                         : -1;
-                    if (page < 0 || page >= p.num_pages) {
-                        status_or(p.status, KVQ_DEV_CAPACITY);
-                        continue;
-                    }
+                    const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
+                    if (page >= 0 && page < p.num_pages) bytes += per_copy;
+                    else status_or(p.status, KVQ_DEV_CAPACITY);
+                }
+                mbar_arrive_expect_tx(bar, bytes);
+                for (int tp = t0; tp < t0 + n; tp += span) {
+                    const int pi = tp / ps;
+                    const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
+                    if (page < 0 || page >= p.num_pages) continue;
                     const int64_t row = (static_cast<int64_t>(page) * p.H + kvh) * ps + (tp % ps);
                     const uint32_t dt = tp - t0;
-                    src[nc] = p.k_codes + row * KROW; off[nc] = dt * KROW; len[nc++] = span * KROW;
-                    src[nc] = reinterpret_cast<const uint8_t *>(p.k_sz + row * ngk);
-                    off[nc] = p.off_ksz + dt * ngk * 4; len[nc++] = span * ngk * 4;
-                    src[nc] = p.v_codes + row * VROW; off[nc] = p.off_vc + dt * VROW; len[nc++] = span * VROW;
-                    src[nc] = reinterpret_cast<const uint8_t *>(p.v_sz + row * ngv);
-                    off[nc] = p.off_vsz + dt * ngv * 4; len[nc++] = span * ngv * 4;
+                    bulk_g2s(st + dt * KROW, p.k_codes + row * KROW, span * KROW, bar);
+                    bulk_g2s(st + p.off_ksz + dt * ngk * 4, p.k_sz + row * ngk, span * ngk * 4, bar);
+                    bulk_g2s(st + p.off_vc + dt * VROW, p.v_codes + row * VROW, span * VROW, bar);
+                    bulk_g2s(st + p.off_vsz + dt * ngv * 4, p.v_sz + row * ngv, span * ngv * 4, bar);
                 }
             }
-            uint32_t bytes = 0;
-            for (int c = 0; c < nc; ++c) bytes += len[c];
-            mbar_arrive_expect_tx(&full[s], bytes);
-            for (int c = 0; c < nc; ++c) bulk_g2s(st + off[c], src[c], len[c], &full[s]);
         }
         // Drain: wait for the copies of the last stages issued so none lands
         // after the CTA has gone.
@@ -545,37 +644,111 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const Decode
     named_sync(1, kConsumers);
 
     const int part = lane & 7;
-    // Query registers in the layout of the key mode (see the header comment):
-    // token-wise codes: 256 q, with qc = sum of the lane's q (zero-point term);
-    // channel-wise codes: set per block below; bf16 keys: q itself.
-    float2 qk[GQA][8];
-    float qc[GQA];
-    auto load_plain_q = [&](float scale_q) {
+    constexpr int kOwnShift = LaneMap<GQA>::kOwnShift;
+    // head held in register slot g (reduce-scatter order for GQA 4)
+    const int perm = (GQA == 4) ? (((part >> 2) & 1) << 1 | ((part >> 1) & 1)) : 0;
+    QueryRegs<GQA> Q;
+    float *qsum = qsum_all + warp * 8 * 3 * GQA;
+    // mode: 0 = token-wise codes, 1 = channel-wise codes (per-channel scales
+    // folded in from `chan_sz`), 2 = bf16 keys.
+    auto load_query = [&](int mode, const uint8_t *chan_sz) {
+        float qa_full = 0.0f, qe_full = 0.0f;
+        __syncwarp();  // this warp is done reading the previous sums
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
-            float s = 0.0f;
+            const int h = g ^ perm;
+            float x[16];
+            float qa = 0.0f, qz = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float a = qs[g * kHeadDim + part * 16 + 2 * j];
-                const float b = qs[g * kHeadDim + part * 16 + 2 * j + 1];
-                qk[g][j] = make_float2(a * scale_q, b * scale_q);
-                s += a + b;
+            for (int j = 0; j < 16; ++j) {
+                const float v = qs[h * kHeadDim + part * 16 + j];
+                qa += v;
+                if (mode == 1) {
+                    const float2 sz = half2_lds(chan_sz + (part * 16 + j) * 4);
+                    x[j] = v * sz.x;
+                    qz = fmaf(v, sz.y, qz);
+                } else {
+                    x[j] = v;
+                }
             }
-            qc[g] = s;
+            float first;
+            if (mode == 2) query_coeffs<K_BF16, 16>(x, Q.qk[g], first);
+            else query_coeffs<KM == K_BF16 ? K_TOKEN : KM, KBITS == 16 ? 4 : KBITS>(x, Q.qk[g], first);
+            if ((lane >> 3) == 0) {
+                qsum[(part * 3 + 0) * GQA + g] = qa;
+                qsum[(part * 3 + 1) * GQA + g] = first;
+                qsum[(part * 3 + 2) * GQA + g] = (mode == 1) ? fmaf(-128.0f, first, qz) : 0.0f;
+            }
         }
+        // Whole-head sums of the lane's own head (natural head order), for the
+        // scale applied after the reduce-scatter when a group spans the head.
+        // (the sum of the coefficients: all q for INT4, q0 + q3/16 per byte for INT2)
+        for (int d = 0; d < kHeadDim; ++d) {
+            const float v = qs[(part >> kOwnShift) * kHeadDim + d];
+            qa_full += v;
+            if (KBITS != 2) qe_full += v;
+            else if (d % 4 == 0) qe_full += v;
+            else if (d % 4 == 3) qe_full += 0.0625f * v;
+        }
+        Q.qa_own = qa_full;
+        Q.qe_own = qe_full;
+        __syncwarp();
     };
-    load_plain_q(KM == K_TOKEN ? 256.0f : 1.0f);
+    if constexpr (KM != K_CHANNEL) load_query(KM == K_BF16 ? 2 : 0, nullptr);
 
-    WarpState<GQA> st;
+    WarpState<GQA, VSLOTS> st;
     st.m_own = -INFINITY;
     st.l_own = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) st.corr[c] = 0.0f;
+    for (int c = 0; c < VSLOTS; ++c) { st.wsum[c] = 0.0f; st.zsum[c] = 0.0f; }
 #pragma unroll
     for (int g = 0; g < GQA; ++g)
 #pragma unroll
         for (int c = 0; c < 4; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
     float *wsm = wsm_all + warp * 16 * 8 * GQA * 2;
+
+    // Turn the value accumulators of quantized tiles into plain channel sums
+    // (adding the zero-point terms), once: before the first bf16 window tile
+    // or at the end. Half-warp 1 adds no group terms, so the halves still sum.
+    bool folded = false;
+    auto fold_values = [&]() {
+        constexpr int kPH = LaneMap<GQA>::kPerHead;
+        float wsum[VSLOTS], zsum[VSLOTS];
+#pragma unroll
+        for (int c = 0; c < VSLOTS; ++c) {
+            wsum[c] = st.wsum[c];
+            wsum[c] += __shfl_xor_sync(0xffffffffu, wsum[c], 8);
+            wsum[c] += __shfl_xor_sync(0xffffffffu, wsum[c], 16);
+            zsum[c] = st.zsum[c];
+            zsum[c] += __shfl_xor_sync(0xffffffffu, zsum[c], 8);
+            zsum[c] += __shfl_xor_sync(0xffffffffu, zsum[c], 16);
+            st.wsum[c] = 0.0f;
+            st.zsum[c] = 0.0f;
+        }
+        const int sl = lane & 15;
+        const int gv_lane = (8 * sl) / p.group_v;
+        const bool first_half = lane < 16;
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) {
+            // group gv of head g: lane (g << kOwnShift) + gv % kPH, slot gv / kPH
+            float Wg = 0.0f, Zg = 0.0f;
+#pragma unroll
+            for (int c = 0; c < VSLOTS; ++c) {
+#pragma unroll
+                for (int r = 0; r < kPH; ++r) {
+                    const float wv = __shfl_sync(0xffffffffu, wsum[c], (g << kOwnShift) + r);
+                    const float zv = __shfl_sync(0xffffffffu, zsum[c], (g << kOwnShift) + r);
+                    if (gv_lane == r + c * kPH) { Wg = wv; Zg = zv; }
+                }
+            }
+            if (!first_half) { Wg = 0.0f; Zg = 0.0f; }
+            float ch[8];
+            value_channels<VM, VBITS>(st.o[g], Wg, ch);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) st.o[g][c] = make_float2(ch[2 * c] + Zg, ch[2 * c + 1] + Zg);
+        }
+        folded = true;
+    };
 
     int cur_block = -1;
     for (int it = 0; it < n_tiles; ++it) {
@@ -589,40 +762,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const Decode
                 const int blk = t0 / p.R;
                 if (blk != cur_block) {  // fold this block's channel scales into q
                     cur_block = blk;
-#pragma unroll
-                    for (int g = 0; g < GQA; ++g) {
-                        float c = 0.0f;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int ch = part * 16 + 2 * j;
-                            const float2 s0 = half2_lds(sb + p.off_ksz + ch * 4);
-                            const float2 s1 = half2_lds(sb + p.off_ksz + (ch + 1) * 4);
-                            const float qa = qs[g * kHeadDim + ch], qb = qs[g * kHeadDim + ch + 1];
-                            qk[g][j] = make_float2(256.0f * qa * s0.x, 256.0f * qb * s1.x);
-                            c = fmaf(qa, fmaf(-128.0f, s0.x, s0.y), c);
-                            c = fmaf(qb, fmaf(-128.0f, s1.x, s1.y), c);
-                        }
-                        qc[g] = c;
-                    }
+                    load_query(1, sb + p.off_ksz);
                 }
             }
-            process_tile<GQA, KM, VM, KBITS, VBITS, kTile / kConsumerWarps>(
-                sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, n, p.group_k, p.group_v, qk, qc,
+            process_tile<GQA, KM, VM, KBITS, VBITS, kTile / kConsumerWarps, VSLOTS>(
+                sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, n, p.group_k, p.group_v, Q, qsum,
                 st, wsm, warp, lane);
         } else {
             if (it == n_qt && KM != K_BF16) {
-                load_plain_q(1.0f);
-#pragma unroll
-                for (int g = 0; g < GQA; ++g) qc[g] = 0.0f;
+                load_query(2, nullptr);
+                if (VM == V_TOKEN && !folded) fold_values();
             }
             const int t0 = w_begin + (it - n_qt) * p.bf_tile;
             const int n = min(p.bf_tile, t_end - t0);
             if constexpr (KM == K_BF16) {
-                process_tile<GQA, K_BF16, V_BF16, 16, 16, kTile / kConsumerWarps>(
-                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, qk, qc, st, wsm, warp, lane);
+                process_tile<GQA, K_BF16, V_BF16, 16, 16, kTile / kConsumerWarps, VSLOTS>(
+                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, Q, qsum, st, wsm, warp, lane);
             } else {
-                process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps>(
-                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, qk, qc, st, wsm, warp, lane);
+                process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, VSLOTS>(
+                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, Q, qsum, st, wsm, warp, lane);
             }
         }
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -630,32 +788,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const Decode
     const bool aborted = *abort_flag != 0;
 
     // ---- merge the four warps ----
-    constexpr int kPerHead = LaneMap<GQA>::kPerHead;
-    constexpr int kOwnShift = LaneMap<GQA>::kOwnShift;
     float l_own = st.l_own;
     l_own += __shfl_xor_sync(0xffffffffu, l_own, 8);
     l_own += __shfl_xor_sync(0xffffffffu, l_own, 16);
-    float corr[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        corr[c] = st.corr[c];
-        corr[c] += __shfl_xor_sync(0xffffffffu, corr[c], 8);
-        corr[c] += __shfl_xor_sync(0xffffffffu, corr[c], 16);
-    }
+    if (VM == V_TOKEN && !folded) fold_values();
     const int slice = lane & 15;
-    const int gv_lane = (VM == V_BF16) ? 0 : (8 * slice) / p.group_v;
 #pragma unroll
     for (int g = 0; g < GQA; ++g) {
-        // group gv of head g lives in lane (g << kOwnShift) + gv % kPerHead, slot gv / kPerHead
-        float zg = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-#pragma unroll
-            for (int r = 0; r < kPerHead; ++r) {
-                const float z = __shfl_sync(0xffffffffu, corr[c], (g << kOwnShift) + r);
-                if (VM == V_TOKEN && gv_lane == r + c * kPerHead) zg = z;
-            }
-        }
         const float mg = __shfl_sync(0xffffffffu, st.m_own, g << kOwnShift);
         const float lg = __shfl_sync(0xffffffffu, l_own, g << kOwnShift);
 #pragma unroll
@@ -664,8 +803,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_splitk_kernel(const Decode
             v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
             v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
             if (lane < 16) {
-                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c] = v.x + zg;
-                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c + 1] = v.y + zg;
+                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c] = v.x;
+                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c + 1] = v.y;
             }
         }
         if (lane == 0) {
@@ -751,20 +890,30 @@ StageLayout stage_layout(const kvq_cache_desc &d) {
 
 template <int GQA>
 size_t tail_bytes(int NS) {
-    return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * 16 * 8 * GQA * 2 + kConsumerWarps * GQA * 130) +
+    return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * 16 * 8 * GQA * 2 +
+                            kConsumerWarps * GQA * 130 + kConsumerWarps * 8 * 3 * GQA) +
            sizeof(uint64_t) * 2 * NS + 16;
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS>
-kvq_status launch_variant(const DecodeParams &p, dim3 grid, cudaStream_t stream) {
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int VSLOTS>
+kvq_status launch_variant_slots(const DecodeParams &p, dim3 grid, cudaStream_t stream) {
     constexpr int NS = (KM == K_BF16) ? 3 : 4;
     const size_t smem = static_cast<size_t>(NS) * p.stage_bytes + tail_bytes<GQA>(NS);
-    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, NS>;
+    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, NS, VSLOTS>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return KVQ_ERR_CUDA;
     kern<<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+// One value-group slot per lane when a head's groups fit one per lane.
+template <int GQA, int KM, int VM, int KBITS, int VBITS>
+kvq_status launch_variant(const DecodeParams &p, dim3 grid, cudaStream_t stream) {
+    const int n_vg = (VM == V_BF16) ? 1 : kHeadDim / p.group_v;
+    if (n_vg <= LaneMap<GQA>::kPerHead)
+        return launch_variant_slots<GQA, KM, VM, KBITS, VBITS, 1>(p, grid, stream);
+    return launch_variant_slots<GQA, KM, VM, KBITS, VBITS, 4>(p, grid, stream);
 }
 
 template <int GQA>
