@@ -76,7 +76,8 @@ kvq_status validate_decode(const kvq_cache_desc *d, const void *q, int q_dtype, 
                            const int32_t *seq_lens, int num_seqs, int max_seq_len) {
     kvq_status s = validate_desc(d, true);
     if (s != KVQ_OK) return s;
-    if (q == nullptr || !dtype_ok(q_dtype) || seq_lens == nullptr) return KVQ_ERR_INVALID_ARG;
+    if (q == nullptr || !aligned16(q) || !dtype_ok(q_dtype) || seq_lens == nullptr)
+        return KVQ_ERR_INVALID_ARG;
     if (num_seqs <= 0 || max_seq_len < 0 || num_q_heads <= 0) return KVQ_ERR_INVALID_ARG;
     if (num_q_heads % d->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
     const int gqa = num_q_heads / d->num_kv_heads;

@@ -9,27 +9,33 @@
 // so no dequantized element is ever formed. Dual-QK (Abstract): queries take
 // the keys' orthogonal transform, so q~ . k~ = q . k.
 //
-// CTA = one (split, KV head, sequence): 4 consumer warps and 1 producer warp.
-// The producer's elected lane stages each tile (K codes, K scale/zero, V
-// codes, V scale/zero; or bf16 rows of the recent-token window) into a
-// shared-memory ring with 1-D bulk copies (TMA engine, mbarrier complete_tx),
-// resolving page-table indirection per page.
+// Work items are (sequence, KV head, split of `chunk` tokens). The kernel is
+// persistent: each CTA (4 consumer warps + 1 producer warp) runs until a
+// global item counter is exhausted. The producer's elected lane claims items
+// and streams every item's tiles (K codes, K scale/zero, V codes, V scale/zero;
+// bf16 rows for the recent-token window; the item's query rows with its first
+// tile) into a shared-memory ring with 1-D bulk copies (TMA engine, mbarrier
+// complete_tx), resolving page tables per page. Each stage carries a small
+// header, so the consumers follow the stream without further coordination and
+// the ring never drains between items.
 //
 // Inner loop. The path is bound by the FP32 FMA pipe, not by the tensor
 // cores: every cached element meets GQA query heads, one multiply-add each.
-// So the loop is built to spend as few issue slots as possible besides those
-// multiply-adds:
+// So the loop spends as few issue slots as possible besides those:
 //   * multiply-adds are packed f32x2 FMAs (two lanes of work per issue);
-//   * a 4-bit or 2-bit code c becomes the float 0.5 + c/256 with ONE byte
-//     permute (the code lands in mantissa bits 16..19 of 0.5); the constant
-//     0.5 is folded into the per-group zero-point terms, exactly;
+//   * codes become floats 0.5 + X/256 with ONE byte permute per code, from
+//     byte planes kept below 128; the query is transformed once per item so
+//     that its dot product with these floats is the one with the codes, and
+//     the value sums are untangled once per item;
 //   * each consumer warp owns a quarter of every tile with its own
 //     online-softmax state, so tiles need no cross-warp synchronisation;
 //   * scores: 8 lanes per token, 16 channels per lane, all GQA heads at once,
-//     a reduce-scatter over the 8 lanes leaves one head's score per lane pair;
+//     a select-free reduce-scatter over the 8 lanes (heads held in a per-lane
+//     permuted order) leaves one head's score per lane pair;
 //   * values: 16 lanes cover the 128 channels (8 each) for all GQA heads; the
-//     two half-warps take alternate tokens.
-// The four warps' states are merged once per split; the merge kernel combines
+//     two half-warps take alternate tokens;
+//   * common group sizes are compile-time constants.
+// The four warps' states are merged once per item; the merge kernel combines
 // the splits.
 #include <algorithm>
 
@@ -53,6 +59,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum KMode { K_TOKEN = 0, K_CHANNEL = 1, K_BF16 = 2 };
 enum VMode { V_TOKEN = 0, V_BF16 = 2 };
 
+// Stage header flags.
+constexpr int kFirst = 1, kLast = 2, kWindow = 4, kDone = 8;
+
+struct TileHdr {
+    int seq, kvh, split, t0;
+    int n, flags, pad0, pad1;
+};
+
 struct DecodeParams {
     const uint8_t *k_codes, *v_codes;  // packed codes, or bf16 rows (bits 16)
     const __half2 *k_sz, *v_sz;
@@ -62,18 +76,19 @@ struct DecodeParams {
     const void *q;
     float *o_part;  // [S][Hq][n_split][D]
     float2 *ml;     // [S][Hq][n_split]
+    int *counter;   // item counter, zeroed before the launch
     int32_t *status;
-    int H, Hq;
-    int group_k, group_v;
+    int S, H, Hq;
+    int gk_log2, gv_log2;  // log2 of the group sizes (token-wise groups)
     int hb;
     float hscale;   // fp32(1/sqrt(hb))
     float qscale;   // softmax_scale * log2(e)
     int R;
     int paged, page_size, max_pages, num_pages, cap;
     int chunk, n_split, max_seq_len;
-    int q_dtype;
+    int q_dtype, q_bytes;  // element type and bytes of q
     // shared-memory stage layout (bytes)
-    int stage_bytes, off_ksz, off_vc, off_vsz;
+    int stage_bytes, off_ksz, off_vc, off_vsz, off_q, off_hdr;
     int bf_tile, bf_off_v;  // bf16 tiles: tokens per tile, offset of the V rows
     int64_t timeout_ns;
     int skip_tile;
@@ -106,18 +121,10 @@ __device__ __forceinline__ void ffma2(float2 &d, float2 a, float2 b) {
 // Plain typed loads: the compiler sees their dependence on the stores and on
 // the mbarrier waits (asm with a memory clobber) and keeps them in order; the
 // pointers all derive from the kernel's shared array.
-__device__ __forceinline__ uint32_t lds32(const void *p) {
-    return *static_cast<const uint32_t *>(p);
-}
-__device__ __forceinline__ uint32_t lds16(const void *p) {
-    return *static_cast<const uint16_t *>(p);
-}
-__device__ __forceinline__ uint2 lds64(const void *p) {
-    return *static_cast<const uint2 *>(p);
-}
-__device__ __forceinline__ uint4 lds128(const void *p) {
-    return *static_cast<const uint4 *>(p);
-}
+__device__ __forceinline__ uint32_t lds32(const void *p) { return *static_cast<const uint32_t *>(p); }
+__device__ __forceinline__ uint32_t lds16(const void *p) { return *static_cast<const uint16_t *>(p); }
+__device__ __forceinline__ uint2 lds64(const void *p) { return *static_cast<const uint2 *>(p); }
+__device__ __forceinline__ uint4 lds128(const void *p) { return *static_cast<const uint4 *>(p); }
 __device__ __forceinline__ float2 half2_lds(const void *p) {
     const uint32_t u = lds32(p);
     return __half22float2(*reinterpret_cast<const __half2 *>(&u));
@@ -130,9 +137,9 @@ __device__ __forceinline__ float2 half2_lds(const void *p) {
 // high nibble planes; INT2 codes use the planes
 //   X0 = c0, X1 = c0 + 4c1, X2 = c0 + 4c1 + 16c2, X3 = c1 + 4c2 + 16c3
 // (three masks and one shift of the packed word), all < 64. The floats are
-// linear in the codes; the query is transformed once per CTA so that its dot
+// linear in the codes; the query is transformed once per item so that its dot
 // product with them is the dot product with the codes (query_coeffs), and the
-// value accumulators are untangled once per split (value_channels).
+// value accumulators are untangled once per item (value_channels).
 __device__ __forceinline__ float byte_f(uint32_t b, int k) {
     return __uint_as_float(__byte_perm(b, 0x3F000000u, 0x7054u | (static_cast<uint32_t>(k) << 8)));
 }
@@ -225,6 +232,33 @@ __device__ __forceinline__ void query_coeffs(const float x[16], float2 qk[8], fl
     }
 }
 
+// Untangle one slice's value accumulators into its 8 channel sums
+// sum_t w_t c_t (without the zero-point term); W = sum_t w_t of its group.
+template <int VM, int VBITS>
+__device__ __forceinline__ void value_channels(const float2 o[4], float W, float out[8]) {
+    if constexpr (VM == V_BF16) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { out[2 * c] = o[c].x; out[2 * c + 1] = o[c].y; }
+    } else if constexpr (VBITS == 4) {
+        // acc = sum w (0.5 + c/256)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            out[2 * c] = fmaf(256.0f, o[c].x, -128.0f * W);
+            out[2 * c + 1] = fmaf(256.0f, o[c].y, -128.0f * W);
+        }
+    } else {
+        // acc_i = sum w (0.5 + X_i/256) with the X planes of value_pairs
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const float2 a = o[2 * b], c = o[2 * b + 1];
+            out[4 * b] = fmaf(256.0f, a.x, -128.0f * W);
+            out[4 * b + 1] = 64.0f * (a.y - a.x);
+            out[4 * b + 2] = 16.0f * (c.x - a.y);
+            out[4 * b + 3] = fmaf(16.0f, c.y, -8.0f * W) - 4.0f * (c.x - a.x);
+        }
+    }
+}
+
 template <int GQA>
 __device__ __forceinline__ void load_sums(const float *p, float v[GQA]) {
     if constexpr (GQA == 4) {
@@ -233,12 +267,31 @@ __device__ __forceinline__ void load_sums(const float *p, float v[GQA]) {
         v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
     } else {
 #pragma unroll
-        for (int g = 0; g < GQA; ++g) v[g] = __uint_as_float(lds32(p + g));
+        for (int g = 0; g < GQA; ++g) v[g] = p[g];
     }
 }
 
-// Per-warp decode state. VSLOTS: value groups a lane accumulates terms for
-// (1 when each head's groups fit one per lane, else 4).
+template <int GQA>
+struct LaneMap {
+    static constexpr int kPerHead = 8 / GQA;  // lanes of a token per head
+    static constexpr int kOwnShift = (GQA == 4) ? 1 : (GQA == 2 ? 2 : 3);
+};
+
+// Group-size geometry: compile-time when GK/GV > 0, else from the params.
+template <int GK, int GV, int GQA>
+struct Geo {
+    int gk_log2, gv_log2;
+    __device__ __forceinline__ int ngk() const { return GK ? kHeadDim / GK : kHeadDim >> gk_log2; }
+    __device__ __forceinline__ int nvg() const { return GV ? kHeadDim / GV : kHeadDim >> gv_log2; }
+    __device__ __forceinline__ int kgroup(int part) const { return GK ? (part * 16) / GK : (part * 16) >> gk_log2; }
+    __device__ __forceinline__ int vgroup(int slice) const { return GV ? (slice * 8) / GV : (slice * 8) >> gv_log2; }
+    __device__ __forceinline__ bool k_whole() const { return GK ? GK == kHeadDim : gk_log2 == 7; }
+    // value-group slots per owner lane
+    static constexpr int kVSlots =
+        GV ? ((kHeadDim / GV + LaneMap<GQA>::kPerHead - 1) / LaneMap<GQA>::kPerHead) : 4;
+};
+
+// Per-warp decode state of the current item.
 template <int GQA, int VSLOTS>
 struct WarpState {
     float m_own;           // running max (log2 domain) used for this lane's head
@@ -248,20 +301,14 @@ struct WarpState {
     float2 o[GQA][4];      // value accumulators: 8 channels (4 pairs) x GQA heads
 };
 
-template <int GQA>
-struct LaneMap {
-    static constexpr int kPerHead = 8 / GQA;  // lanes of a token per head
-    static constexpr int kOwnShift = (GQA == 4) ? 1 : (GQA == 2 ? 2 : 3);
-};
-
 // Scores are kept in log2 units; a new tile maximum only moves the reference
 // when it exceeds the old one by more than this (weights then stay <= 2^8).
 constexpr float kRescaleSlack = 8.0f;
 
 // Per-lane query data for the key pass. Per-lane sums the inner loop needs
 // once per pass live in shared memory (qsum, [8 parts][3][GQA] floats, head
-// order as in qk): [0] sum of q, [1] sum over first-of-byte channels,
-// [2] channel-wise groups: sum q z - 128 sum first-of-byte q s.
+// order as in qk): [0] sum of q, [1] sum of the code-byte coefficients,
+// [2] channel-wise groups: sum q z - 128 * coefficient sum of q s.
 template <int GQA>
 struct QueryRegs {
     float2 qk[GQA][8];     // coefficients, head order permuted for the reduce-scatter
@@ -270,10 +317,10 @@ struct QueryRegs {
 
 // One tile: rows at kc / ks / vc / vs (shared memory), `n` valid tokens, TPW
 // tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)).
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW, int VSLOTS>
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW, int GK, int GV, int VSLOTS>
 __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
                                              const uint8_t *vc, const uint8_t *vs, int n,
-                                             int group_k, int group_v, const QueryRegs<GQA> &Q,
+                                             const Geo<GK, GV, GQA> geo, const QueryRegs<GQA> &Q,
                                              const float *qsum, WarpState<GQA, VSLOTS> &st,
                                              float *wsm, int warp, int lane) {
     constexpr int KROW = KRow<KM, KBITS>::bytes;
@@ -284,9 +331,9 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     const int i = lane >> 3, part = lane & 7;
     const int h_own = part >> kOwnShift;
     const int r_own = part & (kPerHead - 1);  // rank of this lane among its head's lanes
-    const int n_vg = (VM == V_BF16) ? 1 : kHeadDim / group_v;
-    const int ngk = (KM == K_TOKEN) ? kHeadDim / group_k : 0;
-    const bool post_scale = (KM == K_TOKEN) && group_k == kHeadDim;
+    const int n_vg = (VM == V_BF16) ? 1 : geo.nvg();
+    const int ngk = (KM == K_TOKEN) ? geo.ngk() : 0;
+    const bool post_scale = (KM == K_TOKEN) && geo.k_whole();
     const int t_warp = warp * TPW;
 
     // ---- scores ----
@@ -307,7 +354,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
         }
         float2 szf = make_float2(0.0f, 0.0f);
         if constexpr (KM == K_TOKEN) {
-            szf = half2_lds(ks + (tr * ngk + (post_scale ? 0 : (part * 16) / group_k)) * 4);
+            szf = half2_lds(ks + (tr * ngk + (post_scale ? 0 : geo.kgroup(part))) * 4);
             if (!post_scale) {
                 float qa[GQA], qe[GQA];
                 load_sums<GQA>(qsum + (part * 3 + 0) * GQA, qa);
@@ -341,7 +388,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
                 if (h_own == g) val = acc[g];
         }
         if constexpr (KM == K_TOKEN) {
-            if (post_scale) val = fmaf(szf.x, val, fmaf(szf.y, Q.qa_own, -128.0f * szf.x * Q.qe_own));
+            if (post_scale) val = fmaf(szf.x, fmaf(-128.0f, Q.qe_own, val), szf.y * Q.qa_own);
         }
         sc[pass] = tt < n ? val : -INFINITY;
     }
@@ -415,7 +462,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
                 st.o[g][c].y *= alpha_g[g];
             }
     }
-    const int gv_lane = (VM == V_BF16) ? 0 : (8 * slice) / group_v;
+    const int gv_lane = (VM == V_BF16) ? 0 : geo.vgroup(slice);
 #pragma unroll
     for (int k = 0; k < TPW / 2; ++k) {
         const int j = 2 * k + parity;
@@ -444,63 +491,41 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     __syncwarp();
 }
 
-// Untangle one slice's value accumulators into its 8 channel sums
-// sum_t w_t c_t (without the zero-point term); W = sum_t w_t of its group.
-template <int VM, int VBITS>
-__device__ __forceinline__ void value_channels(const float2 o[4], float W, float out[8]) {
-    if constexpr (VM == V_BF16) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) { out[2 * c] = o[c].x; out[2 * c + 1] = o[c].y; }
-    } else if constexpr (VBITS == 4) {
-        // acc = sum w (0.5 + c/256)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            out[2 * c] = fmaf(256.0f, o[c].x, -128.0f * W);
-            out[2 * c + 1] = fmaf(256.0f, o[c].y, -128.0f * W);
-        }
-    } else {
-        // acc_i = sum w (0.5 + X_i/256) with the X planes of value_pairs
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            const float2 a = o[2 * b], c = o[2 * b + 1];
-            out[4 * b] = fmaf(256.0f, a.x, -128.0f * W);
-            out[4 * b + 1] = 64.0f * (a.y - a.x);
-            out[4 * b + 2] = 16.0f * (c.x - a.y);
-            out[4 * b + 3] = fmaf(16.0f, c.y, -8.0f * W) - 4.0f * (c.x - a.x);
-        }
+// Decode an item index into (sequence, KV head, split): items are numbered
+// sequence-major, pref[s] = first item of sequence s.
+__device__ __forceinline__ void item_coords(const int *pref, int S, int H, int item, int &seq,
+                                            int &kvh, int &split) {
+    int lo = 0, hi = S;  // last s with pref[s] <= item
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pref[mid] <= item) lo = mid; else hi = mid;
     }
+    seq = lo;
+    const int r = item - pref[lo];
+    split = r / H;
+    kvh = r - split * H;
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int NS, int VSLOTS>
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int NS, int GK, int GV>
 __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk_kernel(const DecodeParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int split = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+    using G = Geo<GK, GV, GQA>;
+    constexpr int VSLOTS = G::kVSlots;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    int T = __ldg(p.seq_lens + seq);
-    if (T > p.max_seq_len) {
-        if (tid == 0 && split == 0 && kvh == 0) status_or(p.status, KVQ_DEV_SEQLEN);
-        T = p.max_seq_len;
-    }
-    const int t_begin = split * p.chunk;
-    if (t_begin >= T) return;
-    const int t_end = min(T, t_begin + p.chunk);
-    const int Tq = quantized_len(T, p.R);
-    const int q_end = min(t_end, Tq);                // quantized tokens [t_begin, q_end)
-    const int n_qt = q_end > t_begin ? (q_end - t_begin + kTile - 1) / kTile : 0;
-    const int w_begin = max(t_begin, Tq);            // bf16 window tokens [w_begin, t_end)
-    const int n_wt = t_end > w_begin ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
-    const int n_tiles = n_qt + n_wt;
+    const G geo{p.gk_log2, p.gv_log2};
 
     uint8_t *stages = smem;
     uint8_t *tail = smem + static_cast<size_t>(NS) * p.stage_bytes;
-    float *qs = reinterpret_cast<float *>(tail);
-    float *wsm_all = qs + GQA * kHeadDim;
-    float *red = wsm_all + kConsumerWarps * 16 * 8 * GQA * 2;
-    float *qsum_all = red + kConsumerWarps * GQA * 130;           // [4 warps][8][3][GQA]
-    uint64_t *full = reinterpret_cast<uint64_t *>(qsum_all + kConsumerWarps * 8 * 3 * GQA);
+    float *qs = reinterpret_cast<float *>(tail);                    // [GQA][128]
+    float *wsm_all = qs + GQA * kHeadDim;                            // [4][16][8][GQA][2]
+    float *red = wsm_all + kConsumerWarps * 16 * 8 * GQA * 2;        // [4][GQA][130]
+    float *qsum_all = red + kConsumerWarps * GQA * 130;              // [4][8][3][GQA]
+    float *qhead = qsum_all + kConsumerWarps * 8 * 3 * GQA;          // [2][GQA]
+    uint64_t *full = reinterpret_cast<uint64_t *>(qhead + 2 * GQA + 2);
     uint64_t *empty = full + NS;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + NS);
+    int *abort_word = reinterpret_cast<int *>(empty + NS);
+    volatile int *abort_flag = abort_word;
+    int *pref = abort_word + 4;  // [S + 1]
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -512,81 +537,141 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
     }
     __syncthreads();
 
-    const int64_t sh = static_cast<int64_t>(seq) * p.H + kvh;
-
     if (warp == kConsumerWarps) {
         // ------------------------- producer -------------------------
+        // Item prefix over sequences: sequence s has H * ceil(T_s / chunk) items.
+        int carry = 0;
+        for (int base = 0; base < p.S; base += 32) {
+            const int s = base + lane;
+            int cnt = 0;
+            if (s < p.S) {
+                int T = __ldg(p.seq_lens + s);
+                if (T > p.max_seq_len) {
+                    if (blockIdx.x == 0) status_or(p.status, KVQ_DEV_SEQLEN);
+                    T = p.max_seq_len;
+                }
+                cnt = T > 0 ? p.H * ((T + p.chunk - 1) / p.chunk) : 0;
+            }
+            int incl = cnt;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, m);
+                if (lane >= m) incl += o;
+            }
+            if (s < p.S) pref[s] = carry + incl - cnt;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) pref[p.S] = carry;
+        __syncwarp();
         if (lane != 0) return;
+        const int n_items = carry;
+
         constexpr int KROW = KRow<KM, KBITS>::bytes;
         constexpr int VROW = VRow<VM, VBITS>::bytes;
-        const int ngk = (KM == K_TOKEN) ? kHeadDim / p.group_k : 0;
-        const int ngv = (VM == V_TOKEN) ? kHeadDim / p.group_v : 0;
-        int issued = 0;
-        for (int it = 0; it < n_tiles; ++it) {
-            const int s = it % NS, r = it / NS;
-            if (r > 0 &&
-                !mbar_wait_bounded(&empty[s], (r - 1) & 1, p.timeout_ns, p.status, abort_flag))
-                break;
-            issued = it + 1;
-            if (it == p.skip_tile) continue;  // test hook: never arrive
-            uint8_t *st = stages + static_cast<size_t>(s) * p.stage_bytes;
-            uint64_t *bar = &full[s];
-            if (it >= n_qt) {  // bf16 window rows
-                const int t0 = w_begin + (it - n_qt) * p.bf_tile;
-                const uint32_t bytes = min(p.bf_tile, t_end - t0) * kHeadDim * 2;
-                const int64_t slot = sh * p.R + (t0 - Tq);
-                mbar_arrive_expect_tx(bar, 2 * bytes);
-                bulk_g2s(st, p.k_res + slot * kHeadDim, bytes, bar);
-                bulk_g2s(st + p.bf_off_v, p.v_res + slot * kHeadDim, bytes, bar);
-            } else if (!p.paged) {
-                const int t0 = t_begin + it * kTile;
-                const int n = min(kTile, q_end - t0);
-                const int64_t row = sh * p.cap + t0;
-                const uint32_t kb = n * KROW, vb = n * VROW;
-                const uint32_t kzb = (KM == K_TOKEN) ? ((n * ngk * 4 + 15) & ~15)
-                                                     : (KM == K_CHANNEL ? kHeadDim * 4 : 0);
-                const uint32_t vzb = (VM == V_TOKEN) ? ((n * ngv * 4 + 15) & ~15) : 0;
-                mbar_arrive_expect_tx(bar, kb + vb + kzb + vzb);
-                bulk_g2s(st, p.k_codes + row * KROW, kb, bar);
-                bulk_g2s(st + p.off_vc, p.v_codes + row * VROW, vb, bar);
-                if (KM == K_TOKEN) bulk_g2s(st + p.off_ksz, p.k_sz + row * ngk, kzb, bar);
-                if (KM == K_CHANNEL)
-                    bulk_g2s(st + p.off_ksz, p.k_sz + (sh * (p.cap / p.R) + t0 / p.R) * kHeadDim, kzb, bar);
-                if (VM == V_TOKEN) bulk_g2s(st + p.off_vsz, p.v_sz + row * ngv, vzb, bar);
-            } else {
-                // Paged (token-wise groups only): one copy of each part per page.
-                const int t0 = t_begin + it * kTile;
-                const int n = min(kTile, q_end - t0);
-                const int ps = p.page_size;
-                const int span = ps < kTile ? ps : kTile;  // tokens per copy
-                const uint32_t per_copy = span * (KROW + VROW + 4 * ngk + 4 * ngv);
-                const int32_t *bt = p.block_table + static_cast<int64_t>(seq) * p.max_pages;
-                uint32_t bytes = 0;
-                for (int tp = t0; tp < t0 + n; tp += span) {
-                    const int pi = tp / ps;
-                    const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
-                    if (page >= 0 && page < p.num_pages) bytes += per_copy;
-                    else status_or(p.status, KVQ_DEV_CAPACITY);
+        const int ngk = (KM == K_TOKEN) ? geo.ngk() : 0;
+        const int ngv = (VM == V_TOKEN) ? geo.nvg() : 0;
+        int it = 0;  // tile counter of this CTA (stage it % NS, round it / NS)
+        bool stop = false;
+        while (!stop) {
+            const int item = atomicAdd(p.counter, 1);
+            int seq = 0, kvh = 0, split = 0;
+            int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0;
+            if (item < n_items) {
+                item_coords(pref, p.S, p.H, item, seq, kvh, split);
+                const int T = min(__ldg(p.seq_lens + seq), p.max_seq_len);
+                t_begin = split * p.chunk;
+                t_end = min(T, t_begin + p.chunk);
+                Tq = quantized_len(T, p.R);
+                q_end = min(t_end, Tq);
+                n_qt = q_end > t_begin ? (q_end - t_begin + kTile - 1) / kTile : 0;
+                w_begin = max(t_begin, Tq);
+                n_wt = t_end > w_begin ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
+            }
+            const int n_tiles = (item < n_items) ? n_qt + n_wt : 1;  // 1 = the done marker
+            const int64_t sh = static_cast<int64_t>(seq) * p.H + kvh;
+            for (int ti = 0; ti < n_tiles; ++ti, ++it) {
+                const int s = it % NS, r = it / NS;
+                if (r > 0 &&
+                    !mbar_wait_bounded(&empty[s], (r - 1) & 1, p.timeout_ns, p.status, abort_flag)) {
+                    stop = true;
+                    break;
                 }
-                mbar_arrive_expect_tx(bar, bytes);
-                for (int tp = t0; tp < t0 + n; tp += span) {
-                    const int pi = tp / ps;
-                    const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
-                    if (page < 0 || page >= p.num_pages) continue;
-                    const int64_t row = (static_cast<int64_t>(page) * p.H + kvh) * ps + (tp % ps);
-                    const uint32_t dt = tp - t0;
-                    bulk_g2s(st + dt * KROW, p.k_codes + row * KROW, span * KROW, bar);
-                    bulk_g2s(st + p.off_ksz + dt * ngk * 4, p.k_sz + row * ngk, span * ngk * 4, bar);
-                    bulk_g2s(st + p.off_vc + dt * VROW, p.v_codes + row * VROW, span * VROW, bar);
-                    bulk_g2s(st + p.off_vsz + dt * ngv * 4, p.v_sz + row * ngv, span * ngv * 4, bar);
+                uint8_t *st = stages + static_cast<size_t>(s) * p.stage_bytes;
+                uint64_t *bar = &full[s];
+                TileHdr *hdr = reinterpret_cast<TileHdr *>(st + p.off_hdr);
+                if (item >= n_items) {  // no work left: tell the consumers
+                    hdr->flags = kDone;
+                    mbar_arrive(bar);
+                    stop = true;
+                    ++it;
+                    break;
                 }
+                if (it == p.skip_tile) continue;  // test hook: never arrive
+                const bool window = ti >= n_qt;
+                const int t0 = window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * kTile;
+                const int n = window ? min(p.bf_tile, t_end - t0) : min(kTile, q_end - t0);
+                hdr->seq = seq;
+                hdr->kvh = kvh;
+                hdr->split = split;
+                hdr->t0 = t0;
+                hdr->n = n;
+                hdr->flags = (ti == 0 ? kFirst : 0) | (ti == n_tiles - 1 ? kLast : 0) | (window ? kWindow : 0);
+                const uint32_t qb = (ti == 0) ? GQA * kHeadDim * p.q_bytes : 0;
+                const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
+                                      ((static_cast<int64_t>(seq) * p.Hq + kvh * GQA) * kHeadDim) * p.q_bytes;
+                if (window) {
+                    const uint32_t bytes = n * kHeadDim * 2;
+                    const int64_t slot = sh * p.R + (t0 - Tq);
+                    mbar_arrive_expect_tx(bar, 2 * bytes + qb);
+                    bulk_g2s(st, p.k_res + slot * kHeadDim, bytes, bar);
+                    bulk_g2s(st + p.bf_off_v, p.v_res + slot * kHeadDim, bytes, bar);
+                } else if (!p.paged) {
+                    const int64_t row = sh * p.cap + t0;
+                    const uint32_t kb = n * KROW, vb = n * VROW;
+                    const uint32_t kzb = (KM == K_TOKEN) ? ((n * ngk * 4 + 15) & ~15)
+                                                         : (KM == K_CHANNEL ? kHeadDim * 4 : 0);
+                    const uint32_t vzb = (VM == V_TOKEN) ? ((n * ngv * 4 + 15) & ~15) : 0;
+                    mbar_arrive_expect_tx(bar, kb + vb + kzb + vzb + qb);
+                    bulk_g2s(st, p.k_codes + row * KROW, kb, bar);
+                    bulk_g2s(st + p.off_vc, p.v_codes + row * VROW, vb, bar);
+                    if (KM == K_TOKEN) bulk_g2s(st + p.off_ksz, p.k_sz + row * ngk, kzb, bar);
+                    if (KM == K_CHANNEL)
+                        bulk_g2s(st + p.off_ksz, p.k_sz + (sh * (p.cap / p.R) + t0 / p.R) * kHeadDim, kzb, bar);
+                    if (VM == V_TOKEN) bulk_g2s(st + p.off_vsz, p.v_sz + row * ngv, vzb, bar);
+                } else {
+                    // Paged (token-wise groups only): one copy of each part per page.
+                    const int ps = p.page_size;
+                    const int span = ps < kTile ? ps : kTile;  // tokens per copy
+                    const uint32_t per_copy = span * (KROW + VROW + 4 * ngk + 4 * ngv);
+                    const int32_t *bt = p.block_table + static_cast<int64_t>(seq) * p.max_pages;
+                    uint32_t bytes = qb;
+                    for (int tp = t0; tp < t0 + n; tp += span) {
+                        const int pi = tp / ps;
+                        const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
+                        if (page >= 0 && page < p.num_pages) bytes += per_copy;
+                        else status_or(p.status, KVQ_DEV_CAPACITY);
+                    }
+                    mbar_arrive_expect_tx(bar, bytes);
+                    for (int tp = t0; tp < t0 + n; tp += span) {
+                        const int pi = tp / ps;
+                        const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
+                        if (page < 0 || page >= p.num_pages) continue;
+                        const int64_t prow = (static_cast<int64_t>(page) * p.H + kvh) * ps + (tp % ps);
+                        const uint32_t dt = tp - t0;
+                        bulk_g2s(st + dt * KROW, p.k_codes + prow * KROW, span * KROW, bar);
+                        bulk_g2s(st + p.off_ksz + dt * ngk * 4, p.k_sz + prow * ngk, span * ngk * 4, bar);
+                        bulk_g2s(st + p.off_vc + dt * VROW, p.v_codes + prow * VROW, span * VROW, bar);
+                        bulk_g2s(st + p.off_vsz + dt * ngv * 4, p.v_sz + prow * ngv, span * ngv * 4, bar);
+                    }
+                }
+                if (qb) bulk_g2s(st + p.off_q, qsrc, qb, bar);
             }
         }
         // Drain: wait for the copies of the last stages issued so none lands
         // after the CTA has gone.
-        for (int it = max(0, issued - NS); it < issued; ++it) {
-            if (it == p.skip_tile) continue;
-            const int s = it % NS, r = it / NS;
+        for (int j = max(0, it - NS); j < it; ++j) {
+            if (j == p.skip_tile) continue;
+            const int s = j % NS, r = j / NS;
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(&full[s], r & 1)) {
                 if (static_cast<int64_t>(global_timer_ns() - t0) > p.timeout_ns) {
@@ -599,60 +684,17 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
     }
 
     // --------------------------- consumers ---------------------------
-    // Query: warp g < GQA loads head kvh*GQA + g, 4 channels per lane, and
-    // rotates it like the keys; then scales by softmax_scale * log2(e).
-    if (warp < GQA) {
-        const int hq = kvh * GQA + warp;
-        const int64_t base = (static_cast<int64_t>(seq) * p.Hq + hq) * kHeadDim + 4 * lane;
-        float x[4];
-        if (p.q_dtype == KVQ_FP32) {
-            const float4 v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + base);
-            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-        } else {
-            const uint2 v = *reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.q) + base);
-            const uint32_t w[2] = {v.x, v.y};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                if (p.q_dtype == KVQ_BF16) {
-                    x[2 * j] = bf16_bits_to_float(w[j] & 0xFFFFu);
-                    x[2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
-                } else {
-                    x[2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] & 0xFFFFu)));
-                    x[2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] >> 16)));
-                }
-            }
-        }
-        if (p.hb > 0) {
-            if (p.hb > 1) { float a = x[0], b = x[1]; x[0] = a + b; x[1] = a - b;
-                            a = x[2]; b = x[3]; x[2] = a + b; x[3] = a - b; }
-            if (p.hb > 2) { float a = x[0], b = x[2]; x[0] = a + b; x[2] = a - b;
-                            a = x[1]; b = x[3]; x[1] = a + b; x[3] = a - b; }
-            for (int m = 1; m < 32 && 4 * m < p.hb; m <<= 1) {
-                const bool upper = (lane & m) != 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float o = __shfl_xor_sync(0xffffffffu, x[j], m);
-                    x[j] = upper ? o - x[j] : x[j] + o;
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) x[j] *= p.hscale;
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) qs[warp * kHeadDim + 4 * lane + j] = x[j] * p.qscale;
-    }
-    named_sync(1, kConsumers);
-
     const int part = lane & 7;
     constexpr int kOwnShift = LaneMap<GQA>::kOwnShift;
     // head held in register slot g (reduce-scatter order for GQA 4)
     const int perm = (GQA == 4) ? (((part >> 2) & 1) << 1 | ((part >> 1) & 1)) : 0;
     QueryRegs<GQA> Q;
     float *qsum = qsum_all + warp * 8 * 3 * GQA;
+    float *wsm = wsm_all + warp * 16 * 8 * GQA * 2;
+
     // mode: 0 = token-wise codes, 1 = channel-wise codes (per-channel scales
     // folded in from `chan_sz`), 2 = bf16 keys.
     auto load_query = [&](int mode, const uint8_t *chan_sz) {
-        float qa_full = 0.0f, qe_full = 0.0f;
         __syncwarp();  // this warp is done reading the previous sums
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
@@ -680,37 +722,18 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
                 qsum[(part * 3 + 2) * GQA + g] = (mode == 1) ? fmaf(-128.0f, first, qz) : 0.0f;
             }
         }
-        // Whole-head sums of the lane's own head (natural head order), for the
-        // scale applied after the reduce-scatter when a group spans the head.
-        // (the sum of the coefficients: all q for INT4, q0 + q3/16 per byte for INT2)
-        for (int d = 0; d < kHeadDim; ++d) {
-            const float v = qs[(part >> kOwnShift) * kHeadDim + d];
-            qa_full += v;
-            if (KBITS != 2) qe_full += v;
-            else if (d % 4 == 0) qe_full += v;
-            else if (d % 4 == 3) qe_full += 0.0625f * v;
-        }
-        Q.qa_own = qa_full;
-        Q.qe_own = qe_full;
+        // whole-head sums of the lane's own head (written by the item prologue)
+        Q.qa_own = qhead[part >> kOwnShift];
+        Q.qe_own = qhead[GQA + (part >> kOwnShift)];
         __syncwarp();
     };
-    if constexpr (KM != K_CHANNEL) load_query(KM == K_BF16 ? 2 : 0, nullptr);
 
     WarpState<GQA, VSLOTS> st;
-    st.m_own = -INFINITY;
-    st.l_own = 0.0f;
-#pragma unroll
-    for (int c = 0; c < VSLOTS; ++c) { st.wsum[c] = 0.0f; st.zsum[c] = 0.0f; }
-#pragma unroll
-    for (int g = 0; g < GQA; ++g)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
-    float *wsm = wsm_all + warp * 16 * 8 * GQA * 2;
-
+    bool folded = false;
     // Turn the value accumulators of quantized tiles into plain channel sums
     // (adding the zero-point terms), once: before the first bf16 window tile
-    // or at the end. Half-warp 1 adds no group terms, so the halves still sum.
-    bool folded = false;
+    // or at the end of the item. Half-warp 1 adds no group terms, so the
+    // halves still sum.
     auto fold_values = [&]() {
         constexpr int kPH = LaneMap<GQA>::kPerHead;
         float wsum[VSLOTS], zsum[VSLOTS];
@@ -725,8 +748,7 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
             st.wsum[c] = 0.0f;
             st.zsum[c] = 0.0f;
         }
-        const int sl = lane & 15;
-        const int gv_lane = (8 * sl) / p.group_v;
+        const int gv_lane = geo.vgroup(lane & 15);
         const bool first_half = lane < 16;
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
@@ -751,86 +773,153 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
     };
 
     int cur_block = -1;
-    for (int it = 0; it < n_tiles; ++it) {
+    for (int it = 0;; ++it) {
         const int s = it % NS, r = it / NS;
         if (!mbar_wait_bounded(&full[s], r & 1, p.timeout_ns, p.status, abort_flag)) break;
         const uint8_t *sb = stages + static_cast<size_t>(s) * p.stage_bytes;
-        if (it < n_qt) {
-            const int t0 = t_begin + it * kTile;
-            const int n = min(kTile, q_end - t0);
+        const TileHdr hdr = *reinterpret_cast<const TileHdr *>(sb + p.off_hdr);
+        if (hdr.flags & kDone) break;
+
+        if (hdr.flags & kFirst) {
+            // ---- item prologue: the query rows arrived with this tile ----
+            if (warp < GQA) {
+                const uint8_t *qrow = sb + p.off_q + warp * kHeadDim * p.q_bytes;
+                float x[4];
+                if (p.q_dtype == KVQ_FP32) {
+                    const uint4 v = lds128(qrow + 16 * lane);
+                    x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
+                    x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+                } else {
+                    const uint2 v = lds64(qrow + 8 * lane);
+                    const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        if (p.q_dtype == KVQ_BF16) {
+                            x[2 * j] = bf16_bits_to_float(w[j] & 0xFFFFu);
+                            x[2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
+                        } else {
+                            x[2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] & 0xFFFFu)));
+                            x[2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] >> 16)));
+                        }
+                    }
+                }
+                if (p.hb > 0) {
+                    if (p.hb > 1) { float a = x[0], b = x[1]; x[0] = a + b; x[1] = a - b;
+                                    a = x[2]; b = x[3]; x[2] = a + b; x[3] = a - b; }
+                    if (p.hb > 2) { float a = x[0], b = x[2]; x[0] = a + b; x[2] = a - b;
+                                    a = x[1]; b = x[3]; x[1] = a + b; x[3] = a - b; }
+                    for (int m = 1; m < 32 && 4 * m < p.hb; m <<= 1) {
+                        const bool upper = (lane & m) != 0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float o = __shfl_xor_sync(0xffffffffu, x[j], m);
+                            x[j] = upper ? o - x[j] : x[j] + o;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) x[j] *= p.hscale;
+                }
+                float sa = 0.0f, se = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    x[j] *= p.qscale;
+                    qs[warp * kHeadDim + 4 * lane + j] = x[j];
+                    sa += x[j];
+                    // sum of the code-byte coefficients: all q (INT4), q0 + q3/16 (INT2)
+                    se += (KBITS != 2) ? x[j] : (j == 0 ? x[j] : (j == 3 ? 0.0625f * x[j] : 0.0f));
+                }
+#pragma unroll
+                for (int m = 1; m < 32; m <<= 1) {
+                    sa += __shfl_xor_sync(0xffffffffu, sa, m);
+                    se += __shfl_xor_sync(0xffffffffu, se, m);
+                }
+                if (lane == 0) {
+                    qhead[warp] = sa;
+                    qhead[GQA + warp] = se;
+                }
+            }
+            named_sync(1, kConsumers);
+            cur_block = -1;
+            if constexpr (KM != K_CHANNEL) load_query(KM == K_BF16 ? 2 : 0, nullptr);
+            st.m_own = -INFINITY;
+            st.l_own = 0.0f;
+#pragma unroll
+            for (int c = 0; c < VSLOTS; ++c) { st.wsum[c] = 0.0f; st.zsum[c] = 0.0f; }
+#pragma unroll
+            for (int g = 0; g < GQA; ++g)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
+            folded = false;
+        }
+
+        if (!(hdr.flags & kWindow)) {
             if constexpr (KM == K_CHANNEL) {
-                const int blk = t0 / p.R;
+                const int blk = hdr.t0 / p.R;
                 if (blk != cur_block) {  // fold this block's channel scales into q
                     cur_block = blk;
                     load_query(1, sb + p.off_ksz);
                 }
             }
-            process_tile<GQA, KM, VM, KBITS, VBITS, kTile / kConsumerWarps, VSLOTS>(
-                sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, n, p.group_k, p.group_v, Q, qsum,
-                st, wsm, warp, lane);
-        } else {
-            if (it == n_qt && KM != K_BF16) {
+            process_tile<GQA, KM, VM, KBITS, VBITS, kTile / kConsumerWarps, GK, GV, VSLOTS>(
+                sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, geo, Q, qsum, st, wsm,
+                warp, lane);
+        } else if constexpr (KM != K_BF16) {
+            if (!folded) {  // first window tile of the item
                 load_query(2, nullptr);
-                if (VM == V_TOKEN && !folded) fold_values();
+                if (VM == V_TOKEN) fold_values();
+                folded = true;
             }
-            const int t0 = w_begin + (it - n_qt) * p.bf_tile;
-            const int n = min(p.bf_tile, t_end - t0);
-            if constexpr (KM == K_BF16) {
-                process_tile<GQA, K_BF16, V_BF16, 16, 16, kTile / kConsumerWarps, VSLOTS>(
-                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, Q, qsum, st, wsm, warp, lane);
-            } else {
-                process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, VSLOTS>(
-                    sb, nullptr, sb + p.bf_off_v, nullptr, n, 128, 128, Q, qsum, st, wsm, warp, lane);
+            process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, GK, GV, VSLOTS>(
+                sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, geo, Q, qsum, st, wsm, warp, lane);
+        }
+
+        if (hdr.flags & kLast) {
+            // ---- item epilogue: merge the four warps, write the partial ----
+            if (VM == V_TOKEN && !folded) fold_values();
+            float l_own = st.l_own;
+            l_own += __shfl_xor_sync(0xffffffffu, l_own, 8);
+            l_own += __shfl_xor_sync(0xffffffffu, l_own, 16);
+            const int slice = lane & 15;
+#pragma unroll
+            for (int g = 0; g < GQA; ++g) {
+                const float mg = __shfl_sync(0xffffffffu, st.m_own, g << kOwnShift);
+                const float lg = __shfl_sync(0xffffffffu, l_own, g << kOwnShift);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float2 v = st.o[g][c];
+                    v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
+                    v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
+                    if (lane < 16) {
+                        red[(warp * GQA + g) * 130 + 8 * slice + 2 * c] = v.x;
+                        red[(warp * GQA + g) * 130 + 8 * slice + 2 * c + 1] = v.y;
+                    }
+                }
+                if (lane == 0) {
+                    red[(warp * GQA + g) * 130 + 128] = mg;
+                    red[(warp * GQA + g) * 130 + 129] = lg;
+                }
+            }
+            named_sync(1, kConsumers);
+            for (int idx = tid; idx < GQA * kHeadDim; idx += kConsumers) {
+                const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[(w * GQA + g) * 130 + 128]);
+                float o = 0.0f, l = 0.0f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float mw = red[(w * GQA + g) * 130 + 128];
+                    const float e = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
+                    o = fmaf(e, red[(w * GQA + g) * 130 + d], o);
+                    l = fmaf(e, red[(w * GQA + g) * 130 + 129], l);
+                }
+                const int hq = hdr.kvh * GQA + g;
+                const int64_t pi = (static_cast<int64_t>(hdr.seq) * p.Hq + hq) * p.n_split + hdr.split;
+                p.o_part[pi * kHeadDim + d] = o;
+                if (d == 0) p.ml[pi] = make_float2(M, l);
             }
         }
         if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    const bool aborted = *abort_flag != 0;
-
-    // ---- merge the four warps ----
-    float l_own = st.l_own;
-    l_own += __shfl_xor_sync(0xffffffffu, l_own, 8);
-    l_own += __shfl_xor_sync(0xffffffffu, l_own, 16);
-    if (VM == V_TOKEN && !folded) fold_values();
-    const int slice = lane & 15;
-#pragma unroll
-    for (int g = 0; g < GQA; ++g) {
-        const float mg = __shfl_sync(0xffffffffu, st.m_own, g << kOwnShift);
-        const float lg = __shfl_sync(0xffffffffu, l_own, g << kOwnShift);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float2 v = st.o[g][c];
-            v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
-            v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
-            if (lane < 16) {
-                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c] = v.x;
-                red[(warp * GQA + g) * 130 + 8 * slice + 2 * c + 1] = v.y;
-            }
-        }
-        if (lane == 0) {
-            red[(warp * GQA + g) * 130 + 128] = mg;
-            red[(warp * GQA + g) * 130 + 129] = lg;
-        }
-    }
-    named_sync(1, kConsumers);
-    if (aborted) return;
-    for (int idx = tid; idx < GQA * kHeadDim; idx += kConsumers) {
-        const int g = idx / kHeadDim, d = idx - g * kHeadDim;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[(w * GQA + g) * 130 + 128]);
-        float o = 0.0f, l = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = red[(w * GQA + g) * 130 + 128];
-            const float e = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
-            o = fmaf(e, red[(w * GQA + g) * 130 + d], o);
-            l = fmaf(e, red[(w * GQA + g) * 130 + 129], l);
-        }
-        const int hq = kvh * GQA + g;
-        const int64_t pi = (static_cast<int64_t>(seq) * p.Hq + hq) * p.n_split + split;
-        p.o_part[pi * kHeadDim + d] = o;
-        if (d == 0) p.ml[pi] = make_float2(M, l);
     }
 }
 
@@ -859,80 +948,112 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *o_part, 
 // Host side
 // ---------------------------------------------------------------------------
 struct StageLayout {
-    int bytes, off_ksz, off_vc, off_vsz, bf_tile, bf_off_v;
+    int bytes, off_ksz, off_vc, off_vsz, off_q, off_hdr, bf_tile, bf_off_v;
 };
 
 inline int round16(int x) { return (x + 15) & ~15; }
 
-StageLayout stage_layout(const kvq_cache_desc &d) {
+// Stage: tile data, then the query rows of a first tile (GQA x 128 x q_bytes,
+// at most 2 KB), then a 32-byte header.
+StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
     StageLayout L{};
+    int data;
     if (d.bits_k == 16) {  // every tile is bf16 rows: K at 0, V after it
         L.bf_tile = kTile;
         L.bf_off_v = kTile * 256;
         L.off_vc = L.bf_off_v;
-        L.bytes = 2 * kTile * 256;
-        return L;
+        data = 2 * kTile * 256;
+    } else {
+        const int krow = 128 * d.bits_k / 8;
+        const int vrow = 128 * d.bits_v / 8;
+        const int ksz = (d.axis_k == KVQ_PER_CHANNEL) ? 128 * 4 : kTile * (128 / d.group_k) * 4;
+        const int vsz = kTile * (128 / d.group_v) * 4;
+        L.off_ksz = round16(kTile * krow);
+        L.off_vc = L.off_ksz + round16(ksz);
+        L.off_vsz = L.off_vc + round16(kTile * vrow);
+        data = L.off_vsz + round16(vsz);
+        L.bf_tile = kWinTile;
+        L.bf_off_v = kWinTile * 256;
+        if (d.residual_len > 0) data = std::max(data, 2 * kWinTile * 256);
     }
-    const int krow = 128 * d.bits_k / 8;
-    const int vrow = 128 * d.bits_v / 8;
-    const int ksz = (d.axis_k == KVQ_PER_CHANNEL) ? 128 * 4 : kTile * (128 / d.group_k) * 4;
-    const int vsz = kTile * (128 / d.group_v) * 4;
-    L.off_ksz = round16(kTile * krow);
-    L.off_vc = L.off_ksz + round16(ksz);
-    L.off_vsz = L.off_vc + round16(kTile * vrow);
-    L.bytes = L.off_vsz + round16(vsz);
-    L.bf_tile = kWinTile;
-    L.bf_off_v = kWinTile * 256;
-    if (d.residual_len > 0) L.bytes = std::max(L.bytes, 2 * kWinTile * 256);
-    L.bytes = (L.bytes + 127) & ~127;
+    L.off_q = round16(data);
+    L.off_hdr = L.off_q + round16(gqa * kHeadDim * q_bytes);
+    L.bytes = (L.off_hdr + static_cast<int>(sizeof(TileHdr)) + 127) & ~127;
     return L;
 }
 
 template <int GQA>
-size_t tail_bytes(int NS) {
+size_t tail_bytes(int NS, int S) {
     return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * 16 * 8 * GQA * 2 +
-                            kConsumerWarps * GQA * 130 + kConsumerWarps * 8 * 3 * GQA) +
-           sizeof(uint64_t) * 2 * NS + 16;
+                            kConsumerWarps * GQA * 130 + kConsumerWarps * 8 * 3 * GQA + 2 * GQA + 2) +
+           sizeof(uint64_t) * 2 * NS + 16 + sizeof(int) * (S + 1);
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int VSLOTS>
-kvq_status launch_variant_slots(const DecodeParams &p, dim3 grid, cudaStream_t stream) {
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int GK, int GV>
+kvq_status launch_variant(const DecodeParams &p, int max_items, cudaStream_t stream) {
     constexpr int NS = (KM == K_BF16) ? 3 : 4;
-    const size_t smem = static_cast<size_t>(NS) * p.stage_bytes + tail_bytes<GQA>(NS);
-    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, NS, VSLOTS>;
+    const size_t smem = static_cast<size_t>(NS) * p.stage_bytes + tail_bytes<GQA>(NS, p.S);
+    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, NS, GK, GV>;
+    if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;  // too many sequences for one launch
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return KVQ_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess ||
+        per_sm <= 0)
+        per_sm = 1;
+    const int grid = std::max(1, std::min(max_items, per_sm * sm_count()));
+    if (cudaMemsetAsync(p.counter, 0, sizeof(int), stream) != cudaSuccess) return KVQ_ERR_CUDA;
     kern<<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
-// One value-group slot per lane when a head's groups fit one per lane.
+// Compile-time group sizes for the common shapes, runtime ones otherwise.
 template <int GQA, int KM, int VM, int KBITS, int VBITS>
-kvq_status launch_variant(const DecodeParams &p, dim3 grid, cudaStream_t stream) {
-    const int n_vg = (VM == V_BF16) ? 1 : kHeadDim / p.group_v;
-    if (n_vg <= LaneMap<GQA>::kPerHead)
-        return launch_variant_slots<GQA, KM, VM, KBITS, VBITS, 1>(p, grid, stream);
-    return launch_variant_slots<GQA, KM, VM, KBITS, VBITS, 4>(p, grid, stream);
+kvq_status launch_groups(const kvq_cache_desc &d, const DecodeParams &p, int max_items,
+                         cudaStream_t stream) {
+    if constexpr (GQA == 4 && VM == V_TOKEN) {
+        const int gk = (KM == K_TOKEN) ? d.group_k : 0;
+        if (KM == K_TOKEN && gk == 128 && d.group_v == 128)
+            return launch_variant<GQA, KM, VM, KBITS, VBITS, 128, 128>(p, max_items, stream);
+        if (KM == K_TOKEN && gk == 32 && d.group_v == 32)
+            return launch_variant<GQA, KM, VM, KBITS, VBITS, 32, 32>(p, max_items, stream);
+        if (KM == K_CHANNEL && d.group_v == 32)
+            return launch_variant<GQA, KM, VM, KBITS, VBITS, 0, 32>(p, max_items, stream);
+    }
+    return launch_variant<GQA, KM, VM, KBITS, VBITS, 0, 0>(p, max_items, stream);
 }
 
 template <int GQA>
-kvq_status dispatch_modes(const kvq_cache_desc &d, const DecodeParams &p, dim3 grid,
+kvq_status dispatch_modes(const kvq_cache_desc &d, const DecodeParams &p, int max_items,
                           cudaStream_t stream) {
     if (d.bits_k == 16 && d.bits_v == 16)
-        return launch_variant<GQA, K_BF16, V_BF16, 16, 16>(p, grid, stream);
+        return launch_variant<GQA, K_BF16, V_BF16, 16, 16, 0, 0>(p, max_items, stream);
     if (d.axis_k == KVQ_PER_CHANNEL) {
-        if (d.bits_k == 2 && d.bits_v == 2) return launch_variant<GQA, K_CHANNEL, V_TOKEN, 2, 2>(p, grid, stream);
-        if (d.bits_k == 4 && d.bits_v == 4) return launch_variant<GQA, K_CHANNEL, V_TOKEN, 4, 4>(p, grid, stream);
-        if (d.bits_k == 2 && d.bits_v == 4) return launch_variant<GQA, K_CHANNEL, V_TOKEN, 2, 4>(p, grid, stream);
-        if (d.bits_k == 4 && d.bits_v == 2) return launch_variant<GQA, K_CHANNEL, V_TOKEN, 4, 2>(p, grid, stream);
+        if (d.bits_k == 2 && d.bits_v == 2) return launch_groups<GQA, K_CHANNEL, V_TOKEN, 2, 2>(d, p, max_items, stream);
+        if (d.bits_k == 4 && d.bits_v == 4) return launch_groups<GQA, K_CHANNEL, V_TOKEN, 4, 4>(d, p, max_items, stream);
+        if (d.bits_k == 2 && d.bits_v == 4) return launch_groups<GQA, K_CHANNEL, V_TOKEN, 2, 4>(d, p, max_items, stream);
+        if (d.bits_k == 4 && d.bits_v == 2) return launch_groups<GQA, K_CHANNEL, V_TOKEN, 4, 2>(d, p, max_items, stream);
         return KVQ_ERR_UNSUPPORTED;
     }
-    if (d.bits_k == 4 && d.bits_v == 4) return launch_variant<GQA, K_TOKEN, V_TOKEN, 4, 4>(p, grid, stream);
-    if (d.bits_k == 2 && d.bits_v == 2) return launch_variant<GQA, K_TOKEN, V_TOKEN, 2, 2>(p, grid, stream);
-    if (d.bits_k == 4 && d.bits_v == 2) return launch_variant<GQA, K_TOKEN, V_TOKEN, 4, 2>(p, grid, stream);
-    if (d.bits_k == 2 && d.bits_v == 4) return launch_variant<GQA, K_TOKEN, V_TOKEN, 2, 4>(p, grid, stream);
+    if (d.bits_k == 4 && d.bits_v == 4) return launch_groups<GQA, K_TOKEN, V_TOKEN, 4, 4>(d, p, max_items, stream);
+    if (d.bits_k == 2 && d.bits_v == 2) return launch_groups<GQA, K_TOKEN, V_TOKEN, 2, 2>(d, p, max_items, stream);
+    if (d.bits_k == 4 && d.bits_v == 2) return launch_groups<GQA, K_TOKEN, V_TOKEN, 4, 2>(d, p, max_items, stream);
+    if (d.bits_k == 2 && d.bits_v == 4) return launch_groups<GQA, K_TOKEN, V_TOKEN, 2, 4>(d, p, max_items, stream);
     return KVQ_ERR_UNSUPPORTED;
+}
+
+int log2i(int x) {
+    int r = 0;
+    while ((1 << r) < x) ++r;
+    return r;
 }
 
 }  // namespace
@@ -940,18 +1061,19 @@ kvq_status dispatch_modes(const kvq_cache_desc &d, const DecodeParams &p, dim3 g
 bool plan_decode(const kvq_cache_desc &d, int num_seqs, int num_q_heads, int max_seq_len,
                  DecodePlan *plan) {
     if (num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0 || d.num_kv_heads <= 0) return false;
+    // About six items per resident CTA (2 per SM) when every sequence is at
+    // max_seq_len; chunks of 256..4096 tokens, a multiple of the tile.
     const int64_t units = static_cast<int64_t>(num_seqs) * d.num_kv_heads;
-    const int64_t want_ctas = 8 * 148;
-    const int64_t splits = std::max<int64_t>(1, (want_ctas + units - 1) / units);
-    int64_t chunk = (std::max(1, max_seq_len) + splits - 1) / splits;
+    const int64_t target_items = 6 * 2 * 148;
+    int64_t chunk = (units * std::max(1, max_seq_len) + target_items - 1) / target_items;
     chunk = ((chunk + kTile - 1) / kTile) * kTile;
-    chunk = std::max<int64_t>(chunk, 256);
+    chunk = std::min<int64_t>(std::max<int64_t>(chunk, 256), 4096);
     plan->chunk = static_cast<int>(chunk);
     plan->n_split = static_cast<int>(std::max<int64_t>(1, (max_seq_len + chunk - 1) / chunk));
     const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * plan->n_split;
     plan->ws_part = rows * kHeadDim * sizeof(float);
     plan->ws_ml = rows * sizeof(float2);
-    plan->ws_total = plan->ws_part + plan->ws_ml;
+    plan->ws_total = plan->ws_part + plan->ws_ml + 16;  // + the item counter
     return true;
 }
 
@@ -972,11 +1094,13 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.q = q;
     p.o_part = static_cast<float *>(workspace);
     p.ml = reinterpret_cast<float2 *>(static_cast<uint8_t *>(workspace) + plan.ws_part);
+    p.counter = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + plan.ws_part + plan.ws_ml);
     p.status = d.status;
+    p.S = num_seqs;
     p.H = d.num_kv_heads;
     p.Hq = num_q_heads;
-    p.group_k = d.group_k;
-    p.group_v = d.group_v;
+    p.gk_log2 = log2i(std::max(1, d.group_k));
+    p.gv_log2 = log2i(std::max(1, d.group_v));
     p.hb = d.hadamard_block_k;
     p.hscale = hadamard_scale(d.hadamard_block_k);
     p.qscale = softmax_scale * kLog2e;
@@ -990,20 +1114,25 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.n_split = plan.n_split;
     p.max_seq_len = max_seq_len;
     p.q_dtype = q_dtype;
-    const StageLayout L = stage_layout(d);
+    p.q_bytes = (q_dtype == KVQ_FP32) ? 4 : 2;
+    const int gqa = num_q_heads / d.num_kv_heads;
+    const StageLayout L = stage_layout(d, gqa, p.q_bytes);
     p.stage_bytes = L.bytes;
     p.off_ksz = L.off_ksz;
     p.off_vc = L.off_vc;
     p.off_vsz = L.off_vsz;
+    p.off_q = L.off_q;
+    p.off_hdr = L.off_hdr;
     p.bf_tile = L.bf_tile;
     p.bf_off_v = L.bf_off_v;
     p.timeout_ns = debug_hooks().wait_timeout_ns;
     p.skip_tile = debug_hooks().skip_tile;
-    const dim3 grid(plan.n_split, d.num_kv_heads, num_seqs);
-    switch (num_q_heads / d.num_kv_heads) {
-        case 1: return dispatch_modes<1>(d, p, grid, stream);
-        case 2: return dispatch_modes<2>(d, p, grid, stream);
-        case 4: return dispatch_modes<4>(d, p, grid, stream);
+    const int64_t max_items64 = static_cast<int64_t>(num_seqs) * d.num_kv_heads * plan.n_split;
+    const int max_items = static_cast<int>(std::min<int64_t>(max_items64, 1 << 30));
+    switch (gqa) {
+        case 1: return dispatch_modes<1>(d, p, max_items, stream);
+        case 2: return dispatch_modes<2>(d, p, max_items, stream);
+        case 4: return dispatch_modes<4>(d, p, max_items, stream);
         default: return KVQ_ERR_UNSUPPORTED;
     }
 }
