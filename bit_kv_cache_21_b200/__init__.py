@@ -11,7 +11,8 @@ from ._binding import (  # noqa: F401
     DEBUG_WAIT_TIMEOUT_NS, DEBUG_SKIP_TILE,
     OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_TIMEOUT, ERR_CUDA,
     CacheDesc, KvqError, lib, header_symbols, status_string, check,
-    quantize_append, decode_workspace_size, decode_attention, decode_splitk, decode_merge,
+    quantize_append, decode_workspace_size, decode_attention, decode_attention_static,
+    decode_splitk, decode_merge,
     remat_kv, rope_tables, debug_set, version,
 )
 from .cache import CacheSpec, KVCache  # noqa: F401

@@ -74,6 +74,7 @@ _SIGNATURES = {
     "kvq_decode_workspace_size": (_S, [_DESC, _I, _I, _I]),
     "kvq_decode_attention": (_I, [_DESC, _P, _I, _I, _P, _I, _I, ctypes.c_float, _P, _P, _S, _P]),
     "kvq_decode_splitk": (_I, [_DESC, _P, _I, _I, _P, _I, _I, ctypes.c_float, _P, _S, _P]),
+    "kvq_decode_attention_static": (_I, [_DESC, _P, _I, _I, _P, _I, _I, ctypes.c_float, _P, _P]),
     "kvq_decode_merge": (_I, [_DESC, _I, _P, _I, _I, _P, _P, _S, _P]),
     "kvq_remat_kv": (_I, [_DESC, _P, _I, _P, _P, _I, _I, _P, _P, _P]),
     "kvq_rope_tables": (_I, [_P, _P, _I, _I, ctypes.c_double, _P]),
@@ -192,6 +193,24 @@ def decode_attention(desc: CacheDesc, q, seq_lens, max_seq_len: int, softmax_sca
                                     _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream_handle(stream))
     check(st, "kvq_decode_attention")
+    return out
+
+
+def decode_attention_static(desc: CacheDesc, q, seq_lens, max_seq_len: int, softmax_scale: float,
+                            out=None, stream=None):
+    """kvq_decode_attention_static: decode attention with the library's fixed
+    device workspace, for callers that cannot allocate one."""
+    import torch
+    _require(q, "q")
+    _require(seq_lens, "seq_lens", torch.int32)
+    num_seqs, num_q_heads = q.shape[0], q.shape[1]
+    if out is None:
+        out = torch.empty((num_seqs, num_q_heads, 128), dtype=torch.float32, device=q.device)
+    _require(out, "out", torch.float32)
+    st = lib().kvq_decode_attention_static(ctypes.byref(desc), _ptr(q), dtype_code(q), num_q_heads,
+                                           _ptr(seq_lens), num_seqs, max_seq_len,
+                                           float(softmax_scale), _ptr(out), _stream_handle(stream))
+    check(st, "kvq_decode_attention_static")
     return out
 
 

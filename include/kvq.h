@@ -206,6 +206,29 @@ KVQ_API kvq_status kvq_decode_merge(const kvq_cache_desc *desc, int32_t num_q_he
                             void *stream);
 
 /*
+ * kvq_decode_attention_static -- kvq_decode_attention without a workspace
+ * argument, for callers that cannot allocate device memory: a plain C program
+ * or a plugin running inside a runtime that owns every device allocation, or a
+ * decode loop that must not call cudaMalloc (it can synchronize the device).
+ * The method pages have no counterpart; this is an interface convenience.
+ * The workspace is a 16 MiB array in device global memory that the library
+ * declares; it is reserved on every GPU that loads the library until the
+ * process exits. Sizes whose workspace (kvq_decode_workspace_size) exceeds
+ * 16 MiB are rejected with KVQ_ERR_CAPACITY before anything is launched.
+ * The first call on a device looks up the array's device address (once per
+ * device); make that first call before any stream capture. All calls share the
+ * array and it keeps the previous call's contents (what must start at zero is
+ * cleared on the stream by each call), so calls whose work overlaps on the GPU
+ * -- on different streams or from different host threads -- race on it.
+ * Other arguments, results and errors are those of kvq_decode_attention.
+ */
+KVQ_API kvq_status kvq_decode_attention_static(const kvq_cache_desc *desc, const void *q,
+                                               kvq_dtype q_dtype, int32_t num_q_heads,
+                                               const int32_t *seq_lens, int32_t num_seqs,
+                                               int32_t max_seq_len, float softmax_scale,
+                                               float *out, void *stream);
+
+/*
  * kvq_remat_kv -- rematerialize K and V of `batch` sequences for positions
  * [0, ctx_len) from a cache of quantized layer inputs X.
  * x_cache: contiguous per-token cache holding X as hidden/128 "heads" of 128
