@@ -114,3 +114,22 @@ class KVCache:
         if s.paged:
             return t16.view(s.num_pages, s.num_kv_heads, s.page_size, HEAD_DIM // G, 2)
         return t16.view(s.num_seqs, s.num_kv_heads, s.capacity_tokens, HEAD_DIM // G, 2)
+
+
+def bf16_cache_desc(k, v, status=None) -> B.CacheDesc:
+    """Descriptor of an unquantized bf16 cache (bits 16) over k, v
+    [S][H][T][128] -- the layout kvq_remat_kv writes -- so that
+    kvq_decode_attention reads rematerialized keys and values directly."""
+    import torch
+    if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16 or k.shape != v.shape or k.dim() != 4:
+        raise ValueError("k, v must be bf16 tensors of one shape [S][H][T][128]")
+    if not (k.is_contiguous() and v.is_contiguous()) or k.shape[-1] != HEAD_DIM:
+        raise ValueError("k, v must be contiguous with head_dim 128")
+    S, H, T, _ = k.shape
+    return B.CacheDesc(
+        num_seqs=S, num_kv_heads=H, head_dim=HEAD_DIM, bits_k=16, bits_v=16,
+        group_k=0, group_v=0, axis_k=B.PER_TOKEN, axis_v=B.PER_TOKEN, hadamard_block_k=0,
+        residual_len=0, paged=0, page_size=0, max_pages_per_seq=0, num_pages=0,
+        capacity_tokens=T, reserved=0, k_codes=k.data_ptr(), v_codes=v.data_ptr(),
+        k_sz=None, v_sz=None, k_res=None, v_res=None, block_table=None,
+        status=None if status is None else status.data_ptr())
