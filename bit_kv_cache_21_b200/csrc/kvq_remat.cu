@@ -10,19 +10,19 @@
 //
 // Tiles are 128 tokens x 256 output channels (two heads of K or V); one CTA
 // per SM walks the tiles. Warp roles:
-//   warp 0      TMA producer: per 64-wide K step, the W box (256 x 64 bf16,
-//               128-byte swizzle), the X codes box (128 tokens x 32 bytes) and
-//               the tokens' fp16 scale/zero (512 bytes), completing on one
-//               mbarrier. No multicast.
+//   warp 0      W producer: per 64-wide K step, a TMA box of W (256 x 64
+//               bf16, 128-byte swizzle). No multicast.
+//   warp 2      codes producer: the X codes box (128 tokens x 32 bytes) and
+//               the tokens' fp16 scale/zero (512 bytes).
 //   warp 1      allocates 512 TMEM columns (two 256-column fp32
 //               accumulators); one lane issues tcgen05.mma (kind::f16, bf16
-//               operands, M=128, N=256, K=16) and tcgen05.commit frees each
-//               stage and signals a finished accumulator.
-//   warps 2-5   dequantize the codes into the A operand (128 x 64 bf16) in the
+//               operands, M=128, N=256, K=16); tcgen05.commit frees the W and
+//               A slots and signals a finished accumulator.
+//   warps 3-6   dequantize the codes into the A operand (128 x 64 bf16) in the
 //               same 128-byte-swizzled K-major layout TMA gives W, one token
 //               row per thread, then fence the generic-proxy writes for the
 //               tensor core.
-//   warps 6-9   epilogue: tcgen05.ld one accumulator row per thread, RoPE in
+//   warps 7-10  epilogue: tcgen05.ld one accumulator row per thread, RoPE in
 //               fp32 on K, round to bf16, store [B][H][T][128]. Two accumulators
 //               let the epilogue of one tile overlap the main loop of the next.
 // Every mbarrier wait is bounded; on expiry the kernel sets KVQ_DEV_TIMEOUT,
@@ -44,24 +44,37 @@ constexpr int kBM = 128;                    // tokens per tile (MMA M)
 constexpr int kBN = 256;                    // output channels per tile (MMA N)
 constexpr int kBK = 64;                     // hidden channels per stage (one 128-byte row)
 constexpr int kUmmaK = 16;                  // K of one tcgen05.mma kind::f16
-constexpr int kStages = 4;
-constexpr int kBBytes = kBN * kBK * 2;      // 32 KiB
-constexpr int kABytes = kBM * kBK * 2;      // 16 KiB
+// Three rings, each recycled by its own consumer, so that no ring's refill
+// waits for more than one step of the chain TMA -> dequantize -> MMA:
+//   W ring      (TMA -> MMA, freed by tcgen05.commit)
+//   A ring      (dequantizers -> MMA, freed by tcgen05.commit)
+//   codes ring  (TMA -> dequantizers, freed as soon as they hold the codes)
+constexpr int kWStages = 4;
+constexpr int kAStages = 3;
+constexpr int kCStages = 8;
+constexpr int kBBytes = kBN * kBK * 2;      // 32 KiB of W per stage
+constexpr int kABytes = kBM * kBK * 2;      // 16 KiB of bf16 x^ per stage
 constexpr int kCodeBytes = kBM * kBK / 2;   // 4 KiB of INT4 codes
 constexpr int kSzBytes = kBM * 4;           // half2 per token
-constexpr int kOffA = kBBytes;
-constexpr int kOffCodes = kOffA + kABytes;
-constexpr int kOffSz = kOffCodes + kCodeBytes;
-constexpr int kStageBytes = ((kOffSz + kSzBytes) + 1023) & ~1023;  // 53 KiB
-constexpr int kTxBytes = kBBytes + kCodeBytes + kSzBytes;
+constexpr int kCStageBytes = kCodeBytes + kSzBytes;
+constexpr int kOffARing = kWStages * kBBytes;
+constexpr int kOffCRing = kOffARing + kAStages * kABytes;
+constexpr int kRingBytes = kOffCRing + kCStages * kCStageBytes;
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = 256;
-constexpr int kThreads = 320;
-constexpr int kBarBytes = 256;
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + kBarBytes;
+// warps: 0 W producer, 1 MMA issuer (+ TMEM owner), 2 codes producer,
+// 3-6 dequantizers, 7-10 epilogue
+constexpr int kDeqWarp0 = 3;
+constexpr int kEpiWarp0 = 7;
+constexpr int kThreads = 11 * 32;
+constexpr int kNumBars = 2 * kWStages + 2 * kAStages + 2 * kCStages + 5;
+constexpr int kBarBytes = 512;
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kRingBytes) + kBarBytes;
 
-static_assert(kStageBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-static_assert(kOffA % 1024 == 0, "A tile alignment");
+static_assert(kOffARing % 1024 == 0 && kABytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(kOffCRing % 128 == 0 && kCStageBytes % 128 == 0, "TMA destination alignment");
+static_assert(kNumBars * 8 + 8 <= kBarBytes, "barrier area");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 struct RematParams {
     const __half2 *x_sz;   // [S][XH][Tc] (one group of 128 channels per row)
@@ -175,6 +188,95 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)),
+          "l"(*reinterpret_cast<unsigned long long *>(&b)),
+          "l"(*reinterpret_cast<unsigned long long *>(&c)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+
+// Rounding error of the fp32 sum a + b (Knuth's TwoSum): zero iff the sum is exact.
+__device__ __forceinline__ float two_sum_err(float a, float b) {
+    const float s = __fadd_rn(a, b);
+    const float bp = __fsub_rn(s, a);
+    const float ap = __fsub_rn(s, bp);
+    return __fadd_rn(__fsub_rn(a, ap), __fsub_rn(b, bp));
+}
+
+// One row's 32 code bytes and its scale/zero word from shared memory.
+__device__ __forceinline__ void lds_codes(const uint8_t *codes, const uint8_t *sz, uint4 &c0, uint4 &c1,
+                                          uint32_t &szw) {
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w)
+                 : "r"(smem_addr(codes))
+                 : "memory");
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
+                 : "r"(smem_addr(codes + 16))
+                 : "memory");
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(szw) : "r"(smem_addr(sz)) : "memory");
+}
+
+// Dequantize one token row's 64 INT4 codes (32 bytes, element 2i in the low
+// nibble of byte i) into 64 bf16 x^ = bf16_rn(fp32(q*s + z)), written as the
+// row's eight 16-byte chunks of a 128-byte-swizzled K-major tile.
+//
+// Fast form: a byte permute puts nibble q in the top mantissa bits of 1.0,
+// f = 1 + q/128 exactly, and fma(f, 128 s, z - 128 s) equals q*s + z before
+// its single rounding whenever z - 128 s is exact in fp32 (checked per row);
+// otherwise the codes go through 2^23 + q - 2^23 and fma(q, s, z).
+__device__ __forceinline__ void dequant_row(uint4 c0, uint4 c1, float sc, float zp, uint8_t *arow,
+                                            uint32_t swz) {
+    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    const float s128 = __fmul_rn(sc, 128.0f);
+    const float cz = __fsub_rn(zp, s128);
+    if (two_sum_err(zp, -s128) == 0.0f) {
+        const float2 mul = make_float2(s128, s128), add = make_float2(cz, cz);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t w = words[c];
+            const uint32_t lo = (w & 0x0F0F0F0Fu) | 0x80808080u;
+            const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+            uint32_t out[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                // bytes {0, 0, 0x80|q, 0x3F}: the float 1 + q/128
+                const uint32_t sel = 0x7044u | (static_cast<uint32_t>(i) << 8);
+                const float2 f = make_float2(__uint_as_float(prmt(lo, 0x3F000000u, sel)),
+                                             __uint_as_float(prmt(hi, 0x3F000000u, sel)));
+                const float2 x = ffma2(f, mul, add);
+                out[i] = pack_bf16x2(x.x, x.y);
+            }
+            *reinterpret_cast<uint4 *>(arow + ((c ^ swz) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t w = words[c];
+            const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+            uint32_t out[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                // bytes {q, 0, 0, 0x4B}: the float 2^23 + q
+                const uint32_t sel = 0x7440u | static_cast<uint32_t>(i);
+                const float qe = __fsub_rn(__uint_as_float(prmt(lo, 0x4B000000u, sel)), 8388608.0f);
+                const float qo = __fsub_rn(__uint_as_float(prmt(hi, 0x4B000000u, sel)), 8388608.0f);
+                out[i] = pack_bf16x2(__fmaf_rn(qe, sc, zp), __fmaf_rn(qo, sc, zp));
+            }
+            *reinterpret_cast<uint4 *>(arow + ((c ^ swz) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+    }
+}
+
 // Tile id -> (batch row block, N tile). N varies fastest so that the CTAs
 // running at the same time share X rows in L2.
 struct TileCoord {
@@ -196,28 +298,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t *stages = smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
-    uint64_t *full_tma = bars;                 // [kStages] TMA bytes landed
-    uint64_t *full_a = bars + kStages;         // [kStages] A operand written (4 warps)
-    uint64_t *empty = bars + 2 * kStages;      // [kStages] MMAs reading the stage done
-    uint64_t *acc_full = bars + 3 * kStages;   // [2] accumulator ready
-    uint64_t *acc_empty = acc_full + 2;        // [2] accumulator drained (4 warps)
-    uint64_t *mma_done = acc_empty + 2;        // [1] every MMA of this CTA finished
+    uint8_t *w_ring = smem;
+    uint8_t *a_ring = smem + kOffARing;
+    uint8_t *c_ring = smem + kOffCRing;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+    uint64_t *w_full = bars;                       // [kWStages] W landed (tx)
+    uint64_t *w_empty = w_full + kWStages;         // [kWStages] MMAs done with W
+    uint64_t *a_full = w_empty + kWStages;         // [kAStages] x^ written (128 threads)
+    uint64_t *a_empty = a_full + kAStages;         // [kAStages] MMAs done with x^
+    uint64_t *c_full = a_empty + kAStages;         // [kCStages] codes landed (tx)
+    uint64_t *c_empty = c_full + kCStages;         // [kCStages] codes taken (128 threads)
+    uint64_t *acc_full = c_empty + kCStages;       // [2] accumulator ready
+    uint64_t *acc_empty = acc_full + 2;            // [2] accumulator drained (128 threads)
+    uint64_t *mma_done = acc_empty + 2;            // [1] every MMA of this CTA finished
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full_tma[s], 1);
-            mbar_init(&full_a[s], 4);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kWStages; ++s) {
+            mbar_init(&w_full[s], 1);
+            mbar_init(&w_empty[s], 1);
+        }
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&a_full[s], 128);
+            mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < kCStages; ++s) {
+            mbar_init(&c_full[s], 1);
+            mbar_init(&c_empty[s], 128);
         }
         for (int j = 0; j < 2; ++j) {
             mbar_init(&acc_full[j], 1);
-            mbar_init(&acc_empty[j], 4);
+            mbar_init(&acc_empty[j], 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -232,39 +346,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_k = 2 * p.XH;  // K steps of 64 hidden channels
     const int n_total = p.m_tiles * p.n_tiles;
 
+    // Wait (bounded) until the copies of a producer's last `depth` ring slots
+    // have landed, so none arrives after the CTA has gone.
+    auto drain = [&](uint64_t *full, int depth, int issued) {
+        for (int j = max(0, issued - depth); j < issued; ++j) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(&full[j % depth], (j / depth) & 1)) {
+                if (static_cast<int64_t>(global_timer_ns() - t0) > p.timeout_ns) {
+                    status_or(p.status, KVQ_DEV_TIMEOUT);
+                    break;
+                }
+            }
+        }
+    };
+
     if (warp == 0) {
-        // ------------------------------ TMA producer ------------------------------
+        // ------------------------------ W producer --------------------------------
         if (lane == 0) {
             int it = 0;
             bool stop = false;
             for (int tile = blockIdx.x; tile < n_total && !stop; tile += gridDim.x) {
                 const TileCoord c = tile_coord(p, tile);
                 for (int kb = 0; kb < n_k; ++kb, ++it) {
-                    const int s = it % kStages, r = it / kStages;
-                    if (r > 0 && !mbar_wait_bounded(&empty[s], (r - 1) & 1, p.timeout_ns, p.status,
+                    const int s = it % kWStages, r = it / kWStages;
+                    if (r > 0 && !mbar_wait_bounded(&w_empty[s], (r - 1) & 1, p.timeout_ns, p.status,
                                                     abort_flag)) {
                         stop = true;
                         break;
                     }
-                    uint8_t *st = stages + s * kStageBytes;
-                    const int xh = kb >> 1;
-                    const int row = (c.b * p.XH + xh) * p.Tc + c.t0;
-                    mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
-                    tma_load_2d(st, &tm_w, kb * kBK, c.n * kBN, &full_tma[s]);
-                    tma_load_2d(st + kOffCodes, &tm_x, (kb & 1) * (kBK / 2), row, &full_tma[s]);
-                    bulk_g2s(st + kOffSz, p.x_sz + row, kSzBytes, &full_tma[s]);
+                    mbar_arrive_expect_tx(&w_full[s], kBBytes);
+                    tma_load_2d(w_ring + s * kBBytes, &tm_w, kb * kBK, c.n * kBN, &w_full[s]);
                 }
             }
-            // Drain: the copies of the last stages must land before exit.
-            for (int j = max(0, it - kStages); j < it; ++j) {
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(&full_tma[j % kStages], (j / kStages) & 1)) {
-                    if (static_cast<int64_t>(global_timer_ns() - t0) > p.timeout_ns) {
-                        status_or(p.status, KVQ_DEV_TIMEOUT);
+            drain(w_full, kWStages, it);
+        }
+    } else if (warp == 2) {
+        // ---------------------------- codes producer ------------------------------
+        if (lane == 0) {
+            int it = 0;
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < n_total && !stop; tile += gridDim.x) {
+                const TileCoord c = tile_coord(p, tile);
+                for (int kb = 0; kb < n_k; ++kb, ++it) {
+                    const int s = it % kCStages, r = it / kCStages;
+                    if (r > 0 && !mbar_wait_bounded(&c_empty[s], (r - 1) & 1, p.timeout_ns, p.status,
+                                                    abort_flag)) {
+                        stop = true;
                         break;
                     }
+                    uint8_t *st = c_ring + s * kCStageBytes;
+                    const int row = (c.b * p.XH + (kb >> 1)) * p.Tc + c.t0;
+                    mbar_arrive_expect_tx(&c_full[s], kCStageBytes);
+                    tma_load_2d(st, &tm_x, (kb & 1) * (kBK / 2), row, &c_full[s]);
+                    bulk_g2s(st + kCodeBytes, p.x_sz + row, kSzBytes, &c_full[s]);
                 }
             }
+            drain(c_full, kCStages, it);
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer --------------------------------
@@ -279,23 +416,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + j * kAccCols;
                 for (int kb = 0; kb < n_k; ++kb, ++it) {
-                    const int s = it % kStages, r = it / kStages;
-                    if (!mbar_wait_bounded(&full_tma[s], r & 1, p.timeout_ns, p.status, abort_flag) ||
-                        !mbar_wait_bounded(&full_a[s], r & 1, p.timeout_ns, p.status, abort_flag)) {
+                    const int sw = it % kWStages, rw = it / kWStages;
+                    const int sa = it % kAStages, ra = it / kAStages;
+                    if (!mbar_wait_bounded(&w_full[sw], rw & 1, p.timeout_ns, p.status, abort_flag) ||
+                        !mbar_wait_bounded(&a_full[sa], ra & 1, p.timeout_ns, p.status, abort_flag)) {
                         stop = true;
                         break;
                     }
                     tc_fence_after();
-                    uint8_t *st = stages + s * kStageBytes;
-                    const uint64_t a_desc = sw128_desc(smem_addr(st + kOffA));
-                    const uint64_t b_desc = sw128_desc(smem_addr(st));
+                    const uint64_t a_desc = sw128_desc(smem_addr(a_ring + sa * kABytes));
+                    const uint64_t b_desc = sw128_desc(smem_addr(w_ring + sw * kBBytes));
 #pragma unroll
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
                         // +32 bytes along K inside the swizzle atom = +2 in the
                         // descriptor's 16-byte address units.
                         umma_bf16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, (kb | kk) != 0);
                     }
-                    umma_commit(&empty[s]);
+                    umma_commit(&w_empty[sw]);
+                    umma_commit(&a_empty[sa]);
                 }
                 if (!stop) umma_commit(&acc_full[j]);
             }
@@ -309,46 +447,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         // ------------------------------ dequantizers ------------------------------
-        const int row = threadIdx.x - 64;  // token row of the tile, 0..127
-        const uint32_t swz = row & 7;
-        int it = 0;
-        bool stop = false;
-        for (int tile = blockIdx.x; tile < n_total && !stop; tile += gridDim.x) {
-            for (int kb = 0; kb < n_k; ++kb, ++it) {
-                const int s = it % kStages, r = it / kStages;
-                // Warp-uniform outcome: the warp's later steps need all lanes.
-                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_tma[s], r & 1, p.timeout_ns,
-                                                               p.status, abort_flag))) {
-                    stop = true;
-                    break;
-                }
-                uint8_t *st = stages + s * kStageBytes;
-                const uint4 *src = reinterpret_cast<const uint4 *>(st + kOffCodes + row * 32);
-                const uint4 c0 = src[0], c1 = src[1];
-                const __half2 sz = *reinterpret_cast<const __half2 *>(st + kOffSz + row * 4);
-                const float sc = __low2float(sz), zp = __high2float(sz);
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint8_t *arow = st + kOffA + (row >> 3) * 1024 + swz * 128;
-#pragma unroll
-                for (int cidx = 0; cidx < 8; ++cidx) {
-                    // 8 channels: bytes 4c..4c+3, low nibble first.
-                    const uint32_t w = words[cidx];
-                    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-                    uint32_t out[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float qe = small_uint_to_float((lo >> (8 * i)) & 0xFFu);
-                        const float qo = small_uint_to_float((hi >> (8 * i)) & 0xFFu);
-                        out[i] = pack_bf16x2(__fmaf_rn(qe, sc, zp), __fmaf_rn(qo, sc, zp));
+        if (warp >= kDeqWarp0) {
+            const int row = threadIdx.x - kDeqWarp0 * 32;  // token row of the tile, 0..127
+            const uint32_t swz = row & 7;
+            int it = 0;
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < n_total && !stop; tile += gridDim.x) {
+                for (int kb = 0; kb < n_k; ++kb, ++it) {
+                    const int sc = it % kCStages, rc = it / kCStages;
+                    // Warp-uniform outcomes: the warp's later steps need all lanes.
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c_full[sc], rc & 1, p.timeout_ns,
+                                                                   p.status, abort_flag))) {
+                        stop = true;
+                        break;
                     }
-                    *reinterpret_cast<uint4 *>(arow + ((cidx ^ swz) << 4)) =
-                        make_uint4(out[0], out[1], out[2], out[3]);
+                    const uint8_t *cs = c_ring + sc * kCStageBytes;
+                    uint4 c0, c1;
+                    uint32_t szw;
+                    lds_codes(cs + row * 32, cs + kCodeBytes + row * 4, c0, c1, szw);
+                    const int sa = it % kAStages, ra = it / kAStages;
+                    if (ra > 0 &&
+                        !__all_sync(0xffffffffu, mbar_wait_bounded(&a_empty[sa], (ra - 1) & 1,
+                                                                   p.timeout_ns, p.status, abort_flag))) {
+                        stop = true;
+                        break;
+                    }
+                    const __half2 sz = *reinterpret_cast<const __half2 *>(&szw);
+                    uint8_t *arow = a_ring + sa * kABytes + (row >> 3) * 1024 + swz * 128;
+                    dequant_row(c0, c1, __low2float(sz), __high2float(sz), arow, swz);
+                    // Every writer fences its own stores for the async proxy and
+                    // arrives itself: the tensor core must see all 128 rows.
+                    fence_proxy_async_smem();
+                    mbar_arrive(&a_full[sa]);
+                    // Release the codes slot only now. A shared load returns its
+                    // data asynchronously and an arrive issued right after it
+                    // does not wait for that data; the arithmetic above consumed
+                    // the loaded registers, and warps issue in order, so the
+                    // loads have completed before this arrive can issue.
+                    mbar_arrive(&c_empty[sc]);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full_a[s]);
             }
         }
     } else {
@@ -407,8 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[j]);
+            mbar_arrive(&acc_empty[j]);
         }
     }
 

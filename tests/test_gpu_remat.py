@@ -28,13 +28,13 @@ def _inputs(seed, B, T, hidden, H):
     return xs, w
 
 
-def _x_cache(xs, cap):
+def _x_cache(xs, cap, dtype="bf16"):
     B = len(xs)
     T, hidden = xs[0].shape
     XH = hidden // D
     cache = K.KVCache(K.CacheSpec(B, XH, bits_k=4, group_k=128, capacity_tokens=cap, with_v=False))
     lens = lens_tensor([0] * B)
-    append(cache, [x.reshape(T, XH, D) for x in xs], None, lens)
+    append(cache, [x.reshape(T, XH, D) for x in xs], None, lens, dtype=dtype)
     return cache
 
 
@@ -146,6 +146,30 @@ def test_remat_position_zero_and_identity_weights():
     xhat = oracle.dequant_x_bf16(codes, sz, 128, 4)[:, :D]
     assert np.array_equal(v_out[0, 0].float().cpu().numpy(), xhat)
     assert np.array_equal(k_out[0, 0, 0].float().cpu().numpy(), xhat[0])
+
+
+def test_remat_dequant_exact_on_awkward_groups():
+    # Groups far from zero with a small range, and groups spanning a large
+    # range above a tiny (or fp16-subnormal) minimum, where z - 128 s is not
+    # exact in fp32: the dequantized X must still equal the oracle's
+    # bf16_rn(fp32(q*s + z)) bit for bit (V = X^ through identity weights).
+    B, T, hidden, H = 1, 128, 256, 1
+    g = np.random.default_rng(4)
+    x = W.normal(g, (T, hidden))
+    x[0::4] = 1000.0 + 0.01 * x[0::4]
+    x[1::4] = -3000.0 + 0.003 * x[1::4]
+    x[2::4] = np.abs(x[2::4]) * 500.0
+    x[2::4, ::128] = 1e-4
+    x[3::4] = np.abs(x[3::4]) * 500.0
+    x[3::4, ::128] = -2e-5
+    xs = [np.ascontiguousarray(x, np.float32)]
+    w = np.zeros((2 * H * D, hidden), np.float32)
+    w[D + np.arange(D), np.arange(D)] = 1.0
+    cache = _x_cache(xs, T, dtype="fp32")
+    _, v_out = _remat(cache, w, H, B, T)
+    codes, sz = oracle.quantize_tokens(xs[0], 0, 128, 4)
+    xhat = oracle.dequant_x_bf16(codes, sz, 128, 4)[:, :D]
+    assert np.array_equal(v_out[0, 0].float().cpu().numpy(), xhat)
 
 
 def test_attention_over_rematerialized_kv():
