@@ -59,6 +59,16 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
 def source_hash(path):
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
@@ -291,6 +301,84 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
+# ---------------------------------------------------------------------------
+# XQuant rematerialization leg: 8 sequences x 16384 positions, hidden 4096,
+# 8 KV heads / 32 query heads. One step = kvq_remat_kv over the whole context
+# (dequantize X, tensor-core GEMM, RoPE) + decode attention over the bf16 K/V.
+# ---------------------------------------------------------------------------
+XQ_T, XQ_HIDDEN, XQ_H, XQ_HQ = 16384, 4096, 8, 32
+
+
+def run_remat(args, dev):
+    import torch
+    import bit_kv_cache_21_b200 as K
+
+    B, T, hidden, H = args.remat_batch, XQ_T, XQ_HIDDEN, XQ_H
+    XH = hidden // D
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    cache = K.KVCache(K.CacheSpec(B, XH, bits_k=4, group_k=128, capacity_tokens=T, with_v=False),
+                      device=dev)
+    lens = torch.zeros(B, dtype=torch.int32, device=dev)
+    for b in range(B):   # X ~ N(0, 1) bf16, one sequence at a time
+        x = torch.randn((T, XH, D), generator=gen, device=dev).to(torch.bfloat16)
+        cu = torch.zeros(B + 1, dtype=torch.int32, device=dev)
+        cu[b + 1:] = T
+        K.quantize_append(cache.desc, x, None, cu, lens)
+        del x
+    w = (torch.randn((2 * H * D, hidden), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+    q = torch.randn((B, XQ_HQ, D), generator=gen, device=dev).to(torch.bfloat16)
+    cos, sin = K.rope_tables(T, D, 500000.0, device=dev)
+    k_out = torch.empty((B, H, T, D), dtype=torch.bfloat16, device=dev)
+    v_out = torch.empty_like(k_out)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    desc = K.bf16_cache_desc(k_out, v_out, status)
+    full = torch.full((B,), T, dtype=torch.int32, device=dev)
+    ws = torch.empty(K.decode_workspace_size(desc, B, XQ_HQ, T), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, XQ_HQ, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(D)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        K.remat_kv(cache.desc, w, H, cos, sin, B, T, k_out, v_out)
+        if evs:
+            evs[1].record(stream)
+        K.decode_attention(desc, q, full, T, scale, out=out, workspace=ws)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.remat_steps)]
+    for i in range(args.remat_steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0 and int(status[0]) == 0
+    remat_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    flops = 2.0 * B * T * (2 * H * D) * hidden
+    kv_bytes = 2.0 * B * H * T * D * 2
+    peak_b, peak_s, kind = tensor_peaks()
+    tflops = flops / (remat_ms * 1e-3) / 1e12
+    return {"workload": "xquant: %d seqs x %d positions, hidden %d, X INT4 g128, W_k/W_v %dx%d "
+                        "bf16, RoPE theta 500000, then GQA decode attention %d q / %d kv heads "
+                        "over the bf16 K/V" % (B, T, hidden, hidden, H * D, XQ_HQ, H),
+            "steps": args.remat_steps, "ms_per_step": remat_ms + attn_ms,
+            "remat": {"kernel": "remat_kernel", "bound": "tensor", "ms": remat_ms,
+                      "flops_per_launch": flops, "achieved": tflops, "unit": "TFLOP/s",
+                      "peak": peak_b, "peak_kind": kind + " bf16 burst", "frac": tflops / peak_b,
+                      "frac_of_sustained": tflops / peak_s},
+            "attention_bf16": {"ms": attn_ms, "bytes": kv_bytes,
+                               "GBps": kv_bytes / (attn_ms * 1e-3) / 1e9},
+            "gpu_launches_per_step": 4}
+
+
 def cpu_units(n_units, seed=0):
     """Oracle-side cache state of n_units (sequence, KV head) units of the
     workload at context 8193: the oracle's own packed K/V and 4 queries."""
@@ -333,6 +421,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--part", default="all", choices=["all", "decode", "remat"],
+                    help="remat: only the XQuant rematerialization leg (prints its own line)")
+    ap.add_argument("--remat-batch", type=int, default=8)
+    ap.add_argument("--remat-steps", type=int, default=10)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -377,7 +469,21 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    if args.part == "remat":
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        rr = run_remat(args, dev)
+        if rank == 0:
+            print(json.dumps({"metric": "remat TFLOP/s (tensor cores)", "value": rr["remat"]["achieved"],
+                              "unit": "TFLOP/s", "n_gpus": world, "higher_is_better": True,
+                              "data": "synthetic", "dtype": "bf16 MMA, fp32 accumulate",
+                              "config": {"workload": rr["workload"]}, "remat_leg": rr}))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     res = run_ours(args, rank, world, local_rank)
+    rr = run_remat(args, torch.device("cuda", local_rank)) if args.part == "all" else None
 
     # max over ranks of the device time; bytes summed over ranks
     total_ms, total_bytes, e2e_s, e2e_bytes = res["total_ms"], res["bytes"], res["e2e_s"], res["e2e_bytes"]
@@ -421,6 +527,8 @@ def main():
             "gpu_launches": 4 * args.steps,
             "clocks": res["clocks"],
         }
+        if rr is not None:
+            line["xquant_remat"] = rr
         print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()
