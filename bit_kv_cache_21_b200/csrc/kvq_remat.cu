@@ -11,20 +11,21 @@
 // Tiles are 128 tokens x 256 output channels (two heads of K or V); one CTA
 // per SM walks the tiles. Warp roles:
 //   warp 0      W producer: per 64-wide K step, a TMA box of W (256 x 64
-//               bf16, 128-byte swizzle). No multicast.
+//               bf16, 128-byte swizzle) into shared memory. No multicast.
 //   warp 2      codes producer: the X codes box (128 tokens x 32 bytes) and
 //               the tokens' fp16 scale/zero (512 bytes).
-//   warp 1      allocates 512 TMEM columns (two 256-column fp32
-//               accumulators); one lane issues tcgen05.mma (kind::f16, bf16
-//               operands, M=128, N=256, K=16); tcgen05.commit frees the W and
-//               A slots and signals a finished accumulator.
-//   warps 3-6   dequantize the codes into the A operand (128 x 64 bf16) in the
-//               same 128-byte-swizzled K-major layout TMA gives W, one token
-//               row per thread, then fence the generic-proxy writes for the
-//               tensor core.
-//   warps 7-10  epilogue: tcgen05.ld one accumulator row per thread, RoPE in
-//               fp32 on K, round to bf16, store [B][H][T][128]. Two accumulators
-//               let the epilogue of one tile overlap the main loop of the next.
+//   warp 1      allocates 512 TMEM columns (one 256-column fp32 accumulator
+//               and a ring of A stages); one lane issues tcgen05.mma
+//               (kind::f16, A from tensor memory, B from shared memory);
+//               tcgen05.commit frees W and A stages and signals the finished
+//               accumulator.
+//   warps 3-10  dequantize the codes, one token row per thread, in two groups
+//               of four warps taking alternate K steps, and store the bf16 A
+//               operand into tensor memory with tcgen05.st.
+//   warps 11-14 epilogue: tcgen05.ld one accumulator row per thread, RoPE in
+//               fp32 on K, round to bf16 into a swizzled shared staging tile,
+//               release the accumulator; one thread stores the tile to
+//               [B][H][T][128] with TMA while the next tile's main loop runs.
 // Every mbarrier wait is bounded; on expiry the kernel sets KVQ_DEV_TIMEOUT,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
 #include <cuda.h>
@@ -44,37 +45,47 @@ constexpr int kBM = 128;                    // tokens per tile (MMA M)
 constexpr int kBN = 256;                    // output channels per tile (MMA N)
 constexpr int kBK = 64;                     // hidden channels per stage (one 128-byte row)
 constexpr int kUmmaK = 16;                  // K of one tcgen05.mma kind::f16
-// Three rings, each recycled by its own consumer, so that no ring's refill
-// waits for more than one step of the chain TMA -> dequantize -> MMA:
-//   W ring      (TMA -> MMA, freed by tcgen05.commit)
-//   A ring      (dequantizers -> MMA, freed by tcgen05.commit)
-//   codes ring  (TMA -> dequantizers, freed as soon as they hold the codes)
+// Pipelines, each recycled by its own consumer:
+//   W ring      shared memory, TMA -> MMA, freed by tcgen05.commit
+//   codes ring  shared memory, TMA -> dequantizers, freed once they hold the codes
+//   A ring      tensor memory, dequantizers (tcgen05.st) -> MMA, freed by tcgen05.commit
+// Keeping the A operand in tensor memory takes its writes and the tensor
+// core's reads of it off shared-memory bandwidth, which otherwise bounds the
+// loop (the W and codes traffic alone use most of it).
 constexpr int kWStages = 4;
-constexpr int kAStages = 3;
-constexpr int kCStages = 8;
+constexpr int kAStages = 4;
+constexpr int kCStages = 6;
 constexpr int kBBytes = kBN * kBK * 2;      // 32 KiB of W per stage
-constexpr int kABytes = kBM * kBK * 2;      // 16 KiB of bf16 x^ per stage
 constexpr int kCodeBytes = kBM * kBK / 2;   // 4 KiB of INT4 codes
 constexpr int kSzBytes = kBM * 4;           // half2 per token
 constexpr int kCStageBytes = kCodeBytes + kSzBytes;
-constexpr int kOffARing = kWStages * kBBytes;
-constexpr int kOffCRing = kOffARing + kAStages * kABytes;
-constexpr int kRingBytes = kOffCRing + kCStages * kCStageBytes;
+constexpr int kOffCRing = kWStages * kBBytes;
+constexpr int kOffStage = kOffCRing + kCStages * kCStageBytes;
+// Output staging: 2 heads x 2 boxes of 128 rows x 64 bf16 (128-byte swizzle).
+constexpr int kBoxBytes = kBM * 64 * 2;
+constexpr int kStageOutBytes = 4 * kBoxBytes;
+constexpr int kRingBytes = kOffStage + kStageOutBytes;
+// Tensor memory: one fp32 accumulator of 256 columns, then the A stages of
+// 64 bf16 per row = 32 columns each.
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = 256;
+constexpr int kACols = kBK / 2;
+static_assert(kAccCols + kAStages * kACols <= kTmemCols, "tensor memory");
 // warps: 0 W producer, 1 MMA issuer (+ TMEM owner), 2 codes producer,
-// 3-6 dequantizers, 7-10 epilogue
+// 3-10 dequantizers (two groups of four taking alternate K steps), 11-14 epilogue
 constexpr int kDeqWarp0 = 3;
-constexpr int kEpiWarp0 = 7;
-constexpr int kThreads = 11 * 32;
-constexpr int kNumBars = 2 * kWStages + 2 * kAStages + 2 * kCStages + 5;
+constexpr int kDeqGroups = 2;
+constexpr int kEpiWarp0 = kDeqWarp0 + 4 * kDeqGroups;
+constexpr int kThreads = (kEpiWarp0 + 4) * 32;
+constexpr int kNumBars = 2 * kWStages + 2 * kAStages + 2 * kCStages + 3;
 constexpr int kBarBytes = 512;
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kRingBytes) + kBarBytes;
 
-static_assert(kOffARing % 1024 == 0 && kABytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(kBBytes % 1024 == 0 && kOffStage % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kOffCRing % 128 == 0 && kCStageBytes % 128 == 0, "TMA destination alignment");
 static_assert(kNumBars * 8 + 8 <= kBarBytes, "barrier area");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kCStages % kDeqGroups == 0, "a codes slot always goes to the same group");
 
 struct RematParams {
     const __half2 *x_sz;   // [S][XH][Tc] (one group of 128 channels per row)
@@ -133,13 +144,32 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t accumulate) {
+// One tcgen05.mma kind::f16 (M 128, N 256, K 16, fp32 accumulate into
+// d_tmem) with the A operand read from tensor memory (lane = row, 32-bit column
+// c = bf16 elements 2c and 2c+1 along K) and B from a shared-memory descriptor.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(kInstrDesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(kInstrDesc), "r"(accumulate)
+        : "memory");
+}
+
+// Store 32 consecutive 32-bit columns of this thread's TMEM lane and wait for
+// the store to complete.
+__device__ __forceinline__ void tmem_st32_wait(uint32_t taddr, const uint32_t v[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
 }
 
@@ -182,6 +212,22 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
         : "memory");
 }
+
+// 2-D tiled TMA store shared -> global (bulk group of the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, const void *src) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(smem_addr(src))
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the issued bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until the issued bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -227,15 +273,15 @@ __device__ __forceinline__ void lds_codes(const uint8_t *codes, const uint8_t *s
 }
 
 // Dequantize one token row's 64 INT4 codes (32 bytes, element 2i in the low
-// nibble of byte i) into 64 bf16 x^ = bf16_rn(fp32(q*s + z)), written as the
-// row's eight 16-byte chunks of a 128-byte-swizzled K-major tile.
+// nibble of byte i) into 64 bf16 x^ = bf16_rn(fp32(q*s + z)), packed two per
+// word in K order: out[c] = {x^[2c] (low half), x^[2c+1]}, the row's 32
+// tensor-memory columns of the A operand.
 //
 // Fast form: a byte permute puts nibble q in the top mantissa bits of 1.0,
 // f = 1 + q/128 exactly, and fma(f, 128 s, z - 128 s) equals q*s + z before
 // its single rounding whenever z - 128 s is exact in fp32 (checked per row);
 // otherwise the codes go through 2^23 + q - 2^23 and fma(q, s, z).
-__device__ __forceinline__ void dequant_row(uint4 c0, uint4 c1, float sc, float zp, uint8_t *arow,
-                                            uint32_t swz) {
+__device__ __forceinline__ void dequant_row(uint4 c0, uint4 c1, float sc, float zp, uint32_t out[32]) {
     const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
     const float s128 = __fmul_rn(sc, 128.0f);
     const float cz = __fsub_rn(zp, s128);
@@ -246,7 +292,6 @@ __device__ __forceinline__ void dequant_row(uint4 c0, uint4 c1, float sc, float 
             const uint32_t w = words[c];
             const uint32_t lo = (w & 0x0F0F0F0Fu) | 0x80808080u;
             const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-            uint32_t out[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 // bytes {0, 0, 0x80|q, 0x3F}: the float 1 + q/128
@@ -254,25 +299,22 @@ __device__ __forceinline__ void dequant_row(uint4 c0, uint4 c1, float sc, float 
                 const float2 f = make_float2(__uint_as_float(prmt(lo, 0x3F000000u, sel)),
                                              __uint_as_float(prmt(hi, 0x3F000000u, sel)));
                 const float2 x = ffma2(f, mul, add);
-                out[i] = pack_bf16x2(x.x, x.y);
+                out[4 * c + i] = pack_bf16x2(x.x, x.y);
             }
-            *reinterpret_cast<uint4 *>(arow + ((c ^ swz) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
         }
     } else {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const uint32_t w = words[c];
             const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-            uint32_t out[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 // bytes {q, 0, 0, 0x4B}: the float 2^23 + q
                 const uint32_t sel = 0x7440u | static_cast<uint32_t>(i);
                 const float qe = __fsub_rn(__uint_as_float(prmt(lo, 0x4B000000u, sel)), 8388608.0f);
                 const float qo = __fsub_rn(__uint_as_float(prmt(hi, 0x4B000000u, sel)), 8388608.0f);
-                out[i] = pack_bf16x2(__fmaf_rn(qe, sc, zp), __fmaf_rn(qo, sc, zp));
+                out[4 * c + i] = pack_bf16x2(__fmaf_rn(qe, sc, zp), __fmaf_rn(qo, sc, zp));
             }
-            *reinterpret_cast<uint4 *>(arow + ((c ^ swz) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
         }
     }
 }
@@ -294,23 +336,24 @@ __device__ __forceinline__ TileCoord tile_coord(const RematParams &p, int tile) 
 
 __global__ void __launch_bounds__(kThreads, 1)
     remat_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const RematParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *w_ring = smem;
-    uint8_t *a_ring = smem + kOffARing;
     uint8_t *c_ring = smem + kOffCRing;
+    uint8_t *out_stage = smem + kOffStage;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
     uint64_t *w_full = bars;                       // [kWStages] W landed (tx)
     uint64_t *w_empty = w_full + kWStages;         // [kWStages] MMAs done with W
-    uint64_t *a_full = w_empty + kWStages;         // [kAStages] x^ written (128 threads)
+    uint64_t *a_full = w_empty + kWStages;         // [kAStages] x^ stored (128 threads)
     uint64_t *a_empty = a_full + kAStages;         // [kAStages] MMAs done with x^
     uint64_t *c_full = a_empty + kAStages;         // [kCStages] codes landed (tx)
     uint64_t *c_empty = c_full + kCStages;         // [kCStages] codes taken (128 threads)
-    uint64_t *acc_full = c_empty + kCStages;       // [2] accumulator ready
-    uint64_t *acc_empty = acc_full + 2;            // [2] accumulator drained (128 threads)
-    uint64_t *mma_done = acc_empty + 2;            // [1] every MMA of this CTA finished
+    uint64_t *acc_full = c_empty + kCStages;       // accumulator ready
+    uint64_t *acc_empty = acc_full + 1;            // accumulator drained (128 threads)
+    uint64_t *mma_done = acc_empty + 1;            // every MMA of this CTA finished
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -329,10 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&c_full[s], 1);
             mbar_init(&c_empty[s], 128);
         }
-        for (int j = 0; j < 2; ++j) {
-            mbar_init(&acc_full[j], 1);
-            mbar_init(&acc_empty[j], 128);
-        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 128);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -409,12 +450,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0, lt = 0;
             bool stop = false;
             for (int tile = blockIdx.x; tile < n_total && !stop; tile += gridDim.x, ++lt) {
-                const int j = lt & 1, u = lt >> 1;
-                if (u > 0 && !mbar_wait_bounded(&acc_empty[j], (u - 1) & 1, p.timeout_ns, p.status,
-                                                abort_flag))
+                // one accumulator: the previous tile's epilogue must have drained it
+                if (lt > 0 && !mbar_wait_bounded(acc_empty, (lt - 1) & 1, p.timeout_ns, p.status,
+                                                 abort_flag))
                     break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + j * kAccCols;
                 for (int kb = 0; kb < n_k; ++kb, ++it) {
                     const int sw = it % kWStages, rw = it / kWStages;
                     const int sa = it % kAStages, ra = it / kAStages;
@@ -424,18 +464,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t a_desc = sw128_desc(smem_addr(a_ring + sa * kABytes));
+                    const uint32_t a_tmem = tmem_base + kAccCols + sa * kACols;
                     const uint64_t b_desc = sw128_desc(smem_addr(w_ring + sw * kBBytes));
 #pragma unroll
                     for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                        // +32 bytes along K inside the swizzle atom = +2 in the
-                        // descriptor's 16-byte address units.
-                        umma_bf16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, (kb | kk) != 0);
+                        // K step of 16: 8 tensor-memory columns of A; +32 bytes
+                        // inside the W swizzle atom = +2 in descriptor units.
+                        umma_bf16_ts(tmem_base, a_tmem + kk * (kUmmaK / 2), b_desc + 2 * kk,
+                                     (kb | kk) != 0);
                     }
                     umma_commit(&w_empty[sw]);
                     umma_commit(&a_empty[sa]);
                 }
-                if (!stop) umma_commit(&acc_full[j]);
+                if (!stop) umma_commit(acc_full);
             }
             // Every MMA issued must finish before TMEM is freed.
             umma_commit(mma_done);
@@ -449,70 +490,85 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kEpiWarp0) {
         // ------------------------------ dequantizers ------------------------------
-        if (warp >= kDeqWarp0) {
-            const int row = threadIdx.x - kDeqWarp0 * 32;  // token row of the tile, 0..127
-            const uint32_t swz = row & 7;
-            int it = 0;
-            bool stop = false;
-            for (int tile = blockIdx.x; tile < n_total && !stop; tile += gridDim.x) {
-                for (int kb = 0; kb < n_k; ++kb, ++it) {
-                    const int sc = it % kCStages, rc = it / kCStages;
-                    // Warp-uniform outcomes: the warp's later steps need all lanes.
-                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c_full[sc], rc & 1, p.timeout_ns,
-                                                                   p.status, abort_flag))) {
-                        stop = true;
-                        break;
-                    }
-                    const uint8_t *cs = c_ring + sc * kCStageBytes;
-                    uint4 c0, c1;
-                    uint32_t szw;
-                    lds_codes(cs + row * 32, cs + kCodeBytes + row * 4, c0, c1, szw);
-                    const int sa = it % kAStages, ra = it / kAStages;
-                    if (ra > 0 &&
-                        !__all_sync(0xffffffffu, mbar_wait_bounded(&a_empty[sa], (ra - 1) & 1,
-                                                                   p.timeout_ns, p.status, abort_flag))) {
-                        stop = true;
-                        break;
-                    }
-                    const __half2 sz = *reinterpret_cast<const __half2 *>(&szw);
-                    uint8_t *arow = a_ring + sa * kABytes + (row >> 3) * 1024 + swz * 128;
-                    dequant_row(c0, c1, __low2float(sz), __high2float(sz), arow, swz);
-                    // Every writer fences its own stores for the async proxy and
-                    // arrives itself: the tensor core must see all 128 rows.
-                    fence_proxy_async_smem();
-                    mbar_arrive(&a_full[sa]);
-                    // Release the codes slot only now. A shared load returns its
-                    // data asynchronously and an arrive issued right after it
-                    // does not wait for that data; the arithmetic above consumed
-                    // the loaded registers, and warps issue in order, so the
-                    // loads have completed before this arrive can issue.
-                    mbar_arrive(&c_empty[sc]);
+        // Group g takes the K steps it with it % kDeqGroups == g; each of its
+        // four warps owns the 32 rows (tensor-memory lanes) of its quarter.
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;  // token row of the tile = TMEM lane
+        const int group = (warp - kDeqWarp0) >> 2;
+        const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kAccCols;
+        int it = 0;
+        bool stop = false;
+        for (int tile = blockIdx.x; tile < n_total && !stop; tile += gridDim.x) {
+            for (int kb = 0; kb < n_k; ++kb, ++it) {
+                if (it % kDeqGroups != group) continue;
+                const int sc = it % kCStages, rc = it / kCStages;
+                // Warp-uniform outcomes: the warp's later steps need all lanes.
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(&c_full[sc], rc & 1, p.timeout_ns,
+                                                               p.status, abort_flag))) {
+                    stop = true;
+                    break;
                 }
+                const uint8_t *cs = c_ring + sc * kCStageBytes;
+                uint4 c0, c1;
+                uint32_t szw;
+                lds_codes(cs + row * 32, cs + kCodeBytes + row * 4, c0, c1, szw);
+                const __half2 sz = *reinterpret_cast<const __half2 *>(&szw);
+                uint32_t xv[32];
+                dequant_row(c0, c1, __low2float(sz), __high2float(sz), xv);
+                // Release the codes slot only now. A shared load returns its
+                // data asynchronously and an arrive issued right after it does
+                // not wait for that data; the arithmetic above consumed the
+                // loaded registers, and warps issue in order, so the loads have
+                // completed before this arrive can issue.
+                mbar_arrive(&c_empty[sc]);
+                const int sa = it % kAStages, ra = it / kAStages;
+                if (ra > 0 &&
+                    !__all_sync(0xffffffffu, mbar_wait_bounded(&a_empty[sa], (ra - 1) & 1,
+                                                               p.timeout_ns, p.status, abort_flag))) {
+                    stop = true;
+                    break;
+                }
+                tc_fence_after();
+                tmem_st32_wait(a_lane + sa * kACols, xv);
+                tc_fence_before();
+                mbar_arrive(&a_full[sa]);
             }
         }
     } else {
         // ------------------------------ epilogue ----------------------------------
+        // Drain the accumulator into a swizzled bf16 staging tile (RoPE on K
+        // applied on the way), release the accumulator, then one thread
+        // stores the tile with four TMA copies while the next tile's main loop
+        // runs.
         const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;
+        const bool leader = (warp == kEpiWarp0 && lane == 0);
+        const uint32_t swz = row & 7;
         int lt = 0;
+        bool ok = true;
         for (int tile = blockIdx.x; tile < n_total; tile += gridDim.x, ++lt) {
-            const int j = lt & 1, u = lt >> 1;
-            // Warp-uniform outcome: tcgen05.ld needs the whole warp.
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&acc_full[j], u & 1, p.timeout_ns,
-                                                           p.status, abort_flag)))
-                break;
+            // Warp-uniform outcome (tcgen05.ld needs the whole warp). After a
+            // failed wait the warp skips the work but still takes both named
+            // barriers of every tile, so no epilogue warp is left waiting.
+            ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(acc_full, lt & 1, p.timeout_ns,
+                                                                 p.status, abort_flag));
             tc_fence_after();
+            // The staging tile is free once the previous tile's stores read it.
+            if (leader) bulk_wait_read();
+            named_sync(1, 128);
+            if (!ok) {
+                named_sync(1, 128);
+                continue;
+            }
             const TileCoord c = tile_coord(p, tile);
             const int t = c.t0 + row;
-            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + j * kAccCols;
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
-                const int slot = c.n * 2 + half;  // K heads 0..H-1, then V heads
-                const bool is_k = slot < p.H;
-                const int h = is_k ? slot : slot - p.H;
-                uint16_t *dst = (is_k ? p.k_out : p.v_out) +
-                                ((static_cast<int64_t>(c.b) * p.H + h) * p.T + t) * kHeadDim;
+                const bool is_k = c.n * 2 + half < p.H;  // K heads 0..H-1, then V heads
                 const uint32_t col = tbase + half * kHeadDim;
+                uint8_t *box0 = out_stage + (half * 2) * kBoxBytes + row * 128;
+                uint8_t *box1 = box0 + kBoxBytes;
 #pragma unroll 1
                 for (int c32 = 0; c32 < 64; c32 += 32) {
                     float a[32], bv[32];
@@ -534,20 +590,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
-                    uint4 *d0 = reinterpret_cast<uint4 *>(dst + c32);
-                    uint4 *d1 = reinterpret_cast<uint4 *>(dst + 64 + c32);
+                    // channels c32 .. c32+31 -> box 0, 64+c32 .. -> box 1; 16-byte
+                    // chunk j of a row sits at chunk j ^ (row & 7)
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
-                        d0[v] = make_uint4(pack_bf16x2(a[8 * v + 0], a[8 * v + 1]), pack_bf16x2(a[8 * v + 2], a[8 * v + 3]),
-                                           pack_bf16x2(a[8 * v + 4], a[8 * v + 5]), pack_bf16x2(a[8 * v + 6], a[8 * v + 7]));
-                        d1[v] = make_uint4(pack_bf16x2(bv[8 * v + 0], bv[8 * v + 1]), pack_bf16x2(bv[8 * v + 2], bv[8 * v + 3]),
-                                           pack_bf16x2(bv[8 * v + 4], bv[8 * v + 5]), pack_bf16x2(bv[8 * v + 6], bv[8 * v + 7]));
+                        const uint32_t j = static_cast<uint32_t>(c32 / 8 + v);
+                        *reinterpret_cast<uint4 *>(box0 + ((j ^ swz) << 4)) =
+                            make_uint4(pack_bf16x2(a[8 * v + 0], a[8 * v + 1]), pack_bf16x2(a[8 * v + 2], a[8 * v + 3]),
+                                       pack_bf16x2(a[8 * v + 4], a[8 * v + 5]), pack_bf16x2(a[8 * v + 6], a[8 * v + 7]));
+                        *reinterpret_cast<uint4 *>(box1 + ((j ^ swz) << 4)) =
+                            make_uint4(pack_bf16x2(bv[8 * v + 0], bv[8 * v + 1]), pack_bf16x2(bv[8 * v + 2], bv[8 * v + 3]),
+                                       pack_bf16x2(bv[8 * v + 4], bv[8 * v + 5]), pack_bf16x2(bv[8 * v + 6], bv[8 * v + 7]));
                     }
                 }
             }
+            // Accumulator read out: the next tile's MMAs may start.
             tc_fence_before();
-            mbar_arrive(&acc_empty[j]);
+            mbar_arrive(acc_empty);
+            fence_proxy_async_smem();
+            named_sync(1, 128);
+            if (leader && ok) {
+                for (int half = 0; half < 2; ++half) {
+                    const int slot = c.n * 2 + half;
+                    const bool is_k = slot < p.H;
+                    const int h = is_k ? slot : slot - p.H;
+                    const int y = (c.b * p.H + h) * p.T + c.t0;
+                    const CUtensorMap *map = is_k ? &tm_k : &tm_v;
+                    tma_store_2d(map, 0, y, out_stage + (half * 2) * kBoxBytes);
+                    tma_store_2d(map, 64, y, out_stage + (half * 2 + 1) * kBoxBytes);
+                }
+                bulk_commit();
+            }
         }
+        if (leader) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -628,6 +703,16 @@ kvq_status launch_remat(const kvq_cache_desc &x, const void *w_kv, int n_kv_head
         !make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, x.k_codes, kHeadDim / 2, code_rows,
                      kHeadDim / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
         return KVQ_ERR_CUDA;
+    // Outputs [B][H][T][128] bf16 as rows of 128 channels, stored in boxes of
+    // 128 positions x 64 channels.
+    const int64_t out_rows = static_cast<int64_t>(batch) * n_kv_heads * ctx_len;
+    if (out_rows >= (1LL << 31)) return KVQ_ERR_UNSUPPORTED;
+    CUtensorMap tm_k, tm_v;
+    if (!make_map_2d(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k_out, kHeadDim, out_rows, kHeadDim * 2,
+                     64, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v_out, kHeadDim, out_rows, kHeadDim * 2,
+                     64, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return KVQ_ERR_CUDA;
     RematParams p{};
     p.x_sz = static_cast<const __half2 *>(x.k_sz);
     p.rope_cos = rope_cos;
@@ -652,7 +737,7 @@ kvq_status launch_remat(const kvq_cache_desc &x, const void *w_kv, int n_kv_head
     const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
     if (tiles >= (1LL << 31)) return KVQ_ERR_UNSUPPORTED;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
-    remat_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_w, tm_x, p);
+    remat_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_w, tm_x, tm_k, tm_v, p);
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
