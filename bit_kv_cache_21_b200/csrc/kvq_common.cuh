@@ -85,6 +85,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Same test, but a thread whose phase is not complete may be suspended (it
+// issues nothing) until the phase completes or about `hint_ns` pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Suspend hint of the bounded waits: waiters sleep in hardware instead of
+// re-polling; the timeout and the abort flag are checked once per wake-up.
+constexpr uint32_t kWaitSleepNs = 200000;
+
 // Wait until the phase of `bar` with the given parity has completed, or until
 // `timeout_ns` passes (then OR KVQ_DEV_TIMEOUT into *status and raise the
 // CTA's abort flag), or until another thread raised the abort flag.
@@ -95,7 +113,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
         if (*abort_flag) return false;
         if (static_cast<int64_t>(global_timer_ns() - t0) > timeout_ns) {
             status_or(status, KVQ_DEV_TIMEOUT);

@@ -46,9 +46,10 @@ namespace kvq {
 
 namespace {
 
-constexpr int kTile = 64;          // tokens per quantized tile
+constexpr int kTile = 128;         // tokens per quantized tile
 constexpr int kWinTile = 16;       // tokens per bf16 window tile (quantized caches)
 constexpr int kConsumerWarps = 4;
+constexpr int kTokensPerWarp = kTile / kConsumerWarps;  // of a quantized tile
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -90,6 +91,7 @@ struct DecodeParams {
     // shared-memory stage layout (bytes)
     int stage_bytes, off_ksz, off_vc, off_vsz, off_q, off_hdr;
     int bf_tile, bf_off_v;  // bf16 tiles: tokens per tile, offset of the V rows
+    int wsm_floats;         // per-warp value-weight scratch: tokens x value groups x GQA x 2
     int64_t timeout_ns;
     int skip_tile;
 };
@@ -316,8 +318,9 @@ struct QueryRegs {
 };
 
 // One tile: rows at kc / ks / vc / vs (shared memory), `n` valid tokens, TPW
-// tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)).
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW, int GK, int GV, int VSLOTS>
+// tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)). FULL: all
+// 4*TPW tokens are valid, so no token needs masking.
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW, int GK, int GV, int VSLOTS, bool FULL>
 __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
                                              const uint8_t *vc, const uint8_t *vs, int n,
                                              const Geo<GK, GV, GQA> geo, const QueryRegs<GQA> &Q,
@@ -341,7 +344,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 #pragma unroll
     for (int pass = 0; pass < PASSES; ++pass) {
         const int tt = t_warp + pass * 4 + i;
-        const int tr = tt < n ? tt : 0;  // masked tokens read row 0 (always staged)
+        const int tr = (FULL || tt < n) ? tt : 0;  // masked tokens read row 0 (always staged)
         float2 f[8];
         key_pairs<KM, KBITS>(kc + tr * KROW, part, f);
         float acc[GQA];
@@ -390,7 +393,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
         if constexpr (KM == K_TOKEN) {
             if (post_scale) val = fmaf(szf.x, fmaf(-128.0f, Q.qe_own, val), szf.y * Q.qa_own);
         }
-        sc[pass] = tt < n ? val : -INFINITY;
+        sc[pass] = (FULL || tt < n) ? val : -INFINITY;
     }
 
     // ---- online softmax (per warp, per head), lazy rescaling ----
@@ -424,7 +427,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     for (int pass = 0; pass < PASSES; ++pass) {
         const int j = pass * 4 + i;  // warp-local token index
         const int tt = t_warp + j;
-        const int tr = tt < n ? tt : 0;
+        const int tr = (FULL || tt < n) ? tt : 0;
         float2 *wrow = reinterpret_cast<float2 *>(wsm) + j * n_vg * GQA;
         if constexpr (VM == V_BF16) {
             if (r_own == 0) wrow[h_own] = make_float2(p[pass], p[pass]);
@@ -467,7 +470,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     for (int k = 0; k < TPW / 2; ++k) {
         const int j = 2 * k + parity;
         const int tt = t_warp + j;
-        if (VM == V_BF16 && tt >= n) continue;  // stale bf16 rows may be NaN
+        if (VM == V_BF16 && !FULL && tt >= n) continue;  // stale bf16 rows may be NaN
         float2 f[4];
         value_pairs<VM, VBITS>(vc + tt * VROW, slice, f);
         const float2 *wrow = reinterpret_cast<const float2 *>(wsm) + (j * n_vg + gv_lane) * GQA;
@@ -517,8 +520,9 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
     uint8_t *stages = smem;
     uint8_t *tail = smem + static_cast<size_t>(NS) * p.stage_bytes;
     float *qs = reinterpret_cast<float *>(tail);                    // [GQA][128]
-    float *wsm_all = qs + GQA * kHeadDim;                            // [4][16][8][GQA][2]
-    float *red = wsm_all + kConsumerWarps * 16 * 8 * GQA * 2;        // [4][GQA][130]
+    // value weights per warp: [token of the warp][value group][GQA][2]
+    float *wsm_all = qs + GQA * kHeadDim;
+    float *red = wsm_all + kConsumerWarps * p.wsm_floats;            // [4][GQA][130]
     float *qsum_all = red + kConsumerWarps * GQA * 130;              // [4][8][3][GQA]
     float *qhead = qsum_all + kConsumerWarps * 8 * 3 * GQA;          // [2][GQA]
     uint64_t *full = reinterpret_cast<uint64_t *>(qhead + 2 * GQA + 2);
@@ -572,6 +576,8 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
         const int ngv = (VM == V_TOKEN) ? geo.nvg() : 0;
         int it = 0;  // tile counter of this CTA (stage it % NS, round it / NS)
         bool stop = false;
+        // Quantized tiles never straddle a block of per-channel key scales.
+        const int qtile = (KM == K_CHANNEL) ? min(kTile, p.R) : kTile;
         while (!stop) {
             const int item = atomicAdd(p.counter, 1);
             int seq = 0, kvh = 0, split = 0;
@@ -583,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
                 t_end = min(T, t_begin + p.chunk);
                 Tq = quantized_len(T, p.R);
                 q_end = min(t_end, Tq);
-                n_qt = q_end > t_begin ? (q_end - t_begin + kTile - 1) / kTile : 0;
+                n_qt = q_end > t_begin ? (q_end - t_begin + qtile - 1) / qtile : 0;
                 w_begin = max(t_begin, Tq);
                 n_wt = t_end > w_begin ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
             }
@@ -608,8 +614,8 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
                 }
                 if (it == p.skip_tile) continue;  // test hook: never arrive
                 const bool window = ti >= n_qt;
-                const int t0 = window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * kTile;
-                const int n = window ? min(p.bf_tile, t_end - t0) : min(kTile, q_end - t0);
+                const int t0 = window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * qtile;
+                const int n = window ? min(p.bf_tile, t_end - t0) : min(qtile, q_end - t0);
                 hdr->seq = seq;
                 hdr->kvh = kvh;
                 hdr->split = split;
@@ -690,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
     const int perm = (GQA == 4) ? (((part >> 2) & 1) << 1 | ((part >> 1) & 1)) : 0;
     QueryRegs<GQA> Q;
     float *qsum = qsum_all + warp * 8 * 3 * GQA;
-    float *wsm = wsm_all + warp * 16 * 8 * GQA * 2;
+    float *wsm = wsm_all + warp * p.wsm_floats;
 
     // mode: 0 = token-wise codes, 1 = channel-wise codes (per-channel scales
     // folded in from `chan_sz`), 2 = bf16 keys.
@@ -860,16 +866,21 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
                     load_query(1, sb + p.off_ksz);
                 }
             }
-            process_tile<GQA, KM, VM, KBITS, VBITS, kTile / kConsumerWarps, GK, GV, VSLOTS>(
-                sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, geo, Q, qsum, st, wsm,
-                warp, lane);
+            if (hdr.n == kTile)
+                process_tile<GQA, KM, VM, KBITS, VBITS, kTokensPerWarp, GK, GV, VSLOTS, true>(
+                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, geo, Q, qsum, st, wsm,
+                    warp, lane);
+            else
+                process_tile<GQA, KM, VM, KBITS, VBITS, kTokensPerWarp, GK, GV, VSLOTS, false>(
+                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, geo, Q, qsum, st, wsm,
+                    warp, lane);
         } else if constexpr (KM != K_BF16) {
             if (!folded) {  // first window tile of the item
                 load_query(2, nullptr);
                 if (VM == V_TOKEN) fold_values();
                 folded = true;
             }
-            process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, GK, GV, VSLOTS>(
+            process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, GK, GV, VSLOTS, false>(
                 sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, geo, Q, qsum, st, wsm, warp, lane);
         }
 
@@ -983,8 +994,8 @@ StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
 }
 
 template <int GQA>
-size_t tail_bytes(int NS, int S) {
-    return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * 16 * 8 * GQA * 2 +
+size_t tail_bytes(int NS, int S, int wsm_floats) {
+    return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * wsm_floats +
                             kConsumerWarps * GQA * 130 + kConsumerWarps * 8 * 3 * GQA + 2 * GQA + 2) +
            sizeof(uint64_t) * 2 * NS + 16 + sizeof(int) * (S + 1);
 }
@@ -999,7 +1010,7 @@ int sm_count() {
 template <int GQA, int KM, int VM, int KBITS, int VBITS, int GK, int GV>
 kvq_status launch_variant(const DecodeParams &p, int max_items, cudaStream_t stream) {
     constexpr int NS = (KM == K_BF16) ? 3 : 4;
-    const size_t smem = static_cast<size_t>(NS) * p.stage_bytes + tail_bytes<GQA>(NS, p.S);
+    const size_t smem = static_cast<size_t>(NS) * p.stage_bytes + tail_bytes<GQA>(NS, p.S, p.wsm_floats);
     auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, NS, GK, GV>;
     if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;  // too many sequences for one launch
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1125,6 +1136,9 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.off_hdr = L.off_hdr;
     p.bf_tile = L.bf_tile;
     p.bf_off_v = L.bf_off_v;
+    // value groups per token: 1 for bf16 values (and for the bf16 window tiles)
+    const int n_vg = (d.bits_v == 16) ? 1 : kHeadDim / d.group_v;
+    p.wsm_floats = kTokensPerWarp * n_vg * gqa * 2;
     p.timeout_ns = debug_hooks().wait_timeout_ns;
     p.skip_tile = debug_hooks().skip_tile;
     const int64_t max_items64 = static_cast<int64_t>(num_seqs) * d.num_kv_heads * plan.n_split;

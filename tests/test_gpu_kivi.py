@@ -101,6 +101,28 @@ def test_window_flush_and_attention(bits, G_v, per_channel):
                      "seq %d" % s)
 
 
+def test_window_64_channel_blocks():
+    # residual window and per-channel key blocks of 64 tokens: every block of
+    # key scales is its own tile
+    H, Hq, S = 2, 8, 2
+    total = [517, 64]
+    g = np.random.default_rng(64)
+    ch = W.outlier_channels(g)
+    ks = [W.finish(W.keys(g, (t, H, D), ch), "bf16") for t in total]
+    vs = [W.finish(W.normal(g, (t, H, D)), "bf16") for t in total]
+    cache = K.KVCache(_spec(S, H, 576, 2, 32, R=64))
+    sl = lens_tensor([0] * S)
+    append(cache, ks, vs, sl)
+    torch.cuda.synchronize()
+    for s in range(S):
+        _check_state(cache, ks[s], vs[s], total[s], s, 1)
+    qs = W.finish(W.normal(g, (S, Hq, D)), "bf16")
+    out = K.decode_attention(cache.desc, dev(qs, "bf16"), sl, 576, SCALE).cpu().numpy()
+    assert cache.device_status() == 0
+    for s in range(S):
+        assert_close(out[s], _oracle_decode(ks[s], vs[s], qs[s], cache.spec), "seq %d" % s)
+
+
 def test_token_by_token_equals_bulk():
     H = 1
     g = np.random.default_rng(12)
