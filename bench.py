@@ -5,7 +5,7 @@ Workload (the metric's configuration): a Llama-3.1-8B-shaped attention layer,
 outlier channels (x20), keys and queries Hadamard-rotated, K and V INT4 in
 groups of 128 (fp16 scale/zero), contiguous cache, context 8192. A step is
 one decode step: quantize-append one new token per sequence, then split-K
-decode attention over the whole packed cache (split pass + merge pass).
+decode attention over the whole packed cache (split-K pass + merge pass).
 Steps run as episodes of 64 decode steps (context 8193..8256); after each
 episode the sequence lengths are rewound to 8192 outside the timed region.
 
@@ -230,12 +230,10 @@ def run_ours(args, rank, world, local_rank):
         K.quantize_append(cache.desc, k_steps[j], v_steps[j], cu_one, lens)
         if evs:
             evs[1].record(stream)
-        K.decode_splitk(cache.desc, q_steps[j], lens, cap, scale, ws)
+        # split-K pass, then the merge pass (a programmatic dependent launch)
+        K.decode_attention(cache.desc, q_steps[j], lens, cap, scale, out=out, workspace=ws)
         if evs:
             evs[2].record(stream)
-        K.decode_merge(cache.desc, HQ, lens, cap, out, ws)
-        if evs:
-            evs[3].record(stream)
         return CTX + j + 1   # tokens attended per sequence
 
     for i in range(args.warmup):
@@ -243,7 +241,7 @@ def run_ours(args, rank, world, local_rank):
         step(i)
     torch.cuda.synchronize()
     # start the timed episodes at a step boundary of the episode
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     tokens = []
     if world > 1:
         torch.distributed.barrier()
@@ -255,10 +253,25 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    split_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     append1_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    merge_ms = [e[2].elapsed_time(e[3]) for e in evs]
+
+    # the dominant kernel alone, for its roofline: the split-K pass over the
+    # cache as the last step left it, L2 flushed before each launch
+    lens_now = lens.clone()
+    split_bytes = float(lens_now.sum().item()) * HKV * BYTES_PER_TOKEN_HEAD
+    split_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        K.decode_splitk(cache.desc, q_steps[0], lens_now, cap, scale, ws)
+        e1.record(stream)
+        if i >= args.warmup:
+            split_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    split_ms = [a.elapsed_time(b) for a, b in split_ms]
     total_ms = sum(step_ms)
     bytes_total = sum(t * BATCH * HKV * BYTES_PER_TOKEN_HEAD for t in tokens)
     assert cache.device_status() == 0, "device status %d" % cache.device_status()
@@ -294,7 +307,8 @@ def run_ours(args, rank, world, local_rank):
     h2d = dk.numel() * 2 + dv.numel() * 2 + dq.numel() * 2
     d2h = hout.numel() * 4
 
-    res = {"total_ms": total_ms, "bytes": bytes_total, "split_ms": split_ms, "merge_ms": merge_ms,
+    res = {"total_ms": total_ms, "bytes": bytes_total, "split_ms": split_ms, "attn_ms": attn_ms,
+           "split_bytes": split_bytes,
            "append1_ms": append1_ms, "step_ms": step_ms, "clocks": clocks.summary(),
            "append": append_info, "e2e_s": sum(e2e_s), "e2e_bytes": e2e_bytes,
            "h2d": h2d, "d2h": d2h, "tokens": tokens}
@@ -498,7 +512,7 @@ def main():
         hbm_peak, peak_kind = peaks()
         value = total_bytes / (total_ms * 1e-3) / 1e9
         split_mean_ms = statistics.mean(res["split_ms"])
-        bytes_per_launch = res["bytes"] / args.steps
+        bytes_per_launch = res["split_bytes"]
         achieved = bytes_per_launch / (split_mean_ms * 1e-3) / 1e9
         traffic = traffic_per_launch()
         cpu_gbs, cpu_done, cpu_s = cpu_time(cpu_units(16), args.cpu_budget)
@@ -515,8 +529,8 @@ def main():
                          "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": traffic,
                          "bytes_per_launch": bytes_per_launch, "ms_per_launch": split_mean_ms},
-            "breakdown_ms": {"append": statistics.mean(res["append1_ms"]), "splitk": split_mean_ms,
-                             "merge": statistics.mean(res["merge_ms"])},
+            "breakdown_ms": {"append": statistics.mean(res["append1_ms"]),
+                             "attention_splitk_and_merge": statistics.mean(res["attn_ms"])},
             "append": res["append"],
             "cpu_baseline": {"value": cpu_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": "%d (sequence, KV head) units of the decode step at "
@@ -524,7 +538,7 @@ def main():
                                        "+ attention, one thread" % (cpu_done, cpu_s)},
             "e2e": {"value": e2e_bytes / e2e_s / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": 4 * args.steps,   # append, advance lengths, split-K, merge
             "clocks": res["clocks"],
         }
         if rr is not None:

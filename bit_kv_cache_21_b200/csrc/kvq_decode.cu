@@ -540,6 +540,9 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
         fence_mbar_init();
     }
     __syncthreads();
+    // A dependent launch (the merge pass) may be scheduled from now on; it
+    // waits for this grid's completion before reading anything.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == kConsumerWarps) {
         // ------------------------- producer -------------------------
@@ -935,21 +938,34 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
 }
 
 // One CTA of 128 threads per (query head, sequence): combine the splits.
+// Launched as a programmatic dependent of the split-K pass: its CTAs may start
+// while that pass drains and wait here until its partials are complete.
 __global__ void __launch_bounds__(128) decode_merge_kernel(const float *o_part, const float2 *ml,
                                                            const int32_t *seq_lens, float *out,
                                                            int Hq, int n_split, int chunk,
                                                            int max_seq_len) {
+    __shared__ float s_max;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int hq = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
     const int T = min(__ldg(seq_lens + seq), max_seq_len);
     const int nv = T > 0 ? (T + chunk - 1) / chunk : 0;
     const int64_t base = (static_cast<int64_t>(seq) * Hq + hq) * n_split;
-    float M = -INFINITY;
-    for (int j = 0; j < nv; ++j) M = fmaxf(M, ml[base + j].x);
+    if (d < 32) {  // maximum over the splits, one warp
+        float m = -INFINITY;
+        for (int j = d; j < nv; j += 32) m = fmaxf(m, ml[base + j].x);
+#pragma unroll
+        for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
+        if (d == 0) s_max = m;
+    }
+    __syncthreads();
+    const float M = s_max;
     float o = 0.0f, l = 0.0f;
+    const float *op = o_part + base * kHeadDim + d;
+#pragma unroll 4
     for (int j = 0; j < nv; ++j) {
         const float2 v = ml[base + j];
         const float e = (v.x == -INFINITY) ? 0.0f : fast_exp2(v.x - M);
-        o = fmaf(e, o_part[(base + j) * kHeadDim + d], o);
+        o = fmaf(e, op[static_cast<int64_t>(j) * kHeadDim], o);
         l = fmaf(e, v.y, l);
     }
     out[(static_cast<int64_t>(seq) * Hq + hq) * kHeadDim + d] = (l > 0.0f) ? o / l : 0.0f;
@@ -1158,9 +1174,21 @@ kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, 
     const float *o_part = static_cast<const float *>(workspace);
     const float2 *ml =
         reinterpret_cast<const float2 *>(static_cast<const uint8_t *>(workspace) + plan.ws_part);
-    decode_merge_kernel<<<dim3(num_q_heads, num_seqs), 128, 0, stream>>>(
-        o_part, ml, seq_lens, out, num_q_heads, plan.n_split, plan.chunk, max_seq_len);
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(num_q_heads, num_seqs);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int n_split = plan.n_split, chunk = plan.chunk;
+    return cudaLaunchKernelEx(&cfg, decode_merge_kernel, o_part, ml, seq_lens, out, num_q_heads,
+                              n_split, chunk, max_seq_len) == cudaSuccess
+               ? KVQ_OK
+               : KVQ_ERR_CUDA;
 }
 
 }  // namespace kvq
