@@ -248,6 +248,7 @@ __device__ __forceinline__ bool dest_row(const AppendParams &p, int s, int pos, 
 // grid.x: blocks of 64 vectors; grid.y: 0 = keys, 1 = values.
 template <int DT>
 __global__ void __launch_bounds__(256) append_tokens_kernel(const AppendParams p) {
+    pdl_launch_dependents();  // the length advance may be scheduled; it waits for us
     const AppendTensor &T = p.t[blockIdx.y];
     const int lane = threadIdx.x & 31;
     const int part = lane & 3;
@@ -399,6 +400,7 @@ __global__ void __launch_bounds__(256) window_flush_kernel(const WindowParams p)
 // Copy the new tokens that stay in the window into their slots. One thread
 // per 16-byte chunk of a (token, head) row; K and V.
 __global__ void __launch_bounds__(256) window_write_kernel(const WindowParams p) {
+    pdl_launch_dependents();  // the length advance may be scheduled; it waits for us
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t n_chunks = static_cast<int64_t>(p.total_tokens) * p.H * 16;
     if (i >= n_chunks) return;
@@ -420,7 +422,10 @@ __global__ void __launch_bounds__(256) window_write_kernel(const WindowParams p)
         reinterpret_cast<const uint4 *>(p.v_new + vrow * kHeadDim)[c];
 }
 
+// Launched as a programmatic dependent of the append kernel: scheduled early,
+// it waits for that grid (which reads the old lengths) to complete.
 __global__ void advance_lens_kernel(const int32_t *cu_new, int32_t *seq_lens, int num_seqs) {
+    pdl_wait_prior_grid();
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
     if (s < num_seqs) seq_lens[s] += cu_new[s + 1] - cu_new[s];
 }
@@ -484,8 +489,17 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
         }
         if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     }
-    advance_lens_kernel<<<(num_seqs + 127) / 128, 128, 0, stream>>>(cu_new, seq_lens, num_seqs);
-    if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((num_seqs + 127) / 128);
+    cfg.blockDim = dim3(128);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, advance_lens_kernel, cu_new, seq_lens, num_seqs) != cudaSuccess)
+        return KVQ_ERR_CUDA;
     return KVQ_OK;
 }
 

@@ -123,6 +123,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+// Programmatic dependent launch: let the next kernel of the stream (launched
+// with programmatic stream serialization) be scheduled now; and, in that
+// kernel, wait until the previous grid has completed and its writes are
+// visible. Both are no-ops without such a launch.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prior_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // 1-D bulk copy global -> shared through the TMA engine, completing on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16. No multicast.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
