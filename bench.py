@@ -393,6 +393,160 @@ def run_remat(args, dev):
             "gpu_launches_per_step": 4}
 
 
+# ---------------------------------------------------------------------------
+# Other decode workloads (extra objects of the default line; --part selects one)
+# ---------------------------------------------------------------------------
+def _synthetic_kv(gen, n_tok, H, dev, torch, seed):
+    """bf16 K (4 outlier channels x20, drawn as the workload recipe does) and
+    V ~ N(0, 1), [n_tok][H][128]."""
+    import workloads as W
+    ch = torch.as_tensor(W.outlier_channels(W.rng(seed)), dtype=torch.long, device=dev)
+    k = torch.randn((n_tok, H, D), generator=gen, device=dev)
+    k[:, :, ch] *= 20.0
+    v = torch.randn((n_tok, H, D), generator=gen, device=dev)
+    return k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def _time_steps(torch, stream, flush, n_warm, n_steps, step):
+    """Run n_warm + n_steps steps (L2 flushed before each), timing append and
+    attention of the last n_steps with events. step(i, evs) records evs[0..2]."""
+    evs = []
+    for i in range(n_warm + n_steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        step(i, e)
+        if i >= n_warm:
+            evs.append(e)
+    torch.cuda.synchronize()
+    app = [e[0].elapsed_time(e[1]) for e in evs]
+    att = [e[1].elapsed_time(e[2]) for e in evs]
+    return app, att
+
+
+def run_long_int2(args, dev):
+    """1 sequence at 131072 positions, 32 q / 8 KV heads, KIVI INT2: keys per
+    channel in 128-token blocks, values per token in groups of 32, a 128-token
+    bf16 window. A step appends one token and attends over the whole context."""
+    import torch
+    import bit_kv_cache_21_b200 as K
+    H, HQ_, T_END, R = 8, 32, 131072, 128
+    n_steps, n_warm = 40, 3
+    T0 = T_END - (n_steps + n_warm)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3)
+    spec = K.CacheSpec(1, H, bits_k=2, bits_v=2, group_k=R, group_v=32, per_channel_k=True,
+                       residual_len=R, capacity_tokens=T_END + R)
+    cache = K.KVCache(spec, device=dev)
+    lens = torch.zeros(1, dtype=torch.int32, device=dev)
+    k, v = _synthetic_kv(gen, T0, H, dev, torch, 3)
+    K.quantize_append(cache.desc, k, v, torch.tensor([0, T0], dtype=torch.int32, device=dev), lens)
+    del k, v
+    ks, vs = _synthetic_kv(gen, n_steps + n_warm, H, dev, torch, 3)
+    q = torch.randn((1, HQ_, D), generator=gen, device=dev).to(torch.bfloat16)
+    cu_one = torch.tensor([0, 1], dtype=torch.int32, device=dev)
+    ws = torch.empty(K.decode_workspace_size(cache.desc, 1, HQ_, T_END), dtype=torch.uint8, device=dev)
+    out = torch.empty((1, HQ_, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(D)
+
+    def step(i, e):
+        e[0].record(stream)
+        K.quantize_append(cache.desc, ks[i:i + 1], vs[i:i + 1], cu_one, lens)
+        e[1].record(stream)
+        K.decode_attention(cache.desc, q, lens, T_END, scale, out=out, workspace=ws)
+        e[2].record(stream)
+
+    app, att = _time_steps(torch, stream, flush, n_warm, n_steps, step)
+    assert cache.device_status() == 0
+    nbytes = []
+    for i in range(n_warm, n_warm + n_steps):
+        T = T0 + i + 1
+        Tq = R * ((T - 1) // R)
+        nbytes.append(H * (Tq * (32 + 32 + 16) + (Tq // R) * D * 4 + (T - Tq) * 2 * D * 2))
+    mb = statistics.mean(nbytes)
+    return {"workload": "long_int2: 1 seq, 32 q / 8 kv heads, context %d..%d, K INT2 per channel "
+                        "(128-token blocks), V INT2 per token (g32), 128-token bf16 window"
+                        % (T0 + n_warm + 1, T_END),
+            "steps": n_steps, "bytes_per_step": mb,
+            "append_ms": statistics.mean(app), "attention_ms": statistics.mean(att),
+            "attention_GBps": mb / (statistics.mean(att) * 1e-3) / 1e9,
+            "step_GBps": mb / ((statistics.mean(app) + statistics.mean(att)) * 1e-3) / 1e9}
+
+
+def run_paged_mix(args, dev):
+    """64 sequences, lognormal lengths (median 4096, sigma 1, clipped to
+    [1024, 32768]), 16-token pages, INT4 g128, Hadamard keys. A step appends a
+    512-token chunk to 8 sequences and one token to the other 56, then attends
+    over all 64; every 4 steps the lengths are rewound outside the timing."""
+    import numpy as np
+    import torch
+    import bit_kv_cache_21_b200 as K
+    import workloads as W
+    H, HQ_, PS, EP = 8, 32, 16, 4
+    n_steps, n_warm = 20, 4
+    pre = W.paged_lengths(4)
+    new = np.array([512] * 8 + [1] * 56)
+    final = pre + EP * new
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    spec = K.CacheSpec(64, H, hadamard_block_k=128, paged=True, page_size=PS,
+                       max_pages_per_seq=int(final.max()) // PS + 1,
+                       num_pages=int(sum(final // PS + 1)))
+    cache = K.KVCache(spec, device=dev)
+    need = [(int(t) + PS - 1) // PS for t in final]
+    free = np.random.default_rng(4).permutation(spec.num_pages)
+    bt = np.full((64, spec.max_pages_per_seq), -1, np.int32)
+    i0 = 0
+    for s_, n in enumerate(need):
+        bt[s_, :n] = free[i0:i0 + n]
+        i0 += n
+    cache.block_table.copy_(torch.from_numpy(bt))
+    lens = torch.zeros(64, dtype=torch.int32, device=dev)
+    cu_pre = torch.from_numpy(np.concatenate([[0], np.cumsum(pre)]).astype(np.int32)).to(dev)
+    k, v = _synthetic_kv(gen, int(pre.sum()), H, dev, torch, 4)
+    K.quantize_append(cache.desc, k, v, cu_pre, lens)
+    del k, v
+    pre_lens = lens.clone()
+    n_new = int(new.sum())
+    cu_new = torch.from_numpy(np.concatenate([[0], np.cumsum(new)]).astype(np.int32)).to(dev)
+    step_kv = [_synthetic_kv(gen, n_new, H, dev, torch, 4) for _ in range(EP)]
+    q = torch.randn((64, HQ_, D), generator=gen, device=dev).to(torch.bfloat16)
+    max_len = int(final.max())
+    ws = torch.empty(K.decode_workspace_size(cache.desc, 64, HQ_, max_len), dtype=torch.uint8, device=dev)
+    out = torch.empty((64, HQ_, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(D)
+
+    def step(i, e):
+        j = i % EP
+        if j == 0:
+            lens.copy_(pre_lens)
+        kk, vv = step_kv[j]
+        e[0].record(stream)
+        K.quantize_append(cache.desc, kk, vv, cu_new, lens)
+        e[1].record(stream)
+        K.decode_attention(cache.desc, q, lens, max_len, scale, out=out, workspace=ws)
+        e[2].record(stream)
+
+    app, att = _time_steps(torch, stream, flush, n_warm, n_steps, step)
+    assert cache.device_status() == 0
+    nbytes = [float(sum(pre + ((i % EP) + 1) * new)) * H * BYTES_PER_TOKEN_HEAD
+              for i in range(n_warm, n_warm + n_steps)]
+    mb = statistics.mean(nbytes)
+    appended = n_new * H * 2 * (D * 2 + D // 2 + 4)
+    return {"workload": "paged_mix: 64 seqs, lognormal lengths (median 4096, sigma 1) %d..%d tokens, "
+                        "16-token pages, INT4 g128, Hadamard K; per step 8 x 512 + 56 x 1 appended"
+                        % (int(pre.min()), int(final.max())),
+            "steps": n_steps, "bytes_per_step": mb,
+            "append_ms": statistics.mean(app), "append_tokens_per_s": n_new / (statistics.mean(app) * 1e-3),
+            "append_GBps": appended / (statistics.mean(app) * 1e-3) / 1e9,
+            "attention_ms": statistics.mean(att),
+            "attention_GBps": mb / (statistics.mean(att) * 1e-3) / 1e9,
+            "step_GBps": mb / ((statistics.mean(app) + statistics.mean(att)) * 1e-3) / 1e9}
+
+
 def cpu_units(n_units, seed=0):
     """Oracle-side cache state of n_units (sequence, KV head) units of the
     workload at context 8193: the oracle's own packed K/V and 4 queries."""
@@ -435,8 +589,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
-    ap.add_argument("--part", default="all", choices=["all", "decode", "remat"],
-                    help="remat: only the XQuant rematerialization leg (prints its own line)")
+    ap.add_argument("--part", default="all",
+                    choices=["all", "decode", "remat", "long_int2", "paged_mix"],
+                    help="run one leg alone: decode (the metric's step), remat, long_int2 or "
+                         "paged_mix (the last three print their own line)")
     ap.add_argument("--remat-batch", type=int, default=8)
     ap.add_argument("--remat-steps", type=int, default=10)
     args = ap.parse_args()
@@ -483,6 +639,19 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    if args.part in ("long_int2", "paged_mix"):
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        leg = (run_long_int2 if args.part == "long_int2" else run_paged_mix)(args, dev)
+        if rank == 0:
+            print(json.dumps({"metric": "decode-attn packed-KV GB/s", "value": leg["attention_GBps"],
+                              "unit": "GB/s", "n_gpus": world, "higher_is_better": True,
+                              "data": "synthetic", "config": {"workload": leg["workload"]},
+                              args.part: leg}))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.part == "remat":
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
@@ -498,6 +667,8 @@ def main():
         return
     res = run_ours(args, rank, world, local_rank)
     rr = run_remat(args, torch.device("cuda", local_rank)) if args.part == "all" else None
+    li = run_long_int2(args, torch.device("cuda", local_rank)) if args.part == "all" else None
+    pm = run_paged_mix(args, torch.device("cuda", local_rank)) if args.part == "all" else None
 
     # max over ranks of the device time; bytes summed over ranks
     total_ms, total_bytes, e2e_s, e2e_bytes = res["total_ms"], res["bytes"], res["e2e_s"], res["e2e_bytes"]
@@ -543,6 +714,10 @@ def main():
         }
         if rr is not None:
             line["xquant_remat"] = rr
+        if li is not None:
+            line["long_int2"] = li
+        if pm is not None:
+            line["paged_mix"] = pm
         print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()
