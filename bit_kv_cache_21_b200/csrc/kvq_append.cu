@@ -81,21 +81,64 @@ __device__ __forceinline__ void load32(const void *src, int64_t vec, int part, f
     }
 }
 
+// ---- packed f32x2 arithmetic: two independent round-to-nearest fp32 ops ----
+__device__ __forceinline__ unsigned long long f2u(float a, float b) {
+    return (static_cast<unsigned long long>(__float_as_uint(b)) << 32) | __float_as_uint(a);
+}
+__device__ __forceinline__ float lo_f(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long sub2(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 // Normalized Sylvester Walsh-Hadamard transform of each hb-block, the four
 // lanes of a vector holding 32 channels each. Stage half-widths ascend
 // 1, 2, ..., hb/2; butterfly (a, b) -> (a + b, a - b) with a the lower index;
-// finally one multiply by c = fp32(1/sqrt(hb)).
+// finally one multiply by c = fp32(1/sqrt(hb)). Stages of half-width >= 2 run
+// on channel pairs (j, j+1) with packed f32x2 adds; the cross-lane stages
+// compute o + s*x with s = +-1 in one packed fma, which rounds like the add
+// or subtract it stands for.
 __device__ __forceinline__ void fwht_lane(float x[32], int hb, int part, float c) {
+    if (hb > 1) {
 #pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
+        for (int j = 0; j < 32; j += 2) {
+            const float a = x[j], b = x[j + 1];
+            x[j] = __fadd_rn(a, b);
+            x[j + 1] = __fsub_rn(a, b);
+        }
+    }
+    unsigned long long v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = f2u(x[2 * k], x[2 * k + 1]);
+#pragma unroll
+    for (int h = 2; h < 32; h <<= 1) {  // pair index half-width h / 2
         if (h < hb) {
+            const int hp = h / 2;
 #pragma unroll
-            for (int i = 0; i < 32; i += 2 * h) {
+            for (int i = 0; i < 16; i += 2 * hp) {
 #pragma unroll
-                for (int j = i; j < i + h; ++j) {
-                    const float a = x[j], b = x[j + h];
-                    x[j] = __fadd_rn(a, b);
-                    x[j + h] = __fsub_rn(a, b);
+                for (int k = i; k < i + hp; ++k) {
+                    const unsigned long long a = v[k], b = v[k + hp];
+                    v[k] = add2(a, b);
+                    v[k + hp] = sub2(a, b);
                 }
             }
         }
@@ -103,16 +146,23 @@ __device__ __forceinline__ void fwht_lane(float x[32], int hb, int part, float c
 #pragma unroll
     for (int m = 1; m <= 2; m <<= 1) {  // half-widths 32 and 64: partner lane part ^ m
         if (32 * m < hb) {
-            const bool upper = (part & m) != 0;
+            const float sg = (part & m) ? -1.0f : 1.0f;  // upper: o - x, lower: x + o
+            const unsigned long long sg2 = f2u(sg, sg);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float o = __shfl_xor_sync(0xffffffffu, x[j], m);
-                x[j] = upper ? __fsub_rn(o, x[j]) : __fadd_rn(x[j], o);
+            for (int k = 0; k < 16; ++k) {
+                const float o0 = __shfl_xor_sync(0xffffffffu, lo_f(v[k]), m);
+                const float o1 = __shfl_xor_sync(0xffffffffu, hi_f(v[k]), m);
+                v[k] = fma2(sg2, v[k], f2u(o0, o1));
             }
         }
     }
+    const unsigned long long c2 = f2u(c, c);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], c);
+    for (int k = 0; k < 16; ++k) {
+        v[k] = mul2(v[k], c2);
+        x[2 * k] = lo_f(v[k]);
+        x[2 * k + 1] = hi_f(v[k]);
+    }
 }
 
 struct QParams {
@@ -144,6 +194,25 @@ __device__ __forceinline__ uint32_t qcode(float x, const QParams &p, float Lf) {
     return static_cast<uint32_t>(q);
 }
 
+// Codes of n consecutive elements (n even) of one group:
+// q = clamp(rint_even(fp32(fp32(x - z) * r)), 0, L). Every value reaching the
+// rounding lies in [0, L (1 + 3 2^-24)] (z <= x <= max, s >= (max - z) / L up
+// to one rounding, r = fp32(1/s)), so the upper clamp never binds; the lower
+// one also maps NaN to 0. Adding 2^23 rounds to the nearest integer, ties to
+// even, and leaves the code in the low bits of the float: q[j] holds 0x4B00000q.
+// r == 0 exactly when s == 0; then every code is 0.
+__device__ __forceinline__ void qcodes(const float *x, int n, const QParams &p, uint32_t *q) {
+    const unsigned long long z2 = f2u(p.zf, p.zf), r2 = f2u(p.r, p.r);
+    const unsigned long long magic = f2u(8388608.0f, 8388608.0f);
+#pragma unroll
+    for (int j = 0; j < n; j += 2) {
+        const unsigned long long t = mul2(sub2(f2u(x[j], x[j + 1]), z2), r2);
+        const unsigned long long y = add2(f2u(fmaxf(lo_f(t), 0.0f), fmaxf(hi_f(t), 0.0f)), magic);
+        q[j] = static_cast<uint32_t>(y);
+        q[j + 1] = static_cast<uint32_t>(y >> 32);
+    }
+}
+
 // Quantize the lane's 32 channels in groups of G (the group spans G/32 lanes
 // when G > 32) and pack them. Returns the scale/zero pairs of the groups that
 // start in this lane (n_sz of them) and the packed words (4 for INT4, 2 for
@@ -152,8 +221,7 @@ template <int BITS>
 __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32_t words[4],
                                                 __half2 sz[2], int &n_sz, int part) {
     constexpr int L = (1 << BITS) - 1;
-    const float Lf = static_cast<float>(L);
-    uint32_t q[32];
+    uint32_t q[32];  // 0x4B00000q
     if (G >= 32) {
         float mn = x[0], mx = x[0];
 #pragma unroll
@@ -163,8 +231,7 @@ __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
         }
         const QParams p = qparams(mn, mx, L);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) q[j] = qcode(x[j], p, Lf);
+        qcodes(x, 32, p, q);
         sz[0] = p.sz;
         n_sz = ((part * 32) % G == 0) ? 1 : 0;
     } else {  // G == 16: two groups in the lane
@@ -174,26 +241,27 @@ __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32
 #pragma unroll
             for (int j = 1; j < 16; ++j) { mn = fminf(mn, x[16 * g + j]); mx = fmaxf(mx, x[16 * g + j]); }
             const QParams p = qparams(mn, mx, L);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) q[16 * g + j] = qcode(x[16 * g + j], p, Lf);
+            qcodes(x + 16 * g, 16, p, q + 16 * g);
             sz[g] = p.sz;
         }
         n_sz = 2;
     }
     if constexpr (BITS == 4) {
+        // word w: byte k = q[8w+2k] | q[8w+2k+1] << 4. Gather the even and the
+        // odd codes' low bytes with byte permutes, then E + 16 O.
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            uint32_t v = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v |= q[8 * w + j] << (4 * j);
-            words[w] = v;
+            const uint32_t *c = q + 8 * w;
+            const uint32_t e = __byte_perm(__byte_perm(c[0], c[2], 0x0040), __byte_perm(c[4], c[6], 0x0040), 0x5410);
+            const uint32_t o = __byte_perm(__byte_perm(c[1], c[3], 0x0040), __byte_perm(c[5], c[7], 0x0040), 0x5410);
+            words[w] = e + (o << 4);
         }
     } else {
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
             uint32_t v = 0;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v |= q[16 * w + j] << (2 * j);
+            for (int j = 0; j < 16; ++j) v |= (q[16 * w + j] & 3u) << (2 * j);
             words[w] = v;
         }
     }
