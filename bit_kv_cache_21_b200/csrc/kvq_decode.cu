@@ -11,30 +11,38 @@
 //
 // Work items are (sequence, KV head, split of `chunk` tokens). The kernel is
 // persistent: each CTA (4 consumer warps + 1 producer warp) runs until a
-// global item counter is exhausted. The producer's elected lane claims items
-// and streams every item's tiles (K codes, K scale/zero, V codes, V scale/zero;
-// bf16 rows for the recent-token window; the item's query rows with its first
-// tile) into a shared-memory ring with 1-D bulk copies (TMA engine, mbarrier
-// complete_tx), resolving page tables per page. Each stage carries a small
-// header, so the consumers follow the stream without further coordination and
-// the ring never drains between items.
+// global item counter is exhausted. The producer warp claims items and streams
+// every item's tiles (K codes, K scale/zero, V codes, V scale/zero; bf16 rows
+// for the recent-token window; the item's query rows with its first tile) into
+// a shared-memory ring with 1-D bulk copies (TMA engine, mbarrier
+// complete_tx); its lanes issue the copies of a tile in parallel, one page per
+// lane for paged caches. Each stage carries a small header, so the consumers
+// follow the stream without further coordination and the ring never drains
+// between items.
 //
-// Inner loop. The path is bound by the FP32 FMA pipe, not by the tensor
-// cores: every cached element meets GQA query heads, one multiply-add each.
-// So the loop spends as few issue slots as possible besides those:
-//   * multiply-adds are packed f32x2 FMAs (two lanes of work per issue);
+// The path is bound by the FP32 pipe, not by the tensor cores: every cached
+// element meets GQA query heads, one multiply-add each, and on sm_100a the
+// packed f32x2 FMA issues at half rate. So the consumers spend as few issue
+// slots as possible besides those multiply-adds:
+//   * keys: one lane per token. A lane walks its token's code row in 16-byte
+//     chunks and multiplies each code with the GQA heads' query coefficients,
+//     which every lane reads with the same broadcast shared-memory load. No
+//     cross-lane reduction; softmax statistics come out per lane. The chunk
+//     order is XOR-rotated per lane so the 8 lanes of a shared-memory phase
+//     hit 8 distinct bank groups (their rows are 16-64 bytes apart); the
+//     coefficients are stored with a 16-byte pad per chunk for the same
+//     reason.
 //   * codes become floats 0.5 + X/256 with ONE byte permute per code, from
-//     byte planes kept below 128; the query is transformed once per item so
-//     that its dot product with these floats is the one with the codes, and
-//     the value sums are untangled once per item;
-//   * each consumer warp owns a quarter of every tile with its own
-//     online-softmax state, so tiles need no cross-warp synchronisation;
-//   * scores: 8 lanes per token, 16 channels per lane, all GQA heads at once,
-//     a select-free reduce-scatter over the 8 lanes (heads held in a per-lane
-//     permuted order) leaves one head's score per lane pair;
+//     byte planes kept below 128; the query coefficients are transformed once
+//     per item so that their dot product with these floats is the one with the
+//     codes, and the value sums are untangled once per item;
+//   * multiply-adds are packed f32x2 FMAs;
+//   * softmax: each warp keeps a reference maximum per head that moves only
+//     when a score exceeds it by more than 8 (log2 units); a warp vote decides
+//     whether a tile needs the max reduction at all;
 //   * values: 16 lanes cover the 128 channels (8 each) for all GQA heads; the
-//     two half-warps take alternate tokens;
-//   * common group sizes are compile-time constants.
+//     two half-warps take alternate tokens; the weights p*s come from the key
+//     lanes through shared memory, already duplicated into f32x2 pairs.
 // The four warps' states are merged once per item; the merge kernel combines
 // the splits.
 #include <algorithm>
@@ -46,16 +54,15 @@ namespace kvq {
 
 namespace {
 
-constexpr int kTile = 128;         // tokens per quantized tile
+constexpr int kTileQ = 256;        // tokens per quantized tile (64 per warp, 2 per lane)
+constexpr int kTileB = 128;        // tokens per tile of a bf16 cache (32 per warp)
 constexpr int kWinTile = 16;       // tokens per bf16 window tile (quantized caches)
+constexpr int kMaxStages = 4;      // shared-memory ring depth, chosen on the host
 constexpr int kConsumerWarps = 4;
-constexpr int kTokensPerWarp = kTile / kConsumerWarps;  // of a quantized tile
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
+constexpr int kMaxGroups = 8;      // kHeadDim / smallest token-wise group (16)
 constexpr float kLog2e = 1.4426950408889634f;
-#ifndef KVQ_DECODE_MIN_BLOCKS
-#define KVQ_DECODE_MIN_BLOCKS 2  // resident CTAs per SM the register budget targets
-#endif
 
 enum KMode { K_TOKEN = 0, K_CHANNEL = 1, K_BF16 = 2 };
 enum VMode { V_TOKEN = 0, V_BF16 = 2 };
@@ -80,30 +87,48 @@ struct DecodeParams {
     int *counter;   // item counter, zeroed before the launch
     int32_t *status;
     int S, H, Hq;
-    int gk_log2, gv_log2;  // log2 of the group sizes (token-wise groups)
+    int gk, gv;     // token-wise group sizes (K: 128 for per-channel keys)
     int hb;
     float hscale;   // fp32(1/sqrt(hb))
     float qscale;   // softmax_scale * log2(e)
     int R;
     int paged, page_size, max_pages, num_pages, cap;
     int chunk, n_split, max_seq_len;
+    int ns;                // ring depth (stages), <= kMaxStages
     int q_dtype, q_bytes;  // element type and bytes of q
     // shared-memory stage layout (bytes)
     int stage_bytes, off_ksz, off_vc, off_vsz, off_q, off_hdr;
     int bf_tile, bf_off_v;  // bf16 tiles: tokens per tile, offset of the V rows
-    int wsm_floats;         // per-warp value-weight scratch: tokens x value groups x GQA x 2
+    // per-warp scratch (floats): value weights (also the lanes' W/Z partials
+    // when they are summed), then the warp's W/Z totals
+    int warp_floats, off_tot;
+    int n_sets;            // coefficient sets (per-channel keys: 2 x blocks per tile)
     int64_t timeout_ns;
     int skip_tile;
 };
 
-template <int KM, int KBITS>
-struct KRow {
-    static constexpr int bytes = (KM == K_BF16) ? kHeadDim * 2 : kHeadDim * KBITS / 8;
+// ---- key rows ---------------------------------------------------------------
+// A row of KB-bit codes (KB = 16: bf16 values) is read in 16-byte chunks of
+// four 32-bit words; a word yields `npw` float pairs.
+template <int KB>
+struct RowGeo {
+    static constexpr int bytes = (KB == 16) ? kHeadDim * 2 : kHeadDim * KB / 8;
+    static constexpr int nch = bytes / 16;          // chunks per row
+    static constexpr int cpc = kHeadDim / nch;      // channels per chunk
+    static constexpr int cpw = cpc / 4;             // channels per word
+    static constexpr int npw = (KB == 16) ? 1 : cpw / 2;  // float pairs per word
+    static constexpr int cstr = cpc + 4;            // padded coefficient floats per chunk
 };
-template <int VM, int VBITS>
-struct VRow {
-    static constexpr int bytes = (VM == V_BF16) ? kHeadDim * 2 : kHeadDim * VBITS / 8;
-};
+
+// Chunk order of a lane: step k reads chunk k ^ rot. Rows are 64 (INT4), 32
+// (INT2) or 256 (bf16) bytes apart, so without the rotation a phase of 8
+// consecutive rows would hit 2, 4 or 1 distinct 16-byte bank groups. With it
+// every phase covers all 8. XOR keeps aligned runs of chunks contiguous, so a
+// scale group spanning several chunks is still walked in one run.
+template <int KB>
+__device__ __forceinline__ int chunk_rot(int lane) {
+    return KB == 4 ? ((lane >> 1) & 3) : (KB == 2 ? ((lane >> 2) & 1) : (lane & 7));
+}
 
 // ---- packed f32x2 arithmetic (sm_100) --------------------------------------
 __device__ __forceinline__ unsigned long long as_u64(float2 v) {
@@ -119,14 +144,15 @@ __device__ __forceinline__ void ffma2(float2 &d, float2 a, float2 b) {
     d = as_f2(r);
 }
 
-// ---- shared-memory loads ----------------------------------------------------
-// Plain typed loads: the compiler sees their dependence on the stores and on
-// the mbarrier waits (asm with a memory clobber) and keeps them in order; the
-// pointers all derive from the kernel's shared array.
+// ---- shared-memory access ---------------------------------------------------
+// Plain typed loads and stores: the compiler sees their dependence on each
+// other and on the mbarrier waits (asm with a memory clobber) and keeps them in
+// order; the pointers all derive from the kernel's shared array.
 __device__ __forceinline__ uint32_t lds32(const void *p) { return *static_cast<const uint32_t *>(p); }
 __device__ __forceinline__ uint32_t lds16(const void *p) { return *static_cast<const uint16_t *>(p); }
 __device__ __forceinline__ uint2 lds64(const void *p) { return *static_cast<const uint2 *>(p); }
 __device__ __forceinline__ uint4 lds128(const void *p) { return *static_cast<const uint4 *>(p); }
+__device__ __forceinline__ float4 ldsf4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ float2 half2_lds(const void *p) {
     const uint32_t u = lds32(p);
     return __half22float2(*reinterpret_cast<const __half2 *>(&u));
@@ -139,35 +165,28 @@ __device__ __forceinline__ float2 half2_lds(const void *p) {
 // high nibble planes; INT2 codes use the planes
 //   X0 = c0, X1 = c0 + 4c1, X2 = c0 + 4c1 + 16c2, X3 = c1 + 4c2 + 16c3
 // (three masks and one shift of the packed word), all < 64. The floats are
-// linear in the codes; the query is transformed once per item so that its dot
-// product with them is the dot product with the codes (query_coeffs), and the
-// value accumulators are untangled once per item (value_channels).
+// linear in the codes; the query coefficients are transformed once per item so
+// that their dot product with them is the dot product with the codes
+// (build_head), and the value accumulators are untangled once per item
+// (value_channels).
 __device__ __forceinline__ float byte_f(uint32_t b, int k) {
     return __uint_as_float(__byte_perm(b, 0x3F000000u, 0x7054u | (static_cast<uint32_t>(k) << 8)));
 }
 
-// 16 key channels [16*part, 16*part + 16) as 8 float pairs.
+// One 32-bit word of a key row as float pairs, in the order of the coefficient
+// layout (natural channel order; INT2 bytes give their four planes):
 //   INT4 byte k (channels lo, hi): {f(lo), f(hi)}
 //   INT2 byte k (channels c0..c3): {f(X0), f(X1)}, {f(X2), f(X3)}
-//   bf16: the channel values themselves.
-template <int KM, int KBITS>
-__device__ __forceinline__ void key_pairs(const uint8_t *row, int part, float2 f[8]) {
-    if constexpr (KM == K_BF16) {
-        const uint4 a = lds128(row + part * 32), b = lds128(row + part * 32 + 16);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+//   bf16: the two channel values.
+template <int KB>
+__device__ __forceinline__ void word_pairs(uint32_t w, float2 *f) {
+    if constexpr (KB == 16) {
+        f[0] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    } else if constexpr (KB == 4) {
+        const uint32_t a = w & 0x0F0F0F0Fu, b = (w >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
-    } else if constexpr (KBITS == 4) {
-        const uint2 w = lds64(row + part * 8);
-        const uint32_t a0 = w.x & 0x0F0F0F0Fu, b0 = (w.x >> 4) & 0x0F0F0F0Fu;
-        const uint32_t a1 = w.y & 0x0F0F0F0Fu, b1 = (w.y >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            f[k] = make_float2(byte_f(a0, k), byte_f(b0, k));
-            f[4 + k] = make_float2(byte_f(a1, k), byte_f(b1, k));
-        }
+        for (int k = 0; k < 4; ++k) f[k] = make_float2(byte_f(a, k), byte_f(b, k));
     } else {
-        const uint32_t w = lds32(row + part * 4);
         const uint32_t x0 = w & 0x03030303u, x1 = w & 0x0F0F0F0Fu, x2 = w & 0x3F3F3F3Fu;
         const uint32_t x3 = (w >> 2) & 0x3F3F3F3Fu;
 #pragma unroll
@@ -178,302 +197,415 @@ __device__ __forceinline__ void key_pairs(const uint8_t *row, int part, float2 f
     }
 }
 
-// 8 value channels [8*slice, 8*slice + 8) as 4 float pairs, same encoding.
-template <int VM, int VBITS>
-__device__ __forceinline__ void value_pairs(const uint8_t *row, int slice, float2 f[4]) {
-    if constexpr (VM == V_BF16) {
-        const uint4 a = lds128(row + slice * 16);
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) f[j] = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
-    } else if constexpr (VBITS == 4) {
-        const uint32_t w = lds32(row + slice * 4);
-        const uint32_t a = w & 0x0F0F0F0Fu, b = (w >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) f[k] = make_float2(byte_f(a, k), byte_f(b, k));
+// Pairs [jb, jb + 4) of word_pairs (jb = 0 or 4), without converting the rest.
+template <int KB>
+__device__ __forceinline__ void word_pairs4(uint32_t w, int jb, float2 f[4]) {
+    if constexpr (KB == 4) {
+        word_pairs<4>(w, f);
     } else {
-        const uint32_t w = lds16(row + slice * 2);
-        const uint32_t x0 = w & 0x0303u, x1 = w & 0x0F0Fu, x2 = w & 0x3F3Fu, x3 = (w >> 2) & 0x3F3Fu;
+        // INT2: pairs 2k, 2k+1 come from byte k; this block covers bytes jb/2, jb/2 + 1
+        const uint32_t x0 = w & 0x03030303u, x1 = w & 0x0F0F0F0Fu, x2 = w & 0x3F3F3F3Fu;
+        const uint32_t x3 = (w >> 2) & 0x3F3F3F3Fu;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            f[2 * k] = make_float2(byte_f(x0, k), byte_f(x1, k));
-            f[2 * k + 1] = make_float2(byte_f(x2, k), byte_f(x3, k));
+        for (int kk = 0; kk < 2; ++kk) {
+            const int k = jb / 2 + kk;
+            f[2 * kk] = make_float2(byte_f(x0, k), byte_f(x1, k));
+            f[2 * kk + 1] = make_float2(byte_f(x2, k), byte_f(x3, k));
         }
     }
 }
 
-// Query coefficients for 16 channels x[0..15] of one head, in the pair
-// layout of key_pairs and times 256, such that
-//   sum_j qk[j] . f[j] = 128 * first + sum_i x_i c_i,
-// `first` being the sum of the (unscaled) coefficients.
-template <int KM, int KBITS>
-__device__ __forceinline__ void query_coeffs(const float x[16], float2 qk[8], float &first) {
-    first = 0.0f;
-    if constexpr (KM == K_BF16) {
+// 8 value channels [8*slice, 8*slice + 8) of two tokens (rows ra, rb) as 8
+// float pairs {token a, token b}, same encoding: INT4 channel j; INT2 byte k's
+// plane j at 4k + j; bf16 channel j.
+template <int VM, int VBITS>
+__device__ __forceinline__ void value_pairs(const uint8_t *ra, const uint8_t *rb, int slice, float2 f[8]) {
+    if constexpr (VM == V_BF16) {
+        const uint4 a = lds128(ra + slice * 16), b = lds128(rb + slice * 16);
+        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) qk[j] = make_float2(x[2 * j], x[2 * j + 1]);
-    } else if constexpr (KBITS == 4) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            qk[j] = make_float2(256.0f * x[2 * j], 256.0f * x[2 * j + 1]);
-            first += x[2 * j] + x[2 * j + 1];
+        for (int j = 0; j < 4; ++j) {
+            f[2 * j] = make_float2(__uint_as_float(wa[j] << 16), __uint_as_float(wb[j] << 16));
+            f[2 * j + 1] = make_float2(__uint_as_float(wa[j] & 0xFFFF0000u), __uint_as_float(wb[j] & 0xFFFF0000u));
         }
-    } else {
-        // a0 X0 + a1 X1 + a2 X2 + a3 X3 = q0 c0 + q1 c1 + q2 c2 + q3 c3
+    } else if constexpr (VBITS == 4) {
+        const uint32_t wa = lds32(ra + slice * 4), wb = lds32(rb + slice * 4);
+        const uint32_t la = wa & 0x0F0F0F0Fu, ha = (wa >> 4) & 0x0F0F0F0Fu;
+        const uint32_t lb = wb & 0x0F0F0F0Fu, hb = (wb >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const float q0 = x[4 * k], q1 = x[4 * k + 1], q2 = x[4 * k + 2], q3 = x[4 * k + 3];
-            const float a3 = q3 * 0.0625f;
-            const float a2 = (q2 - 4.0f * a3) * 0.0625f;
-            const float a1 = (q1 - 4.0f * a2 - a3) * 0.25f;
-            const float a0 = q0 - a1 - a2;
-            qk[2 * k] = make_float2(256.0f * a0, 256.0f * a1);
-            qk[2 * k + 1] = make_float2(256.0f * a2, 256.0f * a3);
-            first += (a0 + a1) + (a2 + a3);
+            f[2 * k] = make_float2(byte_f(la, k), byte_f(lb, k));
+            f[2 * k + 1] = make_float2(byte_f(ha, k), byte_f(hb, k));
         }
+    } else {
+        const uint32_t wa = lds16(ra + slice * 2), wb = lds16(rb + slice * 2);
+        const uint32_t xa[4] = {wa & 0x0303u, wa & 0x0F0Fu, wa & 0x3F3Fu, (wa >> 2) & 0x3F3Fu};
+        const uint32_t xb[4] = {wb & 0x0303u, wb & 0x0F0Fu, wb & 0x3F3Fu, (wb >> 2) & 0x3F3Fu};
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) f[4 * k + j] = make_float2(byte_f(xa[j], k), byte_f(xb[j], k));
     }
 }
 
-// Untangle one slice's value accumulators into its 8 channel sums
-// sum_t w_t c_t (without the zero-point term); W = sum_t w_t of its group.
+// Untangle one slice's value sums a[8] (in the encoding of value_pairs) into
+// its 8 channel sums sum_t w_t c_t (without the zero-point term);
+// W = sum_t w_t of its group.
 template <int VM, int VBITS>
-__device__ __forceinline__ void value_channels(const float2 o[4], float W, float out[8]) {
+__device__ __forceinline__ void value_channels(const float a[8], float W, float out[8]) {
     if constexpr (VM == V_BF16) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) { out[2 * c] = o[c].x; out[2 * c + 1] = o[c].y; }
+        for (int c = 0; c < 8; ++c) out[c] = a[c];
     } else if constexpr (VBITS == 4) {
-        // acc = sum w (0.5 + c/256)
+        // a = sum w (0.5 + c/256)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            out[2 * c] = fmaf(256.0f, o[c].x, -128.0f * W);
-            out[2 * c + 1] = fmaf(256.0f, o[c].y, -128.0f * W);
-        }
+        for (int c = 0; c < 8; ++c) out[c] = fmaf(256.0f, a[c], -128.0f * W);
     } else {
-        // acc_i = sum w (0.5 + X_i/256) with the X planes of value_pairs
+        // a_j = sum w (0.5 + X_j/256) with the X planes of value_pairs
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-            const float2 a = o[2 * b], c = o[2 * b + 1];
-            out[4 * b] = fmaf(256.0f, a.x, -128.0f * W);
-            out[4 * b + 1] = 64.0f * (a.y - a.x);
-            out[4 * b + 2] = 16.0f * (c.x - a.y);
-            out[4 * b + 3] = fmaf(16.0f, c.y, -8.0f * W) - 4.0f * (c.x - a.x);
+            const float x0 = a[4 * b], x1 = a[4 * b + 1], x2 = a[4 * b + 2], x3 = a[4 * b + 3];
+            out[4 * b] = fmaf(256.0f, x0, -128.0f * W);
+            out[4 * b + 1] = 64.0f * (x1 - x0);
+            out[4 * b + 2] = 16.0f * (x2 - x1);
+            out[4 * b + 3] = fmaf(16.0f, x3, -8.0f * W) - 4.0f * (x2 - x0);
         }
     }
 }
 
-template <int GQA>
-__device__ __forceinline__ void load_sums(const float *p, float v[GQA]) {
-    if constexpr (GQA == 4) {
-        const uint4 u = lds128(p);
-        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
-        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
-    } else {
+// ---- key coefficients -------------------------------------------------------
+// One head's key coefficients, built by one warp from the lane's 4 channels
+// x[0..3] (channels 4*lane..4*lane+3 of the rotated query, scaled to log2
+// units), in the padded chunk layout of RowGeo<KB> at `cg`, and the per-group
+// sums {init, qa} at sums[(group * GQA + g) * 2]:
+//   MODE 0 (token-wise groups, KB 4/2): coefficients 256 * a with a the plane
+//     coefficients of x; a row's dot product then comes out as
+//     128 * first_G + sum_G x c, so the accumulator starts at
+//     init = -128 * first_G; qa = sum_G x.
+//   MODE 1 (per-channel keys, KB 4/2): x is first multiplied by the block's
+//     channel scales `chan_sz`; one group, init = sum x z - 128 * first, so the
+//     dot product ends as q.k^.
+//   MODE 2 (bf16 keys): coefficients = x, init = 0.
+// GKC: compile-time group size (0: runtime gk).
+template <int GQA, int KB, int MODE, int GKC>
+__device__ __forceinline__ void build_head(const float xin[4], const uint8_t *chan_sz, float *cg,
+                                           float *sums, int g, int gk, int lane) {
+    using RG = RowGeo<KB>;
+    const int i0 = 4 * lane;  // the lane's 4 channels
+    const int G = (MODE == 0) ? (GKC ? GKC : gk) : kHeadDim;
+    float x[4] = {xin[0], xin[1], xin[2], xin[3]};
+    float qa = (x[0] + x[1]) + (x[2] + x[3]);
+    float qz = 0.0f;
+    if constexpr (MODE == 1) {
 #pragma unroll
-        for (int g = 0; g < GQA; ++g) v[g] = p[g];
+        for (int j = 0; j < 4; ++j) {
+            const float2 sz = half2_lds(chan_sz + (i0 + j) * 4);
+            qz = fmaf(x[j], sz.y, qz);
+            x[j] *= sz.x;
+        }
+    }
+    float cf[4], first;
+    if constexpr (KB == 16) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cf[j] = x[j];
+        first = 0.0f;
+    } else if constexpr (KB == 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cf[j] = 256.0f * x[j];
+        first = (x[0] + x[1]) + (x[2] + x[3]);
+    } else {
+        // a0 X0 + a1 X1 + a2 X2 + a3 X3 = x0 c0 + x1 c1 + x2 c2 + x3 c3
+        const float a3 = x[3] * 0.0625f;
+        const float a2 = (x[2] - 4.0f * a3) * 0.0625f;
+        const float a1 = (x[1] - 4.0f * a2 - a3) * 0.25f;
+        const float a0 = x[0] - a1 - a2;
+        cf[0] = 256.0f * a0; cf[1] = 256.0f * a1; cf[2] = 256.0f * a2; cf[3] = 256.0f * a3;
+        first = (a0 + a1) + (a2 + a3);
+    }
+    const int c = i0 / RG::cpc, j = i0 - c * RG::cpc;
+    *reinterpret_cast<float4 *>(cg + c * RG::cstr + j) = make_float4(cf[0], cf[1], cf[2], cf[3]);
+    if constexpr (MODE == 2) {
+        if (lane == 0) *reinterpret_cast<float2 *>(sums + g * 2) = make_float2(0.0f, 0.0f);
+        return;
+    }
+    const int lpg = G >> 2;  // lanes per group
+    if (GKC || MODE == 1) {
+#pragma unroll
+        for (int m = 1; m < ((MODE == 0) ? GKC : kHeadDim) / 4; m <<= 1) {
+            first += __shfl_xor_sync(0xffffffffu, first, m);
+            if (MODE == 0) qa += __shfl_xor_sync(0xffffffffu, qa, m);
+            if (MODE == 1) qz += __shfl_xor_sync(0xffffffffu, qz, m);
+        }
+    } else {
+        for (int m = 1; m < lpg; m <<= 1) {
+            first += __shfl_xor_sync(0xffffffffu, first, m);
+            qa += __shfl_xor_sync(0xffffffffu, qa, m);
+        }
+    }
+    if ((lane & (lpg - 1)) == 0) {
+        const int grp = i0 / G;
+        const float init = (MODE == 1) ? fmaf(-128.0f, first, qz) : -128.0f * first;
+        *reinterpret_cast<float2 *>(sums + (grp * GQA + g) * 2) = make_float2(init, qa);
     }
 }
-
-template <int GQA>
-struct LaneMap {
-    static constexpr int kPerHead = 8 / GQA;  // lanes of a token per head
-    static constexpr int kOwnShift = (GQA == 4) ? 1 : (GQA == 2 ? 2 : 3);
-};
-
-// Group-size geometry: compile-time when GK/GV > 0, else from the params.
-template <int GK, int GV, int GQA>
-struct Geo {
-    int gk_log2, gv_log2;
-    __device__ __forceinline__ int ngk() const { return GK ? kHeadDim / GK : kHeadDim >> gk_log2; }
-    __device__ __forceinline__ int nvg() const { return GV ? kHeadDim / GV : kHeadDim >> gv_log2; }
-    __device__ __forceinline__ int kgroup(int part) const { return GK ? (part * 16) / GK : (part * 16) >> gk_log2; }
-    __device__ __forceinline__ int vgroup(int slice) const { return GV ? (slice * 8) / GV : (slice * 8) >> gv_log2; }
-    __device__ __forceinline__ bool k_whole() const { return GK ? GK == kHeadDim : gk_log2 == 7; }
-    // value-group slots per owner lane
-    static constexpr int kVSlots =
-        GV ? ((kHeadDim / GV + LaneMap<GQA>::kPerHead - 1) / LaneMap<GQA>::kPerHead) : 4;
-};
 
 // Per-warp decode state of the current item.
-template <int GQA, int VSLOTS>
+template <int GQA, int NVG>
 struct WarpState {
-    float m_own;           // running max (log2 domain) used for this lane's head
-    float l_own;           // running sum of the weights of this lane's tokens (own head)
-    float wsum[VSLOTS];    // value groups owned by this lane: sum of p*s (own head)
-    float zsum[VSLOTS];    //                                   sum of p*z
-    float2 o[GQA][4];      // value accumulators: 8 channels (4 pairs) x GQA heads
+    float mref[GQA];       // reference maximum per head (log2 units; warp-uniform)
+    float thr[GQA];        // mref + slack: scores above it move the reference
+    float l[GQA];          // this lane's tokens: sum of the weights p
+    float W[GQA][NVG];     //                     sum of p * s per value group
+    float Z[GQA][NVG];     //                     sum of p * z per value group
+    float2 o[GQA][8];      // value accumulators: 8 channels x GQA heads, one
+                           // token of a pair in each half (summed at the end)
 };
 
-// Scores are kept in log2 units; a new tile maximum only moves the reference
-// when it exceeds the old one by more than this (weights then stay <= 2^8).
+// A new tile maximum moves the reference only when it exceeds the old one by
+// more than this (weights then stay <= 2^8).
 constexpr float kRescaleSlack = 8.0f;
 
-// Per-lane query data for the key pass. Per-lane sums the inner loop needs
-// once per pass live in shared memory (qsum, [8 parts][3][GQA] floats, head
-// order as in qk): [0] sum of q, [1] sum of the code-byte coefficients,
-// [2] channel-wise groups: sum q z - 128 * coefficient sum of q s.
-template <int GQA>
-struct QueryRegs {
-    float2 qk[GQA][8];     // coefficients, head order permuted for the reduce-scatter
-    float qa_own, qe_own;  // groups of 128: whole-head sums of the lane's own head
-};
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
+    return v;
+}
 
 // One tile: rows at kc / ks / vc / vs (shared memory), `n` valid tokens, TPW
-// tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)). FULL: all
-// 4*TPW tokens are valid, so no token needs masking.
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int TPW, int GK, int GV, int VSLOTS, bool FULL>
+// tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)).
+//   keys: lane j owns warp tokens j and j + 32 (TPW = 64) or token j (TPW <= 32);
+//   values: token pairs (p, p + TPW/2); the half-warps take alternate pairs,
+//     16 lanes cover the 128 channels (8 each); the weights of a pair sit
+//     side by side, so one f32x2 FMA serves both tokens.
+// FULL: all 4*TPW tokens are valid. KMT/KB: key mode and bits of this tile
+// (window tiles are bf16). GKC: compile-time key group size (0 = runtime
+// gk_rt); GVC likewise for the values (0 = runtime, NVG groups at most).
+template <int GQA, int KMT, int VMT, int KB, int VBITS, int TPW, int GKC, int GVC, int NVG, bool FULL>
 __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
                                              const uint8_t *vc, const uint8_t *vs, int n,
-                                             const Geo<GK, GV, GQA> geo, const QueryRegs<GQA> &Q,
-                                             const float *qsum, WarpState<GQA, VSLOTS> &st,
-                                             float *wsm, int warp, int lane) {
-    constexpr int KROW = KRow<KM, KBITS>::bytes;
-    constexpr int VROW = VRow<VM, VBITS>::bytes;
-    constexpr int PASSES = TPW / 4;
-    constexpr int kPerHead = LaneMap<GQA>::kPerHead;
-    constexpr int kOwnShift = LaneMap<GQA>::kOwnShift;
-    const int i = lane >> 3, part = lane & 7;
-    const int h_own = part >> kOwnShift;
-    const int r_own = part & (kPerHead - 1);  // rank of this lane among its head's lanes
-    const int n_vg = (VM == V_BF16) ? 1 : geo.nvg();
-    const int ngk = (KM == K_TOKEN) ? geo.ngk() : 0;
-    const bool post_scale = (KM == K_TOKEN) && geo.k_whole();
+                                             const float *coef, int hstr, int cstr,
+                                             const float *sums, int gk_rt, int gv_rt,
+                                             WarpState<GQA, NVG> &st, float *wsm, int warp,
+                                             int lane) {
+    using RG = RowGeo<KB>;
+    constexpr int TPL = (TPW >= 64) ? 2 : 1;  // key tokens per lane
+    constexpr int HALF = TPW / 2;             // value pair distance
+    constexpr int VROW = (VMT == V_BF16) ? kHeadDim * 2 : kHeadDim * VBITS / 8;
     const int t_warp = warp * TPW;
-
-    // ---- scores ----
-    float sc[PASSES];
+    int tr[TPL];
+    bool valid[TPL];
 #pragma unroll
-    for (int pass = 0; pass < PASSES; ++pass) {
-        const int tt = t_warp + pass * 4 + i;
-        const int tr = (FULL || tt < n) ? tt : 0;  // masked tokens read row 0 (always staged)
-        float2 f[8];
-        key_pairs<KM, KBITS>(kc + tr * KROW, part, f);
-        float acc[GQA];
+    for (int m = 0; m < TPL; ++m) {
+        const int tok = lane + 32 * m;
+        valid[m] = FULL || (tok < TPW && t_warp + tok < n);
+        tr[m] = valid[m] ? t_warp + tok : 0;  // masked lanes read row 0 (always staged)
+    }
+
+    // ---- keys: this lane's tokens against every head ----
+    const int G = (KMT == K_TOKEN) ? (GKC ? GKC : gk_rt) : kHeadDim;
+    const int ngk = kHeadDim / G;
+    const int rot = chunk_rot<KB>(lane);
+    float sc[TPL][GQA];
+    float2 acc[TPL][GQA];
+#pragma unroll
+    for (int m = 0; m < TPL; ++m)
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) sc[m][g] = 0.0f;
+    auto start_group = [&](int grp) {
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
-            float2 a = make_float2(0.0f, 0.0f);
+            const float init = (KMT == K_BF16) ? 0.0f : sums[(grp * GQA + g) * 2];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) ffma2(a, Q.qk[g][j], f[j]);
-            acc[g] = a.x + a.y;
+            for (int m = 0; m < TPL; ++m) acc[m][g] = make_float2(init, 0.0f);
         }
-        float2 szf = make_float2(0.0f, 0.0f);
-        if constexpr (KM == K_TOKEN) {
-            szf = half2_lds(ks + (tr * ngk + (post_scale ? 0 : geo.kgroup(part))) * 4);
-            if (!post_scale) {
-                float qa[GQA], qe[GQA];
-                load_sums<GQA>(qsum + (part * 3 + 0) * GQA, qa);
-                load_sums<GQA>(qsum + (part * 3 + 1) * GQA, qe);
+    };
+    auto end_group = [&](int grp) {
+        if constexpr (KMT == K_TOKEN) {
+            float qa[GQA];
+#pragma unroll
+            for (int g = 0; g < GQA; ++g) qa[g] = sums[(grp * GQA + g) * 2 + 1];
+#pragma unroll
+            for (int m = 0; m < TPL; ++m) {
+                const float2 sz = half2_lds(ks + (tr[m] * ngk + grp) * 4);
 #pragma unroll
                 for (int g = 0; g < GQA; ++g)
-                    acc[g] = fmaf(szf.x, fmaf(-128.0f, qe[g], acc[g]), szf.y * qa[g]);
+                    sc[m][g] = fmaf(sz.x, acc[m][g].x + acc[m][g].y, fmaf(sz.y, qa[g], sc[m][g]));
             }
-        } else if constexpr (KM == K_CHANNEL) {
-            float qc[GQA];
-            load_sums<GQA>(qsum + (part * 3 + 2) * GQA, qc);
-#pragma unroll
-            for (int g = 0; g < GQA; ++g) acc[g] += qc[g];
-        }
-        float val;
-        if constexpr (GQA == 4) {
-            // heads are held in the order g ^ (2*b2 + b1), so no selects
-            const float ka = acc[0] + __shfl_xor_sync(0xffffffffu, acc[2], 4);
-            const float kb = acc[1] + __shfl_xor_sync(0xffffffffu, acc[3], 4);
-            val = ka + __shfl_xor_sync(0xffffffffu, kb, 2);
-            val += __shfl_xor_sync(0xffffffffu, val, 1);
         } else {
+#pragma unroll
+            for (int m = 0; m < TPL; ++m)
+#pragma unroll
+                for (int g = 0; g < GQA; ++g) sc[m][g] = acc[m][g].x + acc[m][g].y;
+        }
+    };
+    const int cpg = G / RG::cpc;  // chunks per group (0: groups inside a chunk)
+    const int wpg = G / RG::cpw;  // words per group
+    if (KMT == K_BF16) start_group(0);
+#pragma unroll
+    for (int k = 0; k < RG::nch; ++k) {
+        const int c = k ^ rot;
+        if (KMT != K_BF16 && cpg > 0 && (k & (cpg - 1)) == 0) start_group(c / cpg);
+        uint32_t wv[TPL][4];
+#pragma unroll
+        for (int m = 0; m < TPL; ++m) {
+            const uint4 w4 = lds128(kc + tr[m] * RG::bytes + 16 * c);
+            wv[m][0] = w4.x; wv[m][1] = w4.y; wv[m][2] = w4.z; wv[m][3] = w4.w;
+        }
+        const float *cc = coef + c * cstr;
+        if constexpr (KB == 16) {
+            // 4 words = 8 channels; coefficients 8 floats per head
+            float2 f[TPL][4];
+#pragma unroll
+            for (int m = 0; m < TPL; ++m)
+#pragma unroll
+                for (int wi = 0; wi < 4; ++wi) word_pairs<16>(wv[m][wi], &f[m][wi]);
+            float4 cv[GQA][2];
 #pragma unroll
             for (int g = 0; g < GQA; ++g) {
-#pragma unroll
-                for (int m = 1; m < 8; m <<= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], m);
+                cv[g][0] = ldsf4(cc + g * hstr);
+                cv[g][1] = ldsf4(cc + g * hstr + 4);
             }
-            val = acc[0];
 #pragma unroll
-            for (int g = 1; g < GQA; ++g)
-                if (h_own == g) val = acc[g];
-        }
-        if constexpr (KM == K_TOKEN) {
-            if (post_scale) val = fmaf(szf.x, fmaf(-128.0f, Q.qe_own, val), szf.y * Q.qa_own);
-        }
-        sc[pass] = (FULL || tt < n) ? val : -INFINITY;
-    }
-
-    // ---- online softmax (per warp, per head), lazy rescaling ----
-    float mx = sc[0];
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int pass = 1; pass < PASSES; ++pass) mx = fmaxf(mx, sc[pass]);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    float alpha = 1.0f;
-    if (mx > st.m_own + kRescaleSlack) {   // also true the first time (m_own = -inf)
-        alpha = fast_exp2(st.m_own - mx);  // 0 when m_own = -inf
-        st.m_own = mx;
-    }
-    // reference 0 while no token of this warp has been seen (all sc = -inf)
-    const float mref = (st.m_own == -INFINITY) ? 0.0f : st.m_own;
-    float p[PASSES];
+                for (int m = 0; m < TPL; ++m)
 #pragma unroll
-    for (int k = 0; k < PASSES; ++k) p[k] = fast_exp2(sc[k] - mref);  // 0 for masked
-    float psum = p[0];
-#pragma unroll
-    for (int k = 1; k < PASSES; ++k) psum += p[k];
-    st.l_own = fmaf(st.l_own, alpha, psum);
-#pragma unroll
-    for (int c = 0; c < VSLOTS; ++c) {
-        st.wsum[c] *= alpha;
-        st.zsum[c] *= alpha;
-    }
-    // Value weights w = p * s per (token, value group), stored as a pair; the
-    // lanes of a head split the groups between them.
-#pragma unroll
-    for (int pass = 0; pass < PASSES; ++pass) {
-        const int j = pass * 4 + i;  // warp-local token index
-        const int tt = t_warp + j;
-        const int tr = (FULL || tt < n) ? tt : 0;
-        float2 *wrow = reinterpret_cast<float2 *>(wsm) + j * n_vg * GQA;
-        if constexpr (VM == V_BF16) {
-            if (r_own == 0) wrow[h_own] = make_float2(p[pass], p[pass]);
+                    for (int g = 0; g < GQA; ++g) {
+                        const float4 v = cv[g][j >> 1];
+                        ffma2(acc[m][g], (j & 1) ? make_float2(v.z, v.w) : make_float2(v.x, v.y), f[m][j]);
+                    }
         } else {
 #pragma unroll
-            for (int c = 0; c < VSLOTS; ++c) {
-                const int gv = r_own + c * kPerHead;
-                if (gv < n_vg) {
-                    const float2 szf = half2_lds(vs + (tr * n_vg + gv) * 4);
-                    const float w = p[pass] * szf.x;
-                    st.wsum[c] += w;
-                    st.zsum[c] = fmaf(p[pass], szf.y, st.zsum[c]);
-                    wrow[gv * GQA + h_own] = make_float2(w, w);
+            for (int wi = 0; wi < 4; ++wi) {
+                if (cpg == 0 && (wi & (wpg - 1)) == 0) start_group((c * 4 + wi) / wpg);
+                // blocks of 4 pairs: every head's coefficients first, then the
+                // multiply-adds interleaved across tokens and heads
+#pragma unroll
+                for (int jb = 0; jb < RG::npw; jb += 4) {
+                    float2 f[TPL][4];
+#pragma unroll
+                    for (int m = 0; m < TPL; ++m) word_pairs4<KB>(wv[m][wi], jb, f[m]);
+                    float4 cv[GQA][2];
+#pragma unroll
+                    for (int g = 0; g < GQA; ++g) {
+                        const float *cw = cc + g * hstr + wi * RG::cpw + 2 * jb;
+                        cv[g][0] = ldsf4(cw);
+                        cv[g][1] = ldsf4(cw + 4);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int m = 0; m < TPL; ++m)
+#pragma unroll
+                            for (int g = 0; g < GQA; ++g) {
+                                const float4 v = cv[g][j >> 1];
+                                ffma2(acc[m][g], (j & 1) ? make_float2(v.z, v.w) : make_float2(v.x, v.y),
+                                      f[m][j]);
+                            }
                 }
+                if (cpg == 0 && ((wi + 1) & (wpg - 1)) == 0) end_group((c * 4 + wi) / wpg);
+            }
+        }
+        if (KMT != K_BF16 && cpg > 0 && ((k + 1) & (cpg - 1)) == 0) end_group(c / cpg);
+    }
+    if (KMT == K_BF16) end_group(0);
+#pragma unroll
+    for (int m = 0; m < TPL; ++m)
+        if (!valid[m]) {
+#pragma unroll
+            for (int g = 0; g < GQA; ++g) sc[m][g] = -INFINITY;
+        }
+
+    // ---- online softmax (per warp, per head), lazy reference ----
+    bool up = false;
+#pragma unroll
+    for (int m = 0; m < TPL; ++m)
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) up |= sc[m][g] > st.thr[g];
+    if (__any_sync(0xffffffffu, up)) {
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) {
+            float mx = sc[0][g];
+#pragma unroll
+            for (int m = 1; m < TPL; ++m) mx = fmaxf(mx, sc[m][g]);
+            mx = warp_max(mx);
+            if (mx > st.thr[g]) {  // also true the first time (thr = -inf)
+                const float alpha = (st.mref[g] == -INFINITY) ? 0.0f : fast_exp2(st.mref[g] - mx);
+                st.mref[g] = mx;
+                st.thr[g] = mx + kRescaleSlack;
+                st.l[g] *= alpha;
+#pragma unroll
+                for (int v = 0; v < NVG; ++v) { st.W[g][v] *= alpha; st.Z[g][v] *= alpha; }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) { st.o[g][c].x *= alpha; st.o[g][c].y *= alpha; }
             }
         }
     }
-    float alpha_g[GQA];
-    bool rescale = false;
+    float p[TPL][GQA];
 #pragma unroll
     for (int g = 0; g < GQA; ++g) {
-        alpha_g[g] = __shfl_sync(0xffffffffu, alpha, g << kOwnShift);
-        rescale |= alpha_g[g] != 1.0f;
+        // reference 0 while no token of this warp has been seen (all -inf)
+        const float mref = (st.mref[g] == -INFINITY) ? 0.0f : st.mref[g];
+#pragma unroll
+        for (int m = 0; m < TPL; ++m) {
+            p[m][g] = fast_exp2(sc[m][g] - mref);  // 0 for masked tokens
+            st.l[g] += p[m][g];
+        }
+    }
+    // Value weights w = p * s per (token, value group), at their pair slot.
+    const int n_vg = (VMT == V_BF16) ? 1 : (GVC ? kHeadDim / GVC : kHeadDim / gv_rt);
+    float2 *wsm2 = reinterpret_cast<float2 *>(wsm);
+#pragma unroll
+    for (int v = 0; v < ((VMT == V_BF16) ? 1 : NVG); ++v) {
+        if (v < n_vg) {
+            float w[TPL][GQA];
+            if constexpr (VMT == V_BF16) {
+#pragma unroll
+                for (int m = 0; m < TPL; ++m)
+#pragma unroll
+                    for (int g = 0; g < GQA; ++g) w[m][g] = p[m][g];
+            } else {
+#pragma unroll
+                for (int m = 0; m < TPL; ++m) {
+                    const float2 szf = half2_lds(vs + (tr[m] * n_vg + v) * 4);
+#pragma unroll
+                    for (int g = 0; g < GQA; ++g) {
+                        w[m][g] = p[m][g] * szf.x;
+                        st.W[g][v] += w[m][g];
+                        st.Z[g][v] = fmaf(p[m][g], szf.y, st.Z[g][v]);
+                    }
+                }
+            }
+            if constexpr (TPL == 2) {  // lane j owns pair j: both halves
+#pragma unroll
+                for (int g = 0; g < GQA; ++g) wsm2[(lane * n_vg + v) * GQA + g] = make_float2(w[0][g], w[1][g]);
+            } else if (lane < TPW) {
+                const int slot = lane % HALF, half = lane / HALF;
+#pragma unroll
+                for (int g = 0; g < GQA; ++g) wsm[((slot * n_vg + v) * GQA + g) * 2 + half] = w[0][g];
+            }
+        }
     }
     __syncwarp();
 
     // ---- values ----
     const int slice = lane & 15, parity = lane >> 4;
-    if (rescale) {
+    const int gv_lane = (VMT == V_BF16) ? 0 : (slice * 8) / (GVC ? GVC : gv_rt);
+#pragma unroll 2
+    for (int k = 0; k < HALF / 2; ++k) {
+        const int pi = 2 * k + parity;
+        const int ta = t_warp + pi, tb = ta + HALF;
+        float2 f[8];
+        value_pairs<VMT, VBITS>(vc + ta * VROW, vc + tb * VROW, slice, f);
+        if (VMT == V_BF16 && !FULL) {  // stale bf16 rows may be NaN: drop them
+            const bool va = ta < n, vb = tb < n;
 #pragma unroll
-        for (int g = 0; g < GQA; ++g)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                st.o[g][c].x *= alpha_g[g];
-                st.o[g][c].y *= alpha_g[g];
+            for (int c = 0; c < 8; ++c) {
+                f[c].x = va ? f[c].x : 0.0f;
+                f[c].y = vb ? f[c].y : 0.0f;
             }
-    }
-    const int gv_lane = (VM == V_BF16) ? 0 : geo.vgroup(slice);
-#pragma unroll
-    for (int k = 0; k < TPW / 2; ++k) {
-        const int j = 2 * k + parity;
-        const int tt = t_warp + j;
-        if (VM == V_BF16 && !FULL && tt >= n) continue;  // stale bf16 rows may be NaN
-        float2 f[4];
-        value_pairs<VM, VBITS>(vc + tt * VROW, slice, f);
-        const float2 *wrow = reinterpret_cast<const float2 *>(wsm) + (j * n_vg + gv_lane) * GQA;
+        }
+        const float2 *wrow = wsm2 + (pi * n_vg + gv_lane) * GQA;
         float2 w[GQA];
         if constexpr (GQA >= 2) {
 #pragma unroll
@@ -489,7 +621,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 #pragma unroll
         for (int g = 0; g < GQA; ++g)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) ffma2(st.o[g][c], w[g], f[c]);
+            for (int c = 0; c < 8; ++c) ffma2(st.o[g][c], w[g], f[c]);
     }
     __syncwarp();
 }
@@ -509,27 +641,46 @@ __device__ __forceinline__ void item_coords(const int *pref, int S, int H, int i
     kvh = r - split * H;
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int NS, int GK, int GV>
-__global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk_kernel(const DecodeParams p) {
+// Expected-transaction bytes for a bulk copy issued by this thread, without an
+// arrival (the producer's lane 0 arrives once all lanes have added theirs).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Resident CTAs per SM the register budget targets: two, but one for the
+// generic variants (up to 8 value groups of W/Z per lane) and for bf16 caches
+// (whose 128-token stages take 66 KB each).
+constexpr int decode_min_blocks(int km, int vm, int gvc) {
+    return km == K_BF16 ? 1 : ((vm == V_TOKEN && gvc == 0) ? 1 : 2);
+}
+
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int GKC, int GVC>
+__global__ void __launch_bounds__(kThreads, decode_min_blocks(KM, VM, GVC))
+decode_splitk_kernel(const DecodeParams p) {
+    constexpr int NVG = (VM == V_BF16) ? 1 : (GVC ? kHeadDim / GVC : kMaxGroups);
+    constexpr int KBF = (KM == K_BF16) ? 16 : KBITS;  // key form of quantized tiles
+    constexpr int TILE = (KM == K_BF16) ? kTileB : kTileQ;
+    constexpr int TPW = TILE / kConsumerWarps;
+    using RG = RowGeo<KBF>;
+    constexpr int QHSTR = RG::nch * RG::cstr;                 // coefficient floats per head
+    constexpr int CBUF = GQA * QHSTR + kMaxGroups * GQA * 2;  // coefficients + group sums
     extern __shared__ __align__(128) uint8_t smem[];
-    using G = Geo<GK, GV, GQA>;
-    constexpr int VSLOTS = G::kVSlots;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const G geo{p.gk_log2, p.gv_log2};
+    const int NS = p.ns;
 
     uint8_t *stages = smem;
     uint8_t *tail = smem + static_cast<size_t>(NS) * p.stage_bytes;
     float *qs = reinterpret_cast<float *>(tail);                    // [GQA][128]
-    // value weights per warp: [token of the warp][value group][GQA][2]
-    float *wsm_all = qs + GQA * kHeadDim;
-    float *red = wsm_all + kConsumerWarps * p.wsm_floats;            // [4][GQA][130]
-    float *qsum_all = red + kConsumerWarps * GQA * 130;              // [4][8][3][GQA]
-    float *qhead = qsum_all + kConsumerWarps * 8 * 3 * GQA;          // [2][GQA]
-    uint64_t *full = reinterpret_cast<uint64_t *>(qhead + 2 * GQA + 2);
-    uint64_t *empty = full + NS;
-    int *abort_word = reinterpret_cast<int *>(empty + NS);
+    float *coefs = qs + GQA * kHeadDim;                              // [n_sets][CBUF], CTA-shared
+    float *scratch_all = coefs + p.n_sets * CBUF;                    // [4][warp_floats]
+    uint64_t *full = reinterpret_cast<uint64_t *>(scratch_all + kConsumerWarps * p.warp_floats);
+    uint64_t *empty = full + kMaxStages;
+    int *abort_word = reinterpret_cast<int *>(empty + kMaxStages);
     volatile int *abort_flag = abort_word;
     int *pref = abort_word + 4;  // [S + 1]
+    int *lens = pref + p.S + 1;  // [S] clamped lengths
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -542,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
     __syncthreads();
     // A dependent launch (the merge pass) may be scheduled from now on; it
     // waits for this grid's completion before reading anything.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_launch_dependents();
 
     if (warp == kConsumerWarps) {
         // ------------------------- producer -------------------------
@@ -550,14 +701,14 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
         int carry = 0;
         for (int base = 0; base < p.S; base += 32) {
             const int s = base + lane;
-            int cnt = 0;
+            int cnt = 0, T_s = 0;
             if (s < p.S) {
-                int T = __ldg(p.seq_lens + s);
-                if (T > p.max_seq_len) {
+                T_s = __ldg(p.seq_lens + s);
+                if (T_s > p.max_seq_len) {
                     if (blockIdx.x == 0) status_or(p.status, KVQ_DEV_SEQLEN);
-                    T = p.max_seq_len;
+                    T_s = p.max_seq_len;
                 }
-                cnt = T > 0 ? p.H * ((T + p.chunk - 1) / p.chunk) : 0;
+                cnt = T_s > 0 ? p.H * ((T_s + p.chunk - 1) / p.chunk) : 0;
             }
             int incl = cnt;
 #pragma unroll
@@ -565,34 +716,39 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
                 const int o = __shfl_up_sync(0xffffffffu, incl, m);
                 if (lane >= m) incl += o;
             }
-            if (s < p.S) pref[s] = carry + incl - cnt;
+            if (s < p.S) {
+                pref[s] = carry + incl - cnt;
+                lens[s] = T_s;
+            }
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0) pref[p.S] = carry;
         __syncwarp();
-        if (lane != 0) return;
         const int n_items = carry;
 
-        constexpr int KROW = KRow<KM, KBITS>::bytes;
-        constexpr int VROW = VRow<VM, VBITS>::bytes;
-        const int ngk = (KM == K_TOKEN) ? geo.ngk() : 0;
-        const int ngv = (VM == V_TOKEN) ? geo.nvg() : 0;
+        constexpr int KROW = RowGeo<KBF>::bytes;
+        constexpr int VROW = (VM == V_BF16) ? kHeadDim * 2 : kHeadDim * VBITS / 8;
+        const int ngk = (KM == K_TOKEN) ? kHeadDim / p.gk : 0;
+        const int ngv = (VM == V_TOKEN) ? kHeadDim / p.gv : 0;
         int it = 0;  // tile counter of this CTA (stage it % NS, round it / NS)
         bool stop = false;
-        // Quantized tiles never straddle a block of per-channel key scales.
-        const int qtile = (KM == K_CHANNEL) ? min(kTile, p.R) : kTile;
+        // The next item is claimed one item ahead, so the atomic's latency
+        // hides behind the current item's copies.
+        int next = 0;
+        if (lane == 0) next = atomicAdd(p.counter, 1);
         while (!stop) {
-            const int item = atomicAdd(p.counter, 1);
+            int item = __shfl_sync(0xffffffffu, next, 0);
+            if (lane == 0 && item < n_items) next = atomicAdd(p.counter, 1);
             int seq = 0, kvh = 0, split = 0;
             int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0;
             if (item < n_items) {
                 item_coords(pref, p.S, p.H, item, seq, kvh, split);
-                const int T = min(__ldg(p.seq_lens + seq), p.max_seq_len);
+                const int T = lens[seq];
                 t_begin = split * p.chunk;
                 t_end = min(T, t_begin + p.chunk);
                 Tq = quantized_len(T, p.R);
                 q_end = min(t_end, Tq);
-                n_qt = q_end > t_begin ? (q_end - t_begin + qtile - 1) / qtile : 0;
+                n_qt = q_end > t_begin ? (q_end - t_begin + TILE - 1) / TILE : 0;
                 w_begin = max(t_begin, Tq);
                 n_wt = t_end > w_begin ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
             }
@@ -600,8 +756,10 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
             const int64_t sh = static_cast<int64_t>(seq) * p.H + kvh;
             for (int ti = 0; ti < n_tiles; ++ti, ++it) {
                 const int s = it % NS, r = it / NS;
-                if (r > 0 &&
-                    !mbar_wait_bounded(&empty[s], (r - 1) & 1, p.timeout_ns, p.status, abort_flag)) {
+                int ok = 1;
+                if (lane == 0 && r > 0)
+                    ok = mbar_wait_bounded(&empty[s], (r - 1) & 1, p.timeout_ns, p.status, abort_flag);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     stop = true;
                     break;
                 }
@@ -609,83 +767,104 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
                 uint64_t *bar = &full[s];
                 TileHdr *hdr = reinterpret_cast<TileHdr *>(st + p.off_hdr);
                 if (item >= n_items) {  // no work left: tell the consumers
-                    hdr->flags = kDone;
-                    mbar_arrive(bar);
+                    if (lane == 0) {
+                        hdr->flags = kDone;
+                        mbar_arrive(bar);
+                    }
                     stop = true;
                     ++it;
                     break;
                 }
                 if (it == p.skip_tile) continue;  // test hook: never arrive
                 const bool window = ti >= n_qt;
-                const int t0 = window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * qtile;
-                const int n = window ? min(p.bf_tile, t_end - t0) : min(qtile, q_end - t0);
-                hdr->seq = seq;
-                hdr->kvh = kvh;
-                hdr->split = split;
-                hdr->t0 = t0;
-                hdr->n = n;
-                hdr->flags = (ti == 0 ? kFirst : 0) | (ti == n_tiles - 1 ? kLast : 0) | (window ? kWindow : 0);
+                const int t0 = window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * TILE;
+                const int n = window ? min(p.bf_tile, t_end - t0) : min(TILE, q_end - t0);
+                if (lane == 0) {
+                    hdr->seq = seq;
+                    hdr->kvh = kvh;
+                    hdr->split = split;
+                    hdr->t0 = t0;
+                    hdr->n = n;
+                    hdr->flags = (ti == 0 ? kFirst : 0) | (ti == n_tiles - 1 ? kLast : 0) | (window ? kWindow : 0);
+                }
                 const uint32_t qb = (ti == 0) ? GQA * kHeadDim * p.q_bytes : 0;
-                const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
-                                      ((static_cast<int64_t>(seq) * p.Hq + kvh * GQA) * kHeadDim) * p.q_bytes;
+                if (qb && lane == 31) {  // the item's query rows ride with its first tile
+                    const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
+                                          ((static_cast<int64_t>(seq) * p.Hq + kvh * GQA) * kHeadDim) * p.q_bytes;
+                    mbar_expect_tx(bar, qb);
+                    bulk_g2s(st + p.off_q, qsrc, qb, bar);
+                }
                 if (window) {
                     const uint32_t bytes = n * kHeadDim * 2;
                     const int64_t slot = sh * p.R + (t0 - Tq);
-                    mbar_arrive_expect_tx(bar, 2 * bytes + qb);
-                    bulk_g2s(st, p.k_res + slot * kHeadDim, bytes, bar);
-                    bulk_g2s(st + p.bf_off_v, p.v_res + slot * kHeadDim, bytes, bar);
-                } else if (!p.paged) {
-                    const int64_t row = sh * p.cap + t0;
-                    const uint32_t kb = n * KROW, vb = n * VROW;
-                    const uint32_t kzb = (KM == K_TOKEN) ? ((n * ngk * 4 + 15) & ~15)
-                                                         : (KM == K_CHANNEL ? kHeadDim * 4 : 0);
-                    const uint32_t vzb = (VM == V_TOKEN) ? ((n * ngv * 4 + 15) & ~15) : 0;
-                    mbar_arrive_expect_tx(bar, kb + vb + kzb + vzb + qb);
-                    bulk_g2s(st, p.k_codes + row * KROW, kb, bar);
-                    bulk_g2s(st + p.off_vc, p.v_codes + row * VROW, vb, bar);
-                    if (KM == K_TOKEN) bulk_g2s(st + p.off_ksz, p.k_sz + row * ngk, kzb, bar);
-                    if (KM == K_CHANNEL)
-                        bulk_g2s(st + p.off_ksz, p.k_sz + (sh * (p.cap / p.R) + t0 / p.R) * kHeadDim, kzb, bar);
-                    if (VM == V_TOKEN) bulk_g2s(st + p.off_vsz, p.v_sz + row * ngv, vzb, bar);
-                } else {
-                    // Paged (token-wise groups only): one copy of each part per page.
-                    const int ps = p.page_size;
-                    const int span = ps < kTile ? ps : kTile;  // tokens per copy
-                    const uint32_t per_copy = span * (KROW + VROW + 4 * ngk + 4 * ngv);
-                    const int32_t *bt = p.block_table + static_cast<int64_t>(seq) * p.max_pages;
-                    uint32_t bytes = qb;
-                    for (int tp = t0; tp < t0 + n; tp += span) {
-                        const int pi = tp / ps;
-                        const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
-                        if (page >= 0 && page < p.num_pages) bytes += per_copy;
-                        else status_or(p.status, KVQ_DEV_CAPACITY);
+                    if (lane < 2) {
+                        mbar_expect_tx(bar, bytes);
+                        if (lane == 0) bulk_g2s(st, p.k_res + slot * kHeadDim, bytes, bar);
+                        else bulk_g2s(st + p.bf_off_v, p.v_res + slot * kHeadDim, bytes, bar);
                     }
-                    mbar_arrive_expect_tx(bar, bytes);
-                    for (int tp = t0; tp < t0 + n; tp += span) {
+                } else if (!p.paged) {
+                    // one lane per part: K codes, V codes, K scale/zero, V scale/zero
+                    const int64_t row = sh * p.cap + t0;
+                    if (lane == 0) {
+                        mbar_expect_tx(bar, n * KROW);
+                        bulk_g2s(st, p.k_codes + row * KROW, n * KROW, bar);
+                    } else if (lane == 1) {
+                        mbar_expect_tx(bar, n * VROW);
+                        bulk_g2s(st + p.off_vc, p.v_codes + row * VROW, n * VROW, bar);
+                    } else if (lane == 2 && KM == K_TOKEN) {
+                        const uint32_t b = (n * ngk * 4 + 15) & ~15;
+                        mbar_expect_tx(bar, b);
+                        bulk_g2s(st + p.off_ksz, p.k_sz + row * ngk, b, bar);
+                    } else if (lane == 2 && KM == K_CHANNEL) {
+                        // the channel scales of every block the tile touches
+                        const int b0 = t0 / p.R, nb = (t0 + n - 1) / p.R - b0 + 1;
+                        mbar_expect_tx(bar, nb * kHeadDim * 4);
+                        bulk_g2s(st + p.off_ksz, p.k_sz + (sh * (p.cap / p.R) + b0) * kHeadDim,
+                                 nb * kHeadDim * 4, bar);
+                    } else if (lane == 3 && VM == V_TOKEN) {
+                        const uint32_t b = (n * ngv * 4 + 15) & ~15;
+                        mbar_expect_tx(bar, b);
+                        bulk_g2s(st + p.off_vsz, p.v_sz + row * ngv, b, bar);
+                    }
+                } else {
+                    // Paged (token-wise groups only): one lane per page (or per
+                    // tile-sized span of a larger page), four copies each.
+                    const int ps = p.page_size;
+                    const int span = ps < TILE ? ps : TILE;  // tokens per copy
+                    const int tp = t0 + lane * span;
+                    if (tp < t0 + n) {
+                        const int32_t *bt = p.block_table + static_cast<int64_t>(seq) * p.max_pages;
                         const int pi = tp / ps;
                         const int page = (pi < p.max_pages) ? __ldg(bt + pi) : -1;
-                        if (page < 0 || page >= p.num_pages) continue;
-                        const int64_t prow = (static_cast<int64_t>(page) * p.H + kvh) * ps + (tp % ps);
-                        const uint32_t dt = tp - t0;
-                        bulk_g2s(st + dt * KROW, p.k_codes + prow * KROW, span * KROW, bar);
-                        bulk_g2s(st + p.off_ksz + dt * ngk * 4, p.k_sz + prow * ngk, span * ngk * 4, bar);
-                        bulk_g2s(st + p.off_vc + dt * VROW, p.v_codes + prow * VROW, span * VROW, bar);
-                        bulk_g2s(st + p.off_vsz + dt * ngv * 4, p.v_sz + prow * ngv, span * ngv * 4, bar);
+                        if (page >= 0 && page < p.num_pages) {
+                            const int64_t prow = (static_cast<int64_t>(page) * p.H + kvh) * ps + (tp % ps);
+                            const uint32_t dt = tp - t0;
+                            mbar_expect_tx(bar, span * (KROW + VROW + 4 * ngk + 4 * ngv));
+                            bulk_g2s(st + dt * KROW, p.k_codes + prow * KROW, span * KROW, bar);
+                            bulk_g2s(st + p.off_ksz + dt * ngk * 4, p.k_sz + prow * ngk, span * ngk * 4, bar);
+                            bulk_g2s(st + p.off_vc + dt * VROW, p.v_codes + prow * VROW, span * VROW, bar);
+                            bulk_g2s(st + p.off_vsz + dt * ngv * 4, p.v_sz + prow * ngv, span * ngv * 4, bar);
+                        } else {
+                            status_or(p.status, KVQ_DEV_CAPACITY);
+                        }
                     }
                 }
-                if (qb) bulk_g2s(st + p.off_q, qsrc, qb, bar);
+                __syncwarp();  // every lane has added its bytes before the arrival
+                if (lane == 0) mbar_arrive(bar);
             }
         }
         // Drain: wait for the copies of the last stages issued so none lands
         // after the CTA has gone.
-        for (int j = max(0, it - NS); j < it; ++j) {
-            if (j == p.skip_tile) continue;
-            const int s = j % NS, r = j / NS;
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(&full[s], r & 1)) {
-                if (static_cast<int64_t>(global_timer_ns() - t0) > p.timeout_ns) {
-                    status_or(p.status, KVQ_DEV_TIMEOUT);
-                    break;
+        if (lane == 0) {
+            for (int j = max(0, it - NS); j < it; ++j) {
+                if (j == p.skip_tile) continue;
+                const int s = j % NS, r = j / NS;
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(&full[s], r & 1)) {
+                    if (static_cast<int64_t>(global_timer_ns() - t0) > p.timeout_ns) {
+                        status_or(p.status, KVQ_DEV_TIMEOUT);
+                        break;
+                    }
                 }
             }
         }
@@ -693,95 +872,62 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
     }
 
     // --------------------------- consumers ---------------------------
-    const int part = lane & 7;
-    constexpr int kOwnShift = LaneMap<GQA>::kOwnShift;
-    // head held in register slot g (reduce-scatter order for GQA 4)
-    const int perm = (GQA == 4) ? (((part >> 2) & 1) << 1 | ((part >> 1) & 1)) : 0;
-    QueryRegs<GQA> Q;
-    float *qsum = qsum_all + warp * 8 * 3 * GQA;
-    float *wsm = wsm_all + warp * p.wsm_floats;
+    float *scratch = scratch_all + warp * p.warp_floats;
+    float *wsm = scratch;                  // value weights / W-Z partials of the lanes
+    float *totals = scratch + p.off_tot;   // W-Z totals of the warp
+    float *red = scratch;                  // item merge (after the last tile), [GQA][132]
+    constexpr int RSTR = 132;
+    const int slice = lane & 15;
 
-    // mode: 0 = token-wise codes, 1 = channel-wise codes (per-channel scales
-    // folded in from `chan_sz`), 2 = bf16 keys.
-    auto load_query = [&](int mode, const uint8_t *chan_sz) {
-        __syncwarp();  // this warp is done reading the previous sums
-#pragma unroll
-        for (int g = 0; g < GQA; ++g) {
-            const int h = g ^ perm;
-            float x[16];
-            float qa = 0.0f, qz = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float v = qs[h * kHeadDim + part * 16 + j];
-                qa += v;
-                if (mode == 1) {
-                    const float2 sz = half2_lds(chan_sz + (part * 16 + j) * 4);
-                    x[j] = v * sz.x;
-                    qz = fmaf(v, sz.y, qz);
-                } else {
-                    x[j] = v;
-                }
-            }
-            float first;
-            if (mode == 2) query_coeffs<K_BF16, 16>(x, Q.qk[g], first);
-            else query_coeffs<KM == K_BF16 ? K_TOKEN : KM, KBITS == 16 ? 4 : KBITS>(x, Q.qk[g], first);
-            if ((lane >> 3) == 0) {
-                qsum[(part * 3 + 0) * GQA + g] = qa;
-                qsum[(part * 3 + 1) * GQA + g] = first;
-                qsum[(part * 3 + 2) * GQA + g] = (mode == 1) ? fmaf(-128.0f, first, qz) : 0.0f;
-            }
-        }
-        // whole-head sums of the lane's own head (written by the item prologue)
-        Q.qa_own = qhead[part >> kOwnShift];
-        Q.qe_own = qhead[GQA + (part >> kOwnShift)];
-        __syncwarp();
-    };
-
-    WarpState<GQA, VSLOTS> st;
+    WarpState<GQA, NVG> st;
     bool folded = false;
     // Turn the value accumulators of quantized tiles into plain channel sums
     // (adding the zero-point terms), once: before the first bf16 window tile
-    // or at the end of the item. Half-warp 1 adds no group terms, so the
-    // halves still sum.
+    // or at the end of the item. The lanes' W/Z partials are summed through
+    // shared memory (one column per lane). Half-warp 1 adds no group terms, so
+    // the halves still sum.
     auto fold_values = [&]() {
-        constexpr int kPH = LaneMap<GQA>::kPerHead;
-        float wsum[VSLOTS], zsum[VSLOTS];
+        const int n_vg = GVC ? kHeadDim / GVC : kHeadDim / p.gv;
+        const int nv = 2 * GQA * n_vg;  // values per lane: W then Z, [g][v]
 #pragma unroll
-        for (int c = 0; c < VSLOTS; ++c) {
-            wsum[c] = st.wsum[c];
-            wsum[c] += __shfl_xor_sync(0xffffffffu, wsum[c], 8);
-            wsum[c] += __shfl_xor_sync(0xffffffffu, wsum[c], 16);
-            zsum[c] = st.zsum[c];
-            zsum[c] += __shfl_xor_sync(0xffffffffu, zsum[c], 8);
-            zsum[c] += __shfl_xor_sync(0xffffffffu, zsum[c], 16);
-            st.wsum[c] = 0.0f;
-            st.zsum[c] = 0.0f;
+        for (int g = 0; g < GQA; ++g)
+#pragma unroll
+            for (int v = 0; v < NVG; ++v)
+                if (v < n_vg) {
+                    wsm[lane * nv + g * n_vg + v] = st.W[g][v];
+                    wsm[lane * nv + GQA * n_vg + g * n_vg + v] = st.Z[g][v];
+                }
+        __syncwarp();
+        for (int col = lane; col < nv; col += 32) {
+            float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 32; r += 2) {
+                a0 += wsm[r * nv + col];
+                a1 += wsm[(r + 1) * nv + col];
+            }
+            totals[col] = a0 + a1;
         }
-        const int gv_lane = geo.vgroup(lane & 15);
+        __syncwarp();
+        const int gv_lane = (slice * 8) / (GVC ? GVC : p.gv);
         const bool first_half = lane < 16;
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
-            // group gv of head g: lane (g << kOwnShift) + gv % kPH, slot gv / kPH
-            float Wg = 0.0f, Zg = 0.0f;
+            const float Wg = first_half ? totals[g * n_vg + gv_lane] : 0.0f;
+            const float Zg = first_half ? totals[GQA * n_vg + g * n_vg + gv_lane] : 0.0f;
+            float a[8], ch[8];
 #pragma unroll
-            for (int c = 0; c < VSLOTS; ++c) {
+            for (int c = 0; c < 8; ++c) a[c] = st.o[g][c].x + st.o[g][c].y;
+            value_channels<VM, VBITS>(a, Wg, ch);
 #pragma unroll
-                for (int r = 0; r < kPH; ++r) {
-                    const float wv = __shfl_sync(0xffffffffu, wsum[c], (g << kOwnShift) + r);
-                    const float zv = __shfl_sync(0xffffffffu, zsum[c], (g << kOwnShift) + r);
-                    if (gv_lane == r + c * kPH) { Wg = wv; Zg = zv; }
-                }
-            }
-            if (!first_half) { Wg = 0.0f; Zg = 0.0f; }
-            float ch[8];
-            value_channels<VM, VBITS>(st.o[g], Wg, ch);
+            for (int c = 0; c < 8; ++c) st.o[g][c] = make_float2(ch[c] + Zg, 0.0f);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) st.o[g][c] = make_float2(ch[2 * c] + Zg, ch[2 * c + 1] + Zg);
+            for (int v = 0; v < NVG; ++v) { st.W[g][v] = 0.0f; st.Z[g][v] = 0.0f; }
         }
+        __syncwarp();
         folded = true;
     };
 
-    int cur_block = -1;
+    int kc_tiles = 0;  // quantized tiles seen (parity of the per-channel coefficient sets)
     for (int it = 0;; ++it) {
         const int s = it % NS, r = it / NS;
         if (!mbar_wait_bounded(&full[s], r & 1, p.timeout_ns, p.status, abort_flag)) break;
@@ -791,6 +937,8 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
 
         if (hdr.flags & kFirst) {
             // ---- item prologue: the query rows arrived with this tile ----
+            // Warp g rotates head g, stores it (window tiles and per-channel
+            // rebuilds read it) and builds the head's key coefficients.
             if (warp < GQA) {
                 const uint8_t *qrow = sb + p.off_q + warp * kHeadDim * p.q_bytes;
                 float x[4];
@@ -828,109 +976,116 @@ __global__ void __launch_bounds__(kThreads, KVQ_DECODE_MIN_BLOCKS) decode_splitk
 #pragma unroll
                     for (int j = 0; j < 4; ++j) x[j] *= p.hscale;
                 }
-                float sa = 0.0f, se = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    x[j] *= p.qscale;
-                    qs[warp * kHeadDim + 4 * lane + j] = x[j];
-                    sa += x[j];
-                    // sum of the code-byte coefficients: all q (INT4), q0 + q3/16 (INT2)
-                    se += (KBITS != 2) ? x[j] : (j == 0 ? x[j] : (j == 3 ? 0.0625f * x[j] : 0.0f));
-                }
-#pragma unroll
-                for (int m = 1; m < 32; m <<= 1) {
-                    sa += __shfl_xor_sync(0xffffffffu, sa, m);
-                    se += __shfl_xor_sync(0xffffffffu, se, m);
-                }
-                if (lane == 0) {
-                    qhead[warp] = sa;
-                    qhead[GQA + warp] = se;
-                }
+                for (int j = 0; j < 4; ++j) x[j] *= p.qscale;
+                *reinterpret_cast<float4 *>(qs + warp * kHeadDim + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
+                if constexpr (KM == K_TOKEN)
+                    build_head<GQA, KBF, 0, GKC>(x, nullptr, coefs + warp * QHSTR, coefs + GQA * QHSTR, warp, p.gk, lane);
+                if constexpr (KM == K_BF16)
+                    build_head<GQA, 16, 2, 0>(x, nullptr, coefs + warp * QHSTR, coefs + GQA * QHSTR, warp, 128, lane);
             }
             named_sync(1, kConsumers);
-            cur_block = -1;
-            if constexpr (KM != K_CHANNEL) load_query(KM == K_BF16 ? 2 : 0, nullptr);
-            st.m_own = -INFINITY;
-            st.l_own = 0.0f;
 #pragma unroll
-            for (int c = 0; c < VSLOTS; ++c) { st.wsum[c] = 0.0f; st.zsum[c] = 0.0f; }
+            for (int g = 0; g < GQA; ++g) {
+                st.mref[g] = -INFINITY;
+                st.thr[g] = -INFINITY;
+                st.l[g] = 0.0f;
 #pragma unroll
-            for (int g = 0; g < GQA; ++g)
+                for (int v = 0; v < NVG; ++v) { st.W[g][v] = 0.0f; st.Z[g][v] = 0.0f; }
 #pragma unroll
-                for (int c = 0; c < 4; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
+                for (int c = 0; c < 8; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
+            }
             folded = false;
         }
 
         if (!(hdr.flags & kWindow)) {
+            const float *coef = coefs;
             if constexpr (KM == K_CHANNEL) {
-                const int blk = hdr.t0 / p.R;
-                if (blk != cur_block) {  // fold this block's channel scales into q
-                    cur_block = blk;
-                    load_query(1, sb + p.off_ksz);
+                // Fold the channel scales of the tile's blocks into the
+                // coefficients: the warps share the (block, head) builds into
+                // the sets of this tile's parity (no warp still reads them:
+                // all passed the previous tile's barrier), then wait for all.
+                const int nbt = TILE / p.R;  // block sets per tile
+                float *sets = coefs + (kc_tiles & 1) * nbt * CBUF;
+                const int nb = (hdr.n + p.R - 1) / p.R;
+                for (int idx = warp; idx < nb * GQA; idx += kConsumerWarps) {
+                    const int b = idx / GQA, g = idx - b * GQA;
+                    const float4 xv = ldsf4(qs + g * kHeadDim + 4 * lane);
+                    const float x[4] = {xv.x, xv.y, xv.z, xv.w};
+                    float *set = sets + b * CBUF;
+                    build_head<GQA, KBF, 1, 0>(x, sb + p.off_ksz + b * kHeadDim * 4, set + g * QHSTR,
+                                               set + GQA * QHSTR, g, 128, lane);
                 }
+                named_sync(2, kConsumers);
+                ++kc_tiles;
+                coef = sets + min((warp * TPW) / p.R, nbt - 1) * CBUF;
             }
-            if (hdr.n == kTile)
-                process_tile<GQA, KM, VM, KBITS, VBITS, kTokensPerWarp, GK, GV, VSLOTS, true>(
-                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, geo, Q, qsum, st, wsm,
-                    warp, lane);
+            constexpr int GKC_T = (KM == K_TOKEN) ? GKC : kHeadDim;
+            if (hdr.n == TILE)
+                process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, true>(
+                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, coef, QHSTR, RG::cstr,
+                    coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
             else
-                process_tile<GQA, KM, VM, KBITS, VBITS, kTokensPerWarp, GK, GV, VSLOTS, false>(
-                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, geo, Q, qsum, st, wsm,
-                    warp, lane);
+                process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, false>(
+                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, coef, QHSTR, RG::cstr,
+                    coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
         } else if constexpr (KM != K_BF16) {
             if (!folded) {  // first window tile of the item
-                load_query(2, nullptr);
                 if (VM == V_TOKEN) fold_values();
                 folded = true;
             }
-            process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, GK, GV, VSLOTS, false>(
-                sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, geo, Q, qsum, st, wsm, warp, lane);
+            // bf16 keys against the plain query rows (coefficients = q)
+            process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, kHeadDim, 0, NVG, false>(
+                sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, qs, kHeadDim, 8, nullptr, p.gk, p.gv, st,
+                wsm, warp, lane);
         }
 
         if (hdr.flags & kLast) {
             // ---- item epilogue: merge the four warps, write the partial ----
             if (VM == V_TOKEN && !folded) fold_values();
-            float l_own = st.l_own;
-            l_own += __shfl_xor_sync(0xffffffffu, l_own, 8);
-            l_own += __shfl_xor_sync(0xffffffffu, l_own, 16);
-            const int slice = lane & 15;
+            __syncwarp();
 #pragma unroll
             for (int g = 0; g < GQA; ++g) {
-                const float mg = __shfl_sync(0xffffffffu, st.m_own, g << kOwnShift);
-                const float lg = __shfl_sync(0xffffffffu, l_own, g << kOwnShift);
+                float lg = st.l[g];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float2 v = st.o[g][c];
-                    v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
-                    v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
-                    if (lane < 16) {
-                        red[(warp * GQA + g) * 130 + 8 * slice + 2 * c] = v.x;
-                        red[(warp * GQA + g) * 130 + 8 * slice + 2 * c + 1] = v.y;
-                    }
+                for (int m = 16; m > 0; m >>= 1) lg += __shfl_xor_sync(0xffffffffu, lg, m);
+                float v[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float a = st.o[g][c].x + st.o[g][c].y;
+                    v[c] = a + __shfl_xor_sync(0xffffffffu, a, 16);
                 }
-                if (lane == 0) {
-                    red[(warp * GQA + g) * 130 + 128] = mg;
-                    red[(warp * GQA + g) * 130 + 129] = lg;
+                if (lane < 16) {
+                    float *rp = red + g * RSTR + 8 * slice;
+                    *reinterpret_cast<float4 *>(rp) = make_float4(v[0], v[1], v[2], v[3]);
+                    *reinterpret_cast<float4 *>(rp + 4) = make_float4(v[4], v[5], v[6], v[7]);
                 }
+                if (lane == 0) *reinterpret_cast<float2 *>(red + g * RSTR + 128) = make_float2(st.mref[g], lg);
             }
             named_sync(1, kConsumers);
-            for (int idx = tid; idx < GQA * kHeadDim; idx += kConsumers) {
-                const int g = idx / kHeadDim, d = idx - g * kHeadDim;
+            if (warp < GQA) {  // warp g combines head g, 4 channels per lane
+                const int g = warp;
+                float2 mlw[kConsumerWarps];
                 float M = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[(w * GQA + g) * 130 + 128]);
-                float o = 0.0f, l = 0.0f;
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    mlw[w] = *reinterpret_cast<const float2 *>(scratch_all + w * p.warp_floats + g * RSTR + 128);
+                    M = fmaxf(M, mlw[w].x);
+                }
+                float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                float l = 0.0f;
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = red[(w * GQA + g) * 130 + 128];
-                    const float e = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
-                    o = fmaf(e, red[(w * GQA + g) * 130 + d], o);
-                    l = fmaf(e, red[(w * GQA + g) * 130 + 129], l);
+                    const float e = (mlw[w].x == -INFINITY) ? 0.0f : fast_exp2(mlw[w].x - M);
+                    const float4 ov = ldsf4(scratch_all + w * p.warp_floats + g * RSTR + 4 * lane);
+                    o.x = fmaf(e, ov.x, o.x); o.y = fmaf(e, ov.y, o.y);
+                    o.z = fmaf(e, ov.z, o.z); o.w = fmaf(e, ov.w, o.w);
+                    l = fmaf(e, mlw[w].y, l);
                 }
                 const int hq = hdr.kvh * GQA + g;
                 const int64_t pi = (static_cast<int64_t>(hdr.seq) * p.Hq + hq) * p.n_split + hdr.split;
-                p.o_part[pi * kHeadDim + d] = o;
-                if (d == 0) p.ml[pi] = make_float2(M, l);
+                *reinterpret_cast<float4 *>(p.o_part + pi * kHeadDim + 4 * lane) = o;
+                if (lane == 0) p.ml[pi] = make_float2(M, l);
             }
         }
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -945,7 +1100,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *o_part, 
                                                            int Hq, int n_split, int chunk,
                                                            int max_seq_len) {
     __shared__ float s_max;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait_prior_grid();
     const int hq = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
     const int T = min(__ldg(seq_lens + seq), max_seq_len);
     const int nv = T > 0 ? (T + chunk - 1) / chunk : 0;
@@ -986,18 +1141,19 @@ StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
     StageLayout L{};
     int data;
     if (d.bits_k == 16) {  // every tile is bf16 rows: K at 0, V after it
-        L.bf_tile = kTile;
-        L.bf_off_v = kTile * 256;
+        L.bf_tile = kTileB;
+        L.bf_off_v = kTileB * 256;
         L.off_vc = L.bf_off_v;
-        data = 2 * kTile * 256;
+        data = 2 * kTileB * 256;
     } else {
         const int krow = 128 * d.bits_k / 8;
         const int vrow = 128 * d.bits_v / 8;
-        const int ksz = (d.axis_k == KVQ_PER_CHANNEL) ? 128 * 4 : kTile * (128 / d.group_k) * 4;
-        const int vsz = kTile * (128 / d.group_v) * 4;
-        L.off_ksz = round16(kTile * krow);
+        const int ksz = (d.axis_k == KVQ_PER_CHANNEL) ? (kTileQ / d.residual_len) * 128 * 4
+                                                      : kTileQ * (128 / d.group_k) * 4;
+        const int vsz = kTileQ * (128 / d.group_v) * 4;
+        L.off_ksz = round16(kTileQ * krow);
         L.off_vc = L.off_ksz + round16(ksz);
-        L.off_vsz = L.off_vc + round16(kTile * vrow);
+        L.off_vsz = L.off_vc + round16(kTileQ * vrow);
         data = L.off_vsz + round16(vsz);
         L.bf_tile = kWinTile;
         L.bf_off_v = kWinTile * 256;
@@ -1009,11 +1165,19 @@ StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
     return L;
 }
 
-template <int GQA>
-size_t tail_bytes(int NS, int S, int wsm_floats) {
-    return sizeof(float) * (GQA * kHeadDim + kConsumerWarps * wsm_floats +
-                            kConsumerWarps * GQA * 130 + kConsumerWarps * 8 * 3 * GQA + 2 * GQA + 2) +
-           sizeof(uint64_t) * 2 * NS + 16 + sizeof(int) * (S + 1);
+// Per-warp scratch (floats): the value weights of one tile, which also hold
+// the lanes' W/Z partials when they are summed, then the W/Z totals; the item
+// merge reuses the start of it ([GQA][132]).
+struct ScratchLayout {
+    int off_tot, floats;
+};
+
+ScratchLayout scratch_layout(int gqa, int n_vg) {
+    ScratchLayout S{};
+    S.off_tot = 64 * gqa * n_vg;
+    const int used = S.off_tot + 2 * gqa * n_vg;
+    S.floats = (std::max(used, gqa * 132) + 3) & ~3;
+    return S;
 }
 
 int sm_count() {
@@ -1023,11 +1187,26 @@ int sm_count() {
     return n;
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int GK, int GV>
-kvq_status launch_variant(const DecodeParams &p, int max_items, cudaStream_t stream) {
-    constexpr int NS = (KM == K_BF16) ? 3 : 4;
-    const size_t smem = static_cast<size_t>(NS) * p.stage_bytes + tail_bytes<GQA>(NS, p.S, p.wsm_floats);
-    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, NS, GK, GV>;
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int GKC, int GVC>
+kvq_status launch_variant(DecodeParams p, int max_items, cudaStream_t stream) {
+    constexpr int KBF = (KM == K_BF16) ? 16 : KBITS;
+    constexpr int nch = RowGeo<KBF>::nch;
+    constexpr int cbuf = GQA * nch * RowGeo<KBF>::cstr + kMaxGroups * GQA * 2;
+    const int n_vg = (VM == V_BF16) ? 1 : kHeadDim / p.gv;
+    const ScratchLayout SL = scratch_layout(GQA, n_vg);
+    p.warp_floats = SL.floats;
+    p.off_tot = SL.off_tot;
+    p.n_sets = (KM == K_CHANNEL) ? 2 * (kTileQ / p.R) : 1;
+    const size_t tail = sizeof(float) * (static_cast<size_t>(GQA) * kHeadDim + static_cast<size_t>(p.n_sets) * cbuf +
+                                         kConsumerWarps * static_cast<size_t>(p.warp_floats)) +
+                        sizeof(uint64_t) * 2 * kMaxStages + 16 + sizeof(int) * (2 * p.S + 1);
+    // Ring depth: as many stages (2..4) as let the targeted CTAs per SM fit.
+    const int per_sm_target = decode_min_blocks(KM, VM, GVC);
+    const size_t budget = (232448 - 1024 * per_sm_target) / per_sm_target;
+    int ns = static_cast<int>(std::min<size_t>(kMaxStages, (budget > tail ? budget - tail : 0) / p.stage_bytes));
+    p.ns = std::max(2, ns);
+    const size_t smem = static_cast<size_t>(p.ns) * p.stage_bytes + tail;
+    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, GKC, GVC>;
     if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;  // too many sequences for one launch
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
@@ -1046,13 +1225,14 @@ kvq_status launch_variant(const DecodeParams &p, int max_items, cudaStream_t str
 template <int GQA, int KM, int VM, int KBITS, int VBITS>
 kvq_status launch_groups(const kvq_cache_desc &d, const DecodeParams &p, int max_items,
                          cudaStream_t stream) {
-    if constexpr (GQA == 4 && VM == V_TOKEN) {
-        const int gk = (KM == K_TOKEN) ? d.group_k : 0;
-        if (KM == K_TOKEN && gk == 128 && d.group_v == 128)
+    if constexpr (GQA == 4 && VM == V_TOKEN && KM == K_TOKEN && KBITS == 4 && VBITS == 4) {
+        if (d.group_k == 128 && d.group_v == 128)  // llama-shaped INT4 caches
             return launch_variant<GQA, KM, VM, KBITS, VBITS, 128, 128>(p, max_items, stream);
-        if (KM == K_TOKEN && gk == 32 && d.group_v == 32)
+        if (d.group_k == 32 && d.group_v == 32)
             return launch_variant<GQA, KM, VM, KBITS, VBITS, 32, 32>(p, max_items, stream);
-        if (KM == K_CHANNEL && d.group_v == 32)
+    }
+    if constexpr (GQA == 4 && VM == V_TOKEN && KM == K_CHANNEL && KBITS == 2 && VBITS == 2) {
+        if (d.group_v == 32)  // KIVI-style INT2
             return launch_variant<GQA, KM, VM, KBITS, VBITS, 0, 32>(p, max_items, stream);
     }
     return launch_variant<GQA, KM, VM, KBITS, VBITS, 0, 0>(p, max_items, stream);
@@ -1077,23 +1257,17 @@ kvq_status dispatch_modes(const kvq_cache_desc &d, const DecodeParams &p, int ma
     return KVQ_ERR_UNSUPPORTED;
 }
 
-int log2i(int x) {
-    int r = 0;
-    while ((1 << r) < x) ++r;
-    return r;
-}
-
 }  // namespace
 
 bool plan_decode(const kvq_cache_desc &d, int num_seqs, int num_q_heads, int max_seq_len,
                  DecodePlan *plan) {
     if (num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0 || d.num_kv_heads <= 0) return false;
-    // About six items per resident CTA (2 per SM) when every sequence is at
-    // max_seq_len; chunks of 256..4096 tokens, a multiple of the tile.
+    // About eight items per resident CTA (2 per SM) when every sequence is at
+    // max_seq_len; chunks of 256..4096 tokens, a multiple of the tiles.
     const int64_t units = static_cast<int64_t>(num_seqs) * d.num_kv_heads;
-    const int64_t target_items = 6 * 2 * 148;
+    const int64_t target_items = 8 * 2 * 148;
     int64_t chunk = (units * std::max(1, max_seq_len) + target_items - 1) / target_items;
-    chunk = ((chunk + kTile - 1) / kTile) * kTile;
+    chunk = ((chunk + kTileQ - 1) / kTileQ) * kTileQ;
     chunk = std::min<int64_t>(std::max<int64_t>(chunk, 256), 4096);
     plan->chunk = static_cast<int>(chunk);
     plan->n_split = static_cast<int>(std::max<int64_t>(1, (max_seq_len + chunk - 1) / chunk));
@@ -1126,8 +1300,8 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.S = num_seqs;
     p.H = d.num_kv_heads;
     p.Hq = num_q_heads;
-    p.gk_log2 = log2i(std::max(1, d.group_k));
-    p.gv_log2 = log2i(std::max(1, d.group_v));
+    p.gk = (d.bits_k == 16 || d.axis_k == KVQ_PER_CHANNEL) ? kHeadDim : d.group_k;
+    p.gv = (d.bits_v == 16) ? kHeadDim : d.group_v;
     p.hb = d.hadamard_block_k;
     p.hscale = hadamard_scale(d.hadamard_block_k);
     p.qscale = softmax_scale * kLog2e;
@@ -1152,9 +1326,6 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.off_hdr = L.off_hdr;
     p.bf_tile = L.bf_tile;
     p.bf_off_v = L.bf_off_v;
-    // value groups per token: 1 for bf16 values (and for the bf16 window tiles)
-    const int n_vg = (d.bits_v == 16) ? 1 : kHeadDim / d.group_v;
-    p.wsm_floats = kTokensPerWarp * n_vg * gqa * 2;
     p.timeout_ns = debug_hooks().wait_timeout_ns;
     p.skip_tile = debug_hooks().skip_tile;
     const int64_t max_items64 = static_cast<int64_t>(num_seqs) * d.num_kv_heads * plan.n_split;
