@@ -45,6 +45,15 @@ BATCH, HQ, HKV, D, CTX, EPISODE = 16, 32, 8, 128, 8192, 64
 BYTES_PER_TOKEN_HEAD = 2 * (D * 4 // 8 + (D // 128) * 4)   # K + V: 64 B codes + 4 B scale/zero
 NOMINAL_HBM_GBS = 8000.0
 FLUSH_BYTES = 256 << 20
+
+
+def flush_l2(buf):
+    """Evict L2 between timed steps: write a buffer twice the size of L2, then
+    read it back, so the timed work starts from a cold L2 that holds no dirty
+    lines (a write alone would leave ~126 MB of them, whose write-back the next
+    kernel's reads would pay for)."""
+    buf.zero_()
+    buf.amax()
 DECODE_SRC = os.path.join(ROOT, "bit_kv_cache_21_b200", "csrc", "kvq_decode.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_splitk_llama8b_traffic.json")
 
@@ -237,7 +246,7 @@ def run_ours(args, rank, world, local_rank):
         return CTX + j + 1   # tokens attended per sequence
 
     for i in range(args.warmup):
-        flush.zero_()
+        flush_l2(flush)
         step(i)
     torch.cuda.synchronize()
     # start the timed episodes at a step boundary of the episode
@@ -248,7 +257,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     with ClockSampler(dev) as clocks:
         for i in range(args.steps):
-            flush.zero_()
+            flush_l2(flush)
             tokens.append(step(i, evs[i]))
         torch.cuda.synchronize()
     if world > 1:
@@ -263,7 +272,7 @@ def run_ours(args, rank, world, local_rank):
     split_bytes = float(lens_now.sum().item()) * HKV * BYTES_PER_TOKEN_HEAD
     split_ms = []
     for i in range(args.warmup + args.steps):
-        flush.zero_()
+        flush_l2(flush)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         K.decode_splitk(cache.desc, q_steps[0], lens_now, cap, scale, ws)
@@ -290,7 +299,7 @@ def run_ours(args, rank, world, local_rank):
         j = i % EPISODE
         if j == 0:
             lens.copy_(ctx_lens)
-        flush.zero_()
+        flush_l2(flush)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         dk.copy_(hk[j], non_blocking=True)
@@ -365,12 +374,12 @@ def run_remat(args, dev):
             evs[2].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2(flush)
         step()
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.remat_steps)]
     for i in range(args.remat_steps):
-        flush.zero_()
+        flush_l2(flush)
         step(evs[i])
     torch.cuda.synchronize()
     assert cache.device_status() == 0 and int(status[0]) == 0
@@ -412,7 +421,7 @@ def _time_steps(torch, stream, flush, n_warm, n_steps, step):
     attention of the last n_steps with events. step(i, evs) records evs[0..2]."""
     evs = []
     for i in range(n_warm + n_steps):
-        flush.zero_()
+        flush_l2(flush)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         step(i, e)
         if i >= n_warm:
@@ -694,7 +703,7 @@ def main():
             "dtype": "int4 packed K/V, fp32 math", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": BATCH * world, "seq_len": CTX,
                        "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "flushed between steps (256 MiB write)",
+                       "l2": "flushed between steps (256 MiB write, then read back: cold, clean L2)",
                        "pct_of_8TBs": 100.0 * value / NOMINAL_HBM_GBS},
             "roofline": {"kernel": "decode_splitk_kernel", "bound": "hbm", "achieved": achieved,
                          "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",

@@ -46,6 +46,7 @@
 // The four warps' states are merged once per item; the merge kernel combines
 // the splits.
 #include <algorithm>
+#include <mutex>
 
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
@@ -58,6 +59,7 @@ constexpr int kTileQ = 256;        // tokens per quantized tile (64 per warp, 2 
 constexpr int kTileB = 128;        // tokens per tile of a bf16 cache (32 per warp)
 constexpr int kWinTile = 16;       // tokens per bf16 window tile (quantized caches)
 constexpr int kMaxStages = 4;      // shared-memory ring depth, chosen on the host
+constexpr int kMaxDevices = 64;    // launch settings cached per device
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
@@ -1208,13 +1210,32 @@ kvq_status launch_variant(DecodeParams p, int max_items, cudaStream_t stream) {
     const size_t smem = static_cast<size_t>(p.ns) * p.stage_bytes + tail;
     auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, GKC, GVC>;
     if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;  // too many sequences for one launch
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return KVQ_ERR_CUDA;
+    // The shared-memory opt-in and the occupancy query cost host time on every
+    // call; redo them only when this variant's size changes (per device).
+    struct Cached {
+        size_t smem;
+        int per_sm;
+    };
+    static Cached cache[kMaxDevices];
+    static std::mutex lock;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess ||
-        per_sm <= 0)
-        per_sm = 1;
+    {
+        std::lock_guard<std::mutex> guard(lock);
+        if (cache[dev].per_sm > 0 && cache[dev].smem >= smem && cache[dev].smem - smem < 4096) {
+            per_sm = cache[dev].per_sm;
+        } else {
+            const size_t opt_in = std::max(smem, cache[dev].smem);
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(opt_in)) != cudaSuccess)
+                return KVQ_ERR_CUDA;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess ||
+                per_sm <= 0)
+                per_sm = 1;
+            cache[dev] = Cached{opt_in, per_sm};
+        }
+    }
     const int grid = std::max(1, std::min(max_items, per_sm * sm_count()));
     if (cudaMemsetAsync(p.counter, 0, sizeof(int), stream) != cudaSuccess) return KVQ_ERR_CUDA;
     kern<<<grid, kThreads, smem, stream>>>(p);
