@@ -487,23 +487,42 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
                     float2 f[TPL][4];
 #pragma unroll
                     for (int m = 0; m < TPL; ++m) word_pairs4<KB>(wv[m][wi], jb, f[m]);
-                    float4 cv[GQA][2];
+                    if constexpr (NVG == 1) {
+                        // every head's coefficients first, then the multiply-adds
+                        // interleaved across tokens and heads
+                        float4 cv[GQA][2];
 #pragma unroll
-                    for (int g = 0; g < GQA; ++g) {
-                        const float *cw = cc + g * hstr + wi * RG::cpw + 2 * jb;
-                        cv[g][0] = ldsf4(cw);
-                        cv[g][1] = ldsf4(cw + 4);
-                    }
+                        for (int g = 0; g < GQA; ++g) {
+                            const float *cw = cc + g * hstr + wi * RG::cpw + 2 * jb;
+                            cv[g][0] = ldsf4(cw);
+                            cv[g][1] = ldsf4(cw + 4);
+                        }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
+                        for (int j = 0; j < 4; ++j)
 #pragma unroll
-                        for (int m = 0; m < TPL; ++m)
+                            for (int m = 0; m < TPL; ++m)
 #pragma unroll
-                            for (int g = 0; g < GQA; ++g) {
-                                const float4 v = cv[g][j >> 1];
-                                ffma2(acc[m][g], (j & 1) ? make_float2(v.z, v.w) : make_float2(v.x, v.y),
-                                      f[m][j]);
+                                for (int g = 0; g < GQA; ++g) {
+                                    const float4 v = cv[g][j >> 1];
+                                    ffma2(acc[m][g], (j & 1) ? make_float2(v.z, v.w) : make_float2(v.x, v.y),
+                                          f[m][j]);
+                                }
+                    } else {
+                        // head by head (fewer live registers next to the
+                        // per-group value sums)
+#pragma unroll
+                        for (int g = 0; g < GQA; ++g) {
+                            const float *cw = cc + g * hstr + wi * RG::cpw + 2 * jb;
+                            const float4 c0 = ldsf4(cw), c1 = ldsf4(cw + 4);
+#pragma unroll
+                            for (int m = 0; m < TPL; ++m) {
+                                ffma2(acc[m][g], make_float2(c0.x, c0.y), f[m][0]);
+                                ffma2(acc[m][g], make_float2(c0.z, c0.w), f[m][1]);
+                                ffma2(acc[m][g], make_float2(c1.x, c1.y), f[m][2]);
+                                ffma2(acc[m][g], make_float2(c1.z, c1.w), f[m][3]);
                             }
+                        }
+                    }
                 }
                 if (cpg == 0 && ((wi + 1) & (wpg - 1)) == 0) end_group((c * 4 + wi) / wpg);
             }
@@ -557,6 +576,8 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     // Value weights w = p * s per (token, value group), at their pair slot.
     const int n_vg = (VMT == V_BF16) ? 1 : (GVC ? kHeadDim / GVC : kHeadDim / gv_rt);
     float2 *wsm2 = reinterpret_cast<float2 *>(wsm);
+    // pair rows padded by 16 bytes so the lanes' rows start in different bank groups
+    const int pstr = n_vg * GQA + 2;
 #pragma unroll
     for (int v = 0; v < ((VMT == V_BF16) ? 1 : NVG); ++v) {
         if (v < n_vg) {
@@ -580,11 +601,11 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
             }
             if constexpr (TPL == 2) {  // lane j owns pair j: both halves
 #pragma unroll
-                for (int g = 0; g < GQA; ++g) wsm2[(lane * n_vg + v) * GQA + g] = make_float2(w[0][g], w[1][g]);
+                for (int g = 0; g < GQA; ++g) wsm2[lane * pstr + v * GQA + g] = make_float2(w[0][g], w[1][g]);
             } else if (lane < TPW) {
                 const int slot = lane % HALF, half = lane / HALF;
 #pragma unroll
-                for (int g = 0; g < GQA; ++g) wsm[((slot * n_vg + v) * GQA + g) * 2 + half] = w[0][g];
+                for (int g = 0; g < GQA; ++g) wsm[(slot * pstr + v * GQA + g) * 2 + half] = w[0][g];
             }
         }
     }
@@ -607,7 +628,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
                 f[c].y = vb ? f[c].y : 0.0f;
             }
         }
-        const float2 *wrow = wsm2 + (pi * n_vg + gv_lane) * GQA;
+        const float2 *wrow = wsm2 + pi * pstr + gv_lane * GQA;
         float2 w[GQA];
         if constexpr (GQA >= 2) {
 #pragma unroll
@@ -1176,7 +1197,7 @@ struct ScratchLayout {
 
 ScratchLayout scratch_layout(int gqa, int n_vg) {
     ScratchLayout S{};
-    S.off_tot = 64 * gqa * n_vg;
+    S.off_tot = 64 * gqa * n_vg + 128;  // 32 pair rows of (n_vg * gqa + 2) f32x2
     const int used = S.off_tot + 2 * gqa * n_vg;
     S.floats = (std::max(used, gqa * 132) + 3) & ~3;
     return S;
