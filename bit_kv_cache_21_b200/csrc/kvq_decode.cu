@@ -912,21 +912,22 @@ decode_splitk_kernel(const DecodeParams p) {
     auto fold_values = [&]() {
         const int n_vg = GVC ? kHeadDim / GVC : kHeadDim / p.gv;
         const int nv = 2 * GQA * n_vg;  // values per lane: W then Z, [g][v]
+        const int rs = nv + 1;          // odd row stride: the lanes' rows hit distinct banks
 #pragma unroll
         for (int g = 0; g < GQA; ++g)
 #pragma unroll
             for (int v = 0; v < NVG; ++v)
                 if (v < n_vg) {
-                    wsm[lane * nv + g * n_vg + v] = st.W[g][v];
-                    wsm[lane * nv + GQA * n_vg + g * n_vg + v] = st.Z[g][v];
+                    wsm[lane * rs + g * n_vg + v] = st.W[g][v];
+                    wsm[lane * rs + GQA * n_vg + g * n_vg + v] = st.Z[g][v];
                 }
         __syncwarp();
         for (int col = lane; col < nv; col += 32) {
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
             for (int r = 0; r < 32; r += 2) {
-                a0 += wsm[r * nv + col];
-                a1 += wsm[(r + 1) * nv + col];
+                a0 += wsm[r * rs + col];
+                a1 += wsm[(r + 1) * rs + col];
             }
             totals[col] = a0 + a1;
         }
