@@ -483,6 +483,73 @@ def run_long_int2(args, dev):
             "step_GBps": mb / ((statistics.mean(app) + statistics.mean(att)) * 1e-3) / 1e9}
 
 
+def run_rotation_sweep(args, dev):
+    """Accuracy and cost of the key rotation: no rotation, block-diagonal
+    Hadamard with blocks of 32, 64 and 128 channels, each with and without
+    QuaRot's random signs. 16 seqs x 8 KV heads (32 q heads) x 4096 tokens of
+    the outlier-key recipe, INT4 g128 K and V. The error is that of decode
+    attention over the quantized cache against attention over the same tokens
+    kept in bf16 (the library's bits-16 mode); an orthogonal rotation does not
+    change the latter."""
+    import torch
+    import bit_kv_cache_21_b200 as K
+    import workloads as W
+    S, H, HQ_, T = 16, 8, 32, 4096
+    n_rep = 5
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6)
+    k, v = _synthetic_kv(gen, S * T, H, dev, torch, 6)               # [S*T][H][D]
+    q = torch.randn((S, HQ_, D), generator=gen, device=dev).to(torch.bfloat16)
+    kb = k.view(S, T, H, D).permute(0, 2, 1, 3).contiguous()          # [S][H][T][D]
+    vb = v.view(S, T, H, D).permute(0, 2, 1, 3).contiguous()
+    lens_full = torch.full((S,), T, dtype=torch.int32, device=dev)
+    cu = torch.arange(0, (S + 1) * T, T, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ref = K.decode_attention(K.bf16_cache_desc(kb, vb), q, lens_full, T, scale).double()
+    signs = torch.from_numpy(W.hadamard_signs(6)).to(dev)
+    rows = []
+    for hb in (0, 32, 64, 128):
+        for use_signs in ((False, True) if hb else (False,)):
+            spec = K.CacheSpec(S, H, bits_k=4, bits_v=4, group_k=128, group_v=128, hadamard_block_k=hb,
+                               capacity_tokens=T, hadamard_signs=signs if use_signs else None)
+            cache = K.KVCache(spec, device=dev)
+            ws = torch.empty(K.decode_workspace_size(cache.desc, S, HQ_, T), dtype=torch.uint8, device=dev)
+            out = torch.empty((S, HQ_, D), dtype=torch.float32, device=dev)
+            app_ms, att_ms = [], []
+            for rep in range(n_rep + 1):
+                lens = torch.zeros(S, dtype=torch.int32, device=dev)
+                flush_l2(flush)
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record(stream)
+                K.quantize_append(cache.desc, k, v, cu, lens)
+                e[1].record(stream)
+                flush_l2(flush)
+                e[2].record(stream)
+                K.decode_attention(cache.desc, q, lens_full, T, scale, out=out, workspace=ws)
+                e3 = torch.cuda.Event(enable_timing=True)
+                e3.record(stream)
+                torch.cuda.synchronize()
+                if rep > 0:  # the first repetition warms up
+                    app_ms.append(e[0].elapsed_time(e[1]))
+                    att_ms.append(e[2].elapsed_time(e3))
+            assert cache.device_status() == 0
+            d = out.double() - ref
+            rows.append({"hadamard_block": hb, "random_signs": use_signs,
+                         "attn_rel_l2": float(d.norm() / ref.norm()),
+                         "attn_max_abs": float(d.abs().max()),
+                         "append_ms": statistics.mean(app_ms),
+                         "append_tokens_per_s": S * T / (statistics.mean(app_ms) * 1e-3),
+                         "decode_ms": statistics.mean(att_ms),
+                         "decode_GBps": S * H * T * BYTES_PER_TOKEN_HEAD / (statistics.mean(att_ms) * 1e-3) / 1e9})
+            del cache, ws
+    return {"workload": "rotation sweep: 16 seqs x 8 kv / 32 q heads x 4096 tokens, bf16 K with 4 "
+                        "outlier channels x20, INT4 g128 K and V; error of decode attention against "
+                        "attention over the same tokens in bf16",
+            "rows": rows}
+
+
 def run_paged_mix(args, dev):
     """64 sequences, lognormal lengths (median 4096, sigma 1, clipped to
     [1024, 32768]), 16-token pages, INT4 g128, Hadamard keys. A step appends a
@@ -599,9 +666,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--part", default="all",
-                    choices=["all", "decode", "remat", "long_int2", "paged_mix"],
-                    help="run one leg alone: decode (the metric's step), remat, long_int2 or "
-                         "paged_mix (the last three print their own line)")
+                    choices=["all", "decode", "remat", "long_int2", "paged_mix", "rotation_sweep"],
+                    help="run one leg alone: decode (the metric's step), remat, long_int2, "
+                         "paged_mix or rotation_sweep (the last four print their own line)")
     ap.add_argument("--remat-batch", type=int, default=8)
     ap.add_argument("--remat-steps", type=int, default=10)
     args = ap.parse_args()
@@ -661,6 +728,18 @@ def main():
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
         return
+    if args.part == "rotation_sweep":
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        sw = run_rotation_sweep(args, dev)
+        if rank == 0:
+            print(json.dumps({"metric": "decode-attn error vs bf16 and cost per key rotation",
+                              "n_gpus": world, "data": "synthetic",
+                              "config": {"workload": sw["workload"]}, "rotation_sweep": sw}))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.part == "remat":
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
@@ -678,6 +757,7 @@ def main():
     rr = run_remat(args, torch.device("cuda", local_rank)) if args.part == "all" else None
     li = run_long_int2(args, torch.device("cuda", local_rank)) if args.part == "all" else None
     pm = run_paged_mix(args, torch.device("cuda", local_rank)) if args.part == "all" else None
+    sw = run_rotation_sweep(args, torch.device("cuda", local_rank)) if args.part == "all" else None
 
     # max over ranks of the device time; bytes summed over ranks
     total_ms, total_bytes, e2e_s, e2e_bytes = res["total_ms"], res["bytes"], res["e2e_s"], res["e2e_bytes"]
@@ -727,6 +807,8 @@ def main():
             line["long_int2"] = li
         if pm is not None:
             line["paged_mix"] = pm
+        if sw is not None:
+            line["rotation_sweep"] = sw
         print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()

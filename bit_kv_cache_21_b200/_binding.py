@@ -60,6 +60,7 @@ class CacheDesc(ctypes.Structure):
         ("v_res", ctypes.c_void_p),
         ("block_table", ctypes.c_void_p),
         ("status", ctypes.c_void_p),
+        ("hadamard_signs", ctypes.c_void_p),
     ]
 
 

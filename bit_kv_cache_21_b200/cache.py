@@ -29,6 +29,7 @@ class CacheSpec:
     max_pages_per_seq: int = 0
     num_pages: int = 0
     with_v: bool = True
+    hadamard_signs: object = None  # device float32 [128] of +-1 (randomized Hadamard), or None
 
 
 def _row_bytes(bits: int) -> int:
@@ -85,7 +86,7 @@ class KVCache:
             capacity_tokens=s.capacity_tokens, reserved=0,
             k_codes=p(self.k_codes), v_codes=p(self.v_codes), k_sz=p(self.k_sz), v_sz=p(self.v_sz),
             k_res=p(self.k_res), v_res=p(self.v_res), block_table=p(self.block_table),
-            status=p(self.status))
+            status=p(self.status), hadamard_signs=p(s.hadamard_signs))
 
     def device_status(self) -> int:
         return int(self.status[0].item())

@@ -67,6 +67,8 @@ kvq_status validate_desc(const kvq_cache_desc *d, bool need_v) {
         if (!bf16_v && (d->v_sz == nullptr || !aligned16(d->v_sz))) return KVQ_ERR_INVALID_ARG;
     }
     if (d->status != nullptr && (reinterpret_cast<uintptr_t>(d->status) & 3u)) return KVQ_ERR_INVALID_ARG;
+    if (d->hadamard_signs != nullptr && (d->hadamard_block_k == 0 || !aligned16(d->hadamard_signs)))
+        return KVQ_ERR_INVALID_ARG;
     return KVQ_OK;
 }
 

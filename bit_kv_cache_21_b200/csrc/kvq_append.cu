@@ -33,6 +33,7 @@ struct AppendTensor {
     int group;         // 16, 32, 64 or 128
     int hb;            // rotation block, 0 = none
     float hscale;      // fp32(1/sqrt(hb))
+    const float *signs;  // [128] +-1 applied before the rotation, or null
 };
 
 struct AppendParams {
@@ -327,6 +328,14 @@ __global__ void __launch_bounds__(256) append_tokens_kernel(const AppendParams p
 
     float x[32];
     load32<DT>(T.src, v, part, x);
+    if (T.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
+        const float4 *sg = reinterpret_cast<const float4 *>(T.signs + part * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 f = __ldg(sg + i);
+            x[4 * i] *= f.x; x[4 * i + 1] *= f.y; x[4 * i + 2] *= f.z; x[4 * i + 3] *= f.w;
+        }
+    }
     if (T.hb > 0) fwht_lane(x, T.hb, part, T.hscale);
 
     uint32_t words[4];
@@ -539,9 +548,10 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
     } else {
         AppendParams p{};
         p.t[0] = {static_cast<uint8_t *>(d.k_codes), static_cast<__half2 *>(d.k_sz), k_new,
-                  d.bits_k, d.group_k, d.hadamard_block_k, hadamard_scale(d.hadamard_block_k)};
+                  d.bits_k, d.group_k, d.hadamard_block_k, hadamard_scale(d.hadamard_block_k),
+                  d.hadamard_block_k > 0 ? d.hadamard_signs : nullptr};
         p.t[1] = {static_cast<uint8_t *>(d.v_codes), static_cast<__half2 *>(d.v_sz), v_new,
-                  d.bits_v, d.group_v, 0, 0.0f};
+                  d.bits_v, d.group_v, 0, 0.0f, nullptr};
         p.H = d.num_kv_heads;
         p.cu_new = cu_new; p.seq_lens = seq_lens;
         p.num_seqs = num_seqs; p.total_tokens = total_new;

@@ -84,6 +84,7 @@ struct DecodeParams {
     const int32_t *block_table;
     const int32_t *seq_lens;
     const void *q;
+    const float *signs;  // [128] +-1 applied to the query before its rotation, or null
     float *o_part;  // [S][Hq][n_split][D]
     float2 *ml;     // [S][Hq][n_split]
     int *counter;   // item counter, zeroed before the launch
@@ -984,6 +985,10 @@ decode_splitk_kernel(const DecodeParams p) {
                         }
                     }
                 }
+                if (p.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
+                    const float4 sg = __ldg(reinterpret_cast<const float4 *>(p.signs) + lane);
+                    x[0] *= sg.x; x[1] *= sg.y; x[2] *= sg.z; x[3] *= sg.w;
+                }
                 if (p.hb > 0) {
                     if (p.hb > 1) { float a = x[0], b = x[1]; x[0] = a + b; x[1] = a - b;
                                     a = x[2]; b = x[3]; x[2] = a + b; x[3] = a - b; }
@@ -1336,6 +1341,7 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.block_table = d.block_table;
     p.seq_lens = seq_lens;
     p.q = q;
+    p.signs = d.hadamard_block_k > 0 ? d.hadamard_signs : nullptr;
     p.o_part = static_cast<float *>(workspace);
     p.ml = reinterpret_cast<float2 *>(static_cast<uint8_t *>(workspace) + plan.ws_part);
     p.counter = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + plan.ws_part + plan.ws_ml);

@@ -132,6 +132,15 @@ typedef struct {
     void *k_res, *v_res;       /* device, bf16 windows (residual_len > 0) */
     const int32_t *block_table;/* device [S][max_pages_per_seq] (paged) */
     int32_t *status;           /* device status word, may be NULL */
+    const float *hadamard_signs;/* device [128] entries +1.0f / -1.0f, or NULL.
+                                  With hadamard_block_k > 0 the keys (and the
+                                  queries) take x -> H_blk diag(signs) x / sqrt(blk):
+                                  the randomized Hadamard of "QuaRot: Outlier-Free
+                                  4-Bit Inference in Rotated LLMs" (listed among the
+                                  works the pages build on). Multiplying by +-1 is
+                                  exact, and (H D)^T (H D) = blk I, so q.k is kept.
+                                  Other values give a transform that is not
+                                  orthogonal. Requires hadamard_block_k > 0. */
 } kvq_cache_desc;
 
 /*

@@ -176,15 +176,27 @@ def unpack_codes(packed, n, bits):
     return out
 
 
-def quantize_tokens(x, hb, G, bits):
+def apply_signs(x, signs):
+    """diag(signs) x along the last axis: the random sign flip that QuaRot
+    puts before the Hadamard ("QuaRot: Outlier-Free 4-Bit Inference in Rotated
+    LLMs", randomized Hadamard). With signs of +-1 the product is exact in any
+    precision. Returns x itself when signs is None."""
+    if signs is None:
+        return x
+    x = np.asarray(x)
+    return x * np.asarray(signs, x.dtype)
+
+
+def quantize_tokens(x, hb, G, bits, signs=None):
     """Token-wise group quantization (SAW-INT4 Abstract "token-wise INT4";
     InnerQ Abstract groups along the inner dimension of q.k).
 
-    x: float32 [..., D] (bf16 or fp32 values). Each vector is rotated (hb > 0)
-    and split into D/G groups of G consecutive elements.
+    x: float32 [..., D] (bf16 or fp32 values). Each vector is multiplied by
+    the random signs (if given), rotated (hb > 0) and split into D/G groups of
+    G consecutive elements.
     Returns codes uint8 [..., D*bits/8] and sz uint16 [..., D/G, 2] holding
     the fp16 bit patterns (scale, zero)."""
-    a = _c(x, np.float32)
+    a = _c(apply_signs(_c(x, np.float32), signs), np.float32)
     D = a.shape[-1]
     n = a.size // D
     codes = np.zeros(a.shape[:-1] + (D * bits // 8,), np.uint8)
@@ -243,15 +255,15 @@ def attention(q, k, v, scale):
     return out
 
 
-def decode_attention_gqa(q, khat, vhat, scale, rotate_q_block=0):
+def decode_attention_gqa(q, khat, vhat, scale, rotate_q_block=0, signs=None):
     """Decode attention of one sequence with grouped-query heads.
 
     q: [H_q][D] (bf16/fp32 values); khat, vhat: [H_kv][T][D] float64, the
     dequantized cache as attended. Query head h reads KV head
     h // (H_q // H_kv). When the cache keys were rotated with block size
     rotate_q_block, the query is rotated by the same transform first (Dual-QK
-    Abstract), in float64."""
-    q = np.asarray(q, np.float64)
+    Abstract), in float64, random signs included."""
+    q = apply_signs(np.asarray(q, np.float64), signs)
     H_q, D = q.shape
     H_kv = khat.shape[0]
     g = H_q // H_kv

@@ -80,27 +80,28 @@ def gather_tokens(cache: K.KVCache, which: str, seq: int, head: int, T: int):
     return c.cpu().numpy(), z.cpu().numpy().view(np.uint16)
 
 
-def expected_tokens(x_hist: np.ndarray, head: int, hb: int, G: int, bits: int):
+def expected_tokens(x_hist: np.ndarray, head: int, hb: int, G: int, bits: int, signs=None):
     """Oracle codes and scale/zero for one head of a [T][H][D] history."""
-    return oracle.quantize_tokens(np.ascontiguousarray(x_hist[:, head, :]), hb, G, bits)
+    return oracle.quantize_tokens(np.ascontiguousarray(x_hist[:, head, :]), hb, G, bits, signs=signs)
 
 
-def oracle_decode_tokens(k_hist, v_hist, q, spec: K.CacheSpec, scale=SCALE):
+def oracle_decode_tokens(k_hist, v_hist, q, spec: K.CacheSpec, scale=SCALE, signs=None):
     """Expected decode output of one sequence from its K/V history
     [T][H][D] and query [Hq][D]: the oracle quantizes, dequantizes and
-    attends in float64."""
+    attends in float64. `signs`: the randomized Hadamard's signs (numpy)."""
     H = k_hist.shape[1]
     T = k_hist.shape[0]
     kh = np.zeros((H, T, D))
     vh = np.zeros((H, T, D))
     for h in range(H):
         kc, ksz = oracle.quantize_tokens(np.ascontiguousarray(k_hist[:, h]), spec.hadamard_block_k,
-                                         spec.group_k, spec.bits_k)
+                                         spec.group_k, spec.bits_k, signs=signs)
         vc, vsz = oracle.quantize_tokens(np.ascontiguousarray(v_hist[:, h]), 0, spec.group_v,
                                          spec.bits_v)
         kh[h] = oracle.dequant_tokens(kc, ksz, spec.group_k, spec.bits_k)
         vh[h] = oracle.dequant_tokens(vc, vsz, spec.group_v, spec.bits_v)
-    return oracle.decode_attention_gqa(q, kh, vh, scale, rotate_q_block=spec.hadamard_block_k)
+    return oracle.decode_attention_gqa(q, kh, vh, scale, rotate_q_block=spec.hadamard_block_k,
+                                       signs=signs)
 
 
 def oracle_decode_kivi(k_hist, v_hist, q, spec: K.CacheSpec, scale=SCALE):

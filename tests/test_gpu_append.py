@@ -19,16 +19,16 @@ def _history(seed, lens, H, dtype, outliers=True):
     return ks, vs
 
 
-def _check_all(cache, ks, vs, lens, heads=None):
+def _check_all(cache, ks, vs, lens, heads=None, signs=None):
     s = cache.spec
     for q, T in enumerate(lens):
         for h in (heads if heads is not None else range(s.num_kv_heads)):
-            todo = [("k", ks[q], s.hadamard_block_k, s.group_k, s.bits_k)]
+            todo = [("k", ks[q], s.hadamard_block_k, s.group_k, s.bits_k, signs)]
             if s.with_v:
-                todo.append(("v", vs[q], 0, s.group_v, s.bits_v))
-            for which, hist, hb, G, bits in todo:
+                todo.append(("v", vs[q], 0, s.group_v, s.bits_v, None))
+            for which, hist, hb, G, bits, sg in todo:
                 c, z = gather_tokens(cache, which, q, h, T)
-                ec, ez = expected_tokens(hist, h, hb, G, bits)
+                ec, ez = expected_tokens(hist, h, hb, G, bits, signs=sg)
                 assert np.array_equal(c, ec), (which, q, h)
                 assert np.array_equal(z, ez), (which, q, h)
 
@@ -183,3 +183,29 @@ def test_llama8b_prefill_full_size_sampled():
                 c, z = gather_tokens(cache, which, q, h, w.context)
                 ec, ez = expected_tokens(hist, h, hb, 128, 4)
                 assert np.array_equal(c, ec) and np.array_equal(z, ez)
+
+
+@pytest.mark.parametrize("bits,G,hb,paged", [(4, 128, 128, False), (2, 32, 64, False), (4, 64, 32, True)])
+def test_append_randomized_hadamard(bits, G, hb, paged):
+    # QuaRot's randomized Hadamard: keys take H diag(signs) / sqrt(hb); codes
+    # and scale/zero stay bit-exact with the oracle.
+    lens = [150, 33, 1, 64]
+    H = 2
+    ks, vs = _history(700 + bits + G + hb, lens, H, "bf16")
+    signs = W.hadamard_signs(17)
+    sg = torch.from_numpy(signs).cuda()
+    if paged:
+        spec = K.CacheSpec(len(lens), H, bits_k=bits, bits_v=bits, group_k=G, group_v=G,
+                           hadamard_block_k=hb, paged=True, page_size=16, max_pages_per_seq=16,
+                           num_pages=64, hadamard_signs=sg)
+        cache = K.KVCache(spec)
+        assign_pages(cache, lens)
+    else:
+        spec = K.CacheSpec(len(lens), H, bits_k=bits, bits_v=bits, group_k=G, group_v=G,
+                           hadamard_block_k=hb, capacity_tokens=192, hadamard_signs=sg)
+        cache = K.KVCache(spec)
+    sl = lens_tensor([0] * len(lens))
+    append(cache, ks, vs, sl)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    _check_all(cache, ks, vs, lens, signs=signs)

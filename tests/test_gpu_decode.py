@@ -182,3 +182,27 @@ def test_paged_mix_full_size_sampled():
     for s in sorted({0, 8, 63, longest}):
         assert_close(out[s], oracle_decode_tokens(ks[s], vs[s], q[s], spec), "seq %d" % s)
     assert math.isfinite(float(out.sum()))
+
+
+@pytest.mark.parametrize("hb,gqa", [(128, 4), (64, 2)])
+def test_decode_randomized_hadamard(hb, gqa):
+    # Keys and queries both take H diag(signs) / sqrt(hb), so the scores are
+    # those of the unrotated vectors; the output matches the oracle's float64
+    # attention over its own dequantized cache.
+    lens = [257, 70, 1]
+    H = 2
+    Hq = H * gqa
+    ks, vs = _hist(900 + hb, lens, H, "bf16")
+    signs = W.hadamard_signs(23)
+    spec = K.CacheSpec(len(lens), H, bits_k=4, bits_v=4, group_k=128, group_v=128,
+                       hadamard_block_k=hb, capacity_tokens=384,
+                       hadamard_signs=torch.from_numpy(signs).cuda())
+    cache = K.KVCache(spec)
+    sl = lens_tensor([0] * len(lens))
+    append(cache, ks, vs, sl)
+    q = _queries(31, len(lens), Hq, "bf16")
+    out = K.decode_attention(cache.desc, dev(q, "bf16"), sl, 384, SCALE).cpu().numpy()
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    for s_, T in enumerate(lens):
+        assert_close(out[s_], oracle_decode_tokens(ks[s_], vs[s_], q[s_], spec, signs=signs), "seq %d" % s_)

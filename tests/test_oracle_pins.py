@@ -410,3 +410,49 @@ def test_quantizer_permutation_invariance_with_signed_zeros():
         s2, z2, q2 = oracle.quantize_group(x[perm], 4)
         assert (s1, z1) == (s2, z2)
         assert np.array_equal(q1[perm], q2)
+
+
+# ---------------------------------------------------------------------------
+# Randomized Hadamard (QuaRot): signs first, then the block transform
+# ---------------------------------------------------------------------------
+
+RH_D = 128  # head dimension
+
+def test_randomized_hadamard_golden_worked_example():
+    with open(os.path.join(GOLDEN, "randomized_hadamard_h4.txt")) as f:
+        lines = [l for l in f if l.strip() and not l.startswith("#")]
+    assert len(lines) == 2
+    for line in lines:
+        s, x, y = (np.array([float(t) for t in part.split()]) for part in line.split(";"))
+        got = oracle.rotate_f64(oracle.apply_signs(x, s), 4)
+        assert np.array_equal(got, y), (got, y)
+        got32 = oracle.rotate_f32(oracle.apply_signs(x.astype(np.float32), s), 4)
+        assert np.array_equal(got32.astype(np.float64), y)
+
+
+def test_randomized_hadamard_is_orthogonal_and_keeps_dot_products():
+    import workloads as W
+    s = W.hadamard_signs(11)
+    assert set(np.unique(s)) == {-1.0, 1.0}
+    for hb in (32, 64, 128):
+        # columns of M = H_blk diag(s) / sqrt(blk), block-diagonal over 128
+        M = oracle.rotate_f64(oracle.apply_signs(np.eye(RH_D), s), hb).T
+        assert np.allclose(M @ M.T, np.eye(RH_D), atol=1e-12)
+        rng = np.random.default_rng(hb)
+        q, k = rng.standard_normal(RH_D), rng.standard_normal(RH_D)
+        qr = oracle.rotate_f64(oracle.apply_signs(q, s), hb)
+        kr = oracle.rotate_f64(oracle.apply_signs(k, s), hb)
+        assert abs(qr @ kr - q @ k) <= 1e-12 * (abs(q) @ abs(k))
+
+
+def test_all_plus_signs_quantize_like_the_plain_rotation():
+    import workloads as W
+    x = W.finish(W.normal(np.random.default_rng(5), (16, RH_D)), "bf16")
+    ones = np.ones(RH_D, np.float32)
+    for bits, G in ((4, 128), (2, 32)):
+        a = oracle.quantize_tokens(x, 128, G, bits)
+        b = oracle.quantize_tokens(x, 128, G, bits, signs=ones)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    s = W.hadamard_signs(3)
+    c = oracle.quantize_tokens(x, 128, 128, 4, signs=s)
+    assert not np.array_equal(c[0], oracle.quantize_tokens(x, 128, 128, 4)[0])

@@ -13,6 +13,8 @@ to bf16 where the workload is bf16):
   * paged mix: context lengths lognormal(ln 4096, sigma = 1), rounded and
     clipped to [1024, 32768].
   * XQuant: X ~ N(0, 1), W_k and W_v ~ N(0, 0.02^2).
+  * randomized Hadamard (QuaRot): 128 signs, each -1 or +1 with probability
+    1/2 (``hadamard_signs``).
 These stand in for the pages' Llama-3.1-8B-shaped layers at 4K-128K contexts;
 no dataset or trained weights are used.
 """
@@ -144,3 +146,10 @@ def xquant_inputs(w: Workload, n_tokens: int, seed_offset: int = 0):
     x = finish(normal(g, (n_tokens, w.hidden)), "bf16")
     wkv = finish(normal(g, (2 * w.n_kv_heads * HEAD_DIM, w.hidden), std=0.02), "bf16")
     return x, wkv
+
+
+def hadamard_signs(seed: int, n: int = HEAD_DIM) -> np.ndarray:
+    """n random signs (+1.0 / -1.0, float32) for a randomized Hadamard
+    rotation; a seeded input of the method, drawn here so both sides share it."""
+    rng = np.random.default_rng(seed)
+    return np.where(rng.random(n) < 0.5, -1.0, 1.0).astype(np.float32)
