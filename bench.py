@@ -486,7 +486,8 @@ def run_long_int2(args, dev):
 def run_rotation_sweep(args, dev):
     """Accuracy and cost of the key rotation: no rotation, block-diagonal
     Hadamard with blocks of 32, 64 and 128 channels, each with and without
-    QuaRot's random signs. 16 seqs x 8 KV heads (32 q heads) x 4096 tokens of
+    QuaRot's random signs, and the 128 block with a 64-token attention-sink
+    window. 16 seqs x 8 KV heads (32 q heads) x 4096 tokens of
     the outlier-key recipe, INT4 g128 K and V. The error is that of decode
     attention over the quantized cache against attention over the same tokens
     kept in bf16 (the library's bits-16 mode); an orthogonal rotation does not
@@ -510,10 +511,13 @@ def run_rotation_sweep(args, dev):
     ref = K.decode_attention(K.bf16_cache_desc(kb, vb), q, lens_full, T, scale).double()
     signs = torch.from_numpy(W.hadamard_signs(6)).to(dev)
     rows = []
-    for hb in (0, 32, 64, 128):
-        for use_signs in ((False, True) if hb else (False,)):
+    configs = [(hb, sg, 0) for hb in (0, 32, 64, 128) for sg in ((False, True) if hb else (False,))]
+    configs.append((128, False, 64))   # plus InnerQ's attention-sink window of 64 bf16 tokens
+    for hb, use_signs, sink in configs:
+        if True:
             spec = K.CacheSpec(S, H, bits_k=4, bits_v=4, group_k=128, group_v=128, hadamard_block_k=hb,
-                               capacity_tokens=T, hadamard_signs=signs if use_signs else None)
+                               capacity_tokens=T, hadamard_signs=signs if use_signs else None,
+                               sink_len=sink)
             cache = K.KVCache(spec, device=dev)
             ws = torch.empty(K.decode_workspace_size(cache.desc, S, HQ_, T), dtype=torch.uint8, device=dev)
             out = torch.empty((S, HQ_, D), dtype=torch.float32, device=dev)
@@ -536,7 +540,7 @@ def run_rotation_sweep(args, dev):
                     att_ms.append(e[2].elapsed_time(e3))
             assert cache.device_status() == 0
             d = out.double() - ref
-            rows.append({"hadamard_block": hb, "random_signs": use_signs,
+            rows.append({"hadamard_block": hb, "random_signs": use_signs, "sink_tokens": sink,
                          "attn_rel_l2": float(d.norm() / ref.norm()),
                          "attn_max_abs": float(d.abs().max()),
                          "append_ms": statistics.mean(app_ms),

@@ -15,4 +15,4 @@ from ._binding import (  # noqa: F401
     decode_splitk, decode_merge,
     remat_kv, rope_tables, debug_set, version,
 )
-from .cache import CacheSpec, KVCache, bf16_cache_desc  # noqa: F401
+from .cache import CacheSpec, KVCache, bf16_cache_desc, sink_view  # noqa: F401

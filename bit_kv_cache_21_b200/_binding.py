@@ -61,6 +61,10 @@ class CacheDesc(ctypes.Structure):
         ("block_table", ctypes.c_void_p),
         ("status", ctypes.c_void_p),
         ("hadamard_signs", ctypes.c_void_p),
+        ("k_sink", ctypes.c_void_p),
+        ("v_sink", ctypes.c_void_p),
+        ("sink_len", ctypes.c_int32),
+        ("reserved2", ctypes.c_int32),
     ]
 
 

@@ -30,6 +30,7 @@ class CacheSpec:
     num_pages: int = 0
     with_v: bool = True
     hadamard_signs: object = None  # device float32 [128] of +-1 (randomized Hadamard), or None
+    sink_len: int = 0              # attention-sink tokens kept in bf16
 
 
 def _row_bytes(bits: int) -> int:
@@ -65,6 +66,11 @@ class KVCache:
             n = s.num_seqs * s.num_kv_heads * s.residual_len * HEAD_DIM
             self.k_res = torch.zeros(n, dtype=torch.bfloat16, device=device)
             self.v_res = torch.zeros(n, dtype=torch.bfloat16, device=device)
+        self.k_sink = self.v_sink = None
+        if s.sink_len:
+            n = s.num_seqs * s.num_kv_heads * s.sink_len * HEAD_DIM
+            self.k_sink = torch.zeros(n, dtype=torch.bfloat16, device=device)
+            self.v_sink = torch.zeros(n, dtype=torch.bfloat16, device=device)
         self.block_table = None
         if s.paged:
             self.block_table = torch.full((s.num_seqs, s.max_pages_per_seq), -1,
@@ -86,7 +92,8 @@ class KVCache:
             capacity_tokens=s.capacity_tokens, reserved=0,
             k_codes=p(self.k_codes), v_codes=p(self.v_codes), k_sz=p(self.k_sz), v_sz=p(self.v_sz),
             k_res=p(self.k_res), v_res=p(self.v_res), block_table=p(self.block_table),
-            status=p(self.status), hadamard_signs=p(s.hadamard_signs))
+            status=p(self.status), hadamard_signs=p(s.hadamard_signs),
+            k_sink=p(self.k_sink), v_sink=p(self.v_sink), sink_len=s.sink_len, reserved2=0)
 
     def device_status(self) -> int:
         return int(self.status[0].item())
@@ -134,3 +141,10 @@ def bf16_cache_desc(k, v, status=None) -> B.CacheDesc:
         capacity_tokens=T, reserved=0, k_codes=k.data_ptr(), v_codes=v.data_ptr(),
         k_sz=None, v_sz=None, k_res=None, v_res=None, block_table=None,
         status=None if status is None else status.data_ptr())
+
+
+def sink_view(cache: KVCache, which: str):
+    """bf16 [S][H][sink_len][128] view of a cache's attention-sink rows."""
+    s = cache.spec
+    t = cache.k_sink if which == "k" else cache.v_sink
+    return t.view(s.num_seqs, s.num_kv_heads, s.sink_len, HEAD_DIM)

@@ -69,6 +69,12 @@ kvq_status validate_desc(const kvq_cache_desc *d, bool need_v) {
     if (d->status != nullptr && (reinterpret_cast<uintptr_t>(d->status) & 3u)) return KVQ_ERR_INVALID_ARG;
     if (d->hadamard_signs != nullptr && (d->hadamard_block_k == 0 || !aligned16(d->hadamard_signs)))
         return KVQ_ERR_INVALID_ARG;
+    if (d->reserved2 != 0 || d->sink_len < 0 || d->sink_len > 64) return KVQ_ERR_INVALID_ARG;
+    if (d->sink_len > 0) {
+        if (!need_v || bf16_k || d->axis_k != KVQ_PER_TOKEN || d->residual_len != 0) return KVQ_ERR_UNSUPPORTED;
+        if (d->k_sink == nullptr || d->v_sink == nullptr || !aligned16(d->k_sink) || !aligned16(d->v_sink))
+            return KVQ_ERR_INVALID_ARG;
+    }
     return KVQ_OK;
 }
 
@@ -84,6 +90,7 @@ kvq_status validate_decode(const kvq_cache_desc *d, const void *q, int q_dtype, 
     if (num_q_heads % d->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
     const int gqa = num_q_heads / d->num_kv_heads;
     if (gqa != 1 && gqa != 2 && gqa != 4) return KVQ_ERR_UNSUPPORTED;
+    if (d->sink_len > 0 && num_seqs > d->num_seqs) return KVQ_ERR_INVALID_ARG;
     if (!d->paged) {
         if (num_seqs > d->num_seqs || max_seq_len > d->capacity_tokens) return KVQ_ERR_INVALID_ARG;
     } else if (static_cast<int64_t>(max_seq_len) >
@@ -109,7 +116,7 @@ kvq_status kvq_quantize_append(const kvq_cache_desc *desc, const void *k_new, co
     if (desc->bits_k == 16) return KVQ_ERR_UNSUPPORTED;
     if (!dtype_ok(dtype) || cu_new == nullptr || seq_lens == nullptr) return KVQ_ERR_INVALID_ARG;
     if (num_seqs <= 0 || total_new_tokens < 0) return KVQ_ERR_INVALID_ARG;
-    if (!desc->paged && num_seqs > desc->num_seqs) return KVQ_ERR_INVALID_ARG;
+    if ((!desc->paged || desc->sink_len > 0) && num_seqs > desc->num_seqs) return KVQ_ERR_INVALID_ARG;
     if (total_new_tokens == 0) return KVQ_OK;  // nothing to write, lengths unchanged
     if ((v_new != nullptr) != need_v) return KVQ_ERR_INVALID_ARG;
     if (k_new == nullptr || !aligned16(k_new) || (need_v && !aligned16(v_new)))

@@ -46,6 +46,8 @@ struct AppendParams {
     int paged, page_size, max_pages, num_pages, cap;
     const int32_t *block_table;
     int32_t *status;
+    uint16_t *sink[2];  // bf16 [S][H][sink_len][D] for keys and values, or null
+    int sink_len;
 };
 
 // ---- lane-level building blocks -------------------------------------------
@@ -349,6 +351,22 @@ __global__ void __launch_bounds__(256) append_tokens_kernel(const AppendParams p
     const int h = static_cast<int>(v - static_cast<int64_t>(tok) * p.H);
     const int seq = find_seq(p.cu_new, p.num_seqs, tok);
     const int pos = __ldg(p.seq_lens + seq) + (tok - __ldg(p.cu_new + seq));
+    if (pos >= 0 && pos < p.sink_len) {
+        // attention-sink token: kept as the input rounded to bf16, not quantized
+        float raw[32];
+        load32<DT>(T.src, v, part, raw);
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(raw[2 * j], raw[2 * j + 1]);
+            w[j] = *reinterpret_cast<const uint32_t *>(&b2);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(
+            p.sink[blockIdx.y] + ((static_cast<int64_t>(seq) * p.H + h) * p.sink_len + pos) * kHeadDim + part * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        return;
+    }
     int64_t row;
     if (!dest_row(p, seq, pos, h, row)) {
         if (part == 0) status_or(p.status, KVQ_DEV_CAPACITY);
@@ -558,6 +576,9 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
         p.paged = d.paged; p.page_size = d.page_size; p.max_pages = d.max_pages_per_seq;
         p.num_pages = d.num_pages; p.cap = d.capacity_tokens;
         p.block_table = d.block_table; p.status = d.status;
+        p.sink[0] = static_cast<uint16_t *>(d.k_sink);
+        p.sink[1] = static_cast<uint16_t *>(d.v_sink);
+        p.sink_len = d.sink_len;
         const int64_t n_vec = static_cast<int64_t>(total_new) * d.num_kv_heads;
         const dim3 grid(static_cast<unsigned>((n_vec + 63) / 64), has_v ? 2 : 1);
         switch (dtype) {

@@ -58,6 +58,7 @@ namespace {
 constexpr int kTileQ = 256;        // tokens per quantized tile (64 per warp, 2 per lane)
 constexpr int kTileB = 128;        // tokens per tile of a bf16 cache (32 per warp)
 constexpr int kWinTile = 16;       // tokens per bf16 window tile (quantized caches)
+constexpr int kSinkTile = 64;      // most attention-sink tokens (one bf16 tile)
 constexpr int kMaxStages = 4;      // shared-memory ring depth, chosen on the host
 constexpr int kMaxDevices = 64;    // launch settings cached per device
 constexpr int kConsumerWarps = 4;
@@ -69,12 +70,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 enum KMode { K_TOKEN = 0, K_CHANNEL = 1, K_BF16 = 2 };
 enum VMode { V_TOKEN = 0, V_BF16 = 2 };
 
-// Stage header flags.
-constexpr int kFirst = 1, kLast = 2, kWindow = 4, kDone = 8;
+// Stage header flags. kWindow marks bf16 tiles; kSink those of the sink window.
+constexpr int kFirst = 1, kLast = 2, kWindow = 4, kDone = 8, kSink = 16;
 
 struct TileHdr {
     int seq, kvh, split, t0;
-    int n, flags, pad0, pad1;
+    int n, flags, start, pad1;  // tokens [start, n) of the tile are attended
 };
 
 struct DecodeParams {
@@ -85,6 +86,8 @@ struct DecodeParams {
     const int32_t *seq_lens;
     const void *q;
     const float *signs;  // [128] +-1 applied to the query before its rotation, or null
+    const uint16_t *k_sink, *v_sink;  // bf16 [S][H][sink_len][D], or null
+    int sink_len, sink_off_v;          // sink tokens; byte offset of the V rows in a sink tile
     float *o_part;  // [S][Hq][n_split][D]
     float2 *ml;     // [S][Hq][n_split]
     int *counter;   // item counter, zeroed before the launch
@@ -374,7 +377,7 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// One tile: rows at kc / ks / vc / vs (shared memory), `n` valid tokens, TPW
+// One tile: rows at kc / ks / vc / vs (shared memory), tokens [start, n) valid, TPW
 // tokens per warp (warp w owns tile tokens [w*TPW, w*TPW + TPW)).
 //   keys: lane j owns warp tokens j and j + 32 (TPW = 64) or token j (TPW <= 32);
 //   values: token pairs (p, p + TPW/2); the half-warps take alternate pairs,
@@ -385,7 +388,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // gk_rt); GVC likewise for the values (0 = runtime, NVG groups at most).
 template <int GQA, int KMT, int VMT, int KB, int VBITS, int TPW, int GKC, int GVC, int NVG, bool FULL>
 __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
-                                             const uint8_t *vc, const uint8_t *vs, int n,
+                                             const uint8_t *vc, const uint8_t *vs, int n, int start,
                                              const float *coef, int hstr, int cstr,
                                              const float *sums, int gk_rt, int gv_rt,
                                              WarpState<GQA, NVG> &st, float *wsm, int warp,
@@ -400,8 +403,8 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 #pragma unroll
     for (int m = 0; m < TPL; ++m) {
         const int tok = lane + 32 * m;
-        valid[m] = FULL || (tok < TPW && t_warp + tok < n);
-        tr[m] = valid[m] ? t_warp + tok : 0;  // masked lanes read row 0 (always staged)
+        valid[m] = FULL || (tok < TPW && t_warp + tok < n && t_warp + tok >= start);
+        tr[m] = valid[m] ? t_warp + tok : start;  // masked lanes read a staged, valid row
     }
 
     // ---- keys: this lane's tokens against every head ----
@@ -697,7 +700,8 @@ decode_splitk_kernel(const DecodeParams p) {
     uint8_t *stages = smem;
     uint8_t *tail = smem + static_cast<size_t>(NS) * p.stage_bytes;
     float *qs = reinterpret_cast<float *>(tail);                    // [GQA][128]
-    float *coefs = qs + GQA * kHeadDim;                              // [n_sets][CBUF], CTA-shared
+    float *qs_raw = qs + GQA * kHeadDim;                             // [GQA][128] unrotated (sinks)
+    float *coefs = qs_raw + GQA * kHeadDim;                          // [n_sets][CBUF], CTA-shared
     float *scratch_all = coefs + p.n_sets * CBUF;                    // [4][warp_floats]
     uint64_t *full = reinterpret_cast<uint64_t *>(scratch_all + kConsumerWarps * p.warp_floats);
     uint64_t *empty = full + kMaxStages;
@@ -764,7 +768,7 @@ decode_splitk_kernel(const DecodeParams p) {
             int item = __shfl_sync(0xffffffffu, next, 0);
             if (lane == 0 && item < n_items) next = atomicAdd(p.counter, 1);
             int seq = 0, kvh = 0, split = 0;
-            int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0;
+            int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0, n_sink = 0;
             if (item < n_items) {
                 item_coords(pref, p.S, p.H, item, seq, kvh, split);
                 const int T = lens[seq];
@@ -772,11 +776,15 @@ decode_splitk_kernel(const DecodeParams p) {
                 t_end = min(T, t_begin + p.chunk);
                 Tq = quantized_len(T, p.R);
                 q_end = min(t_end, Tq);
-                n_qt = q_end > t_begin ? (q_end - t_begin + TILE - 1) / TILE : 0;
+                // sink positions [0, sink_len) are read from the sink rows, as the
+                // item's last tile (after the quantized ones, so the value sums
+                // are folded first)
+                n_qt = q_end > max(t_begin, p.sink_len) ? (q_end - t_begin + TILE - 1) / TILE : 0;
                 w_begin = max(t_begin, Tq);
                 n_wt = t_end > w_begin ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
+                n_sink = (split == 0 && p.sink_len > 0) ? min(p.sink_len, T) : 0;
             }
-            const int n_tiles = (item < n_items) ? n_qt + n_wt : 1;  // 1 = the done marker
+            const int n_tiles = (item < n_items) ? n_qt + n_wt + (n_sink > 0) : 1;  // 1 = the done marker
             const int64_t sh = static_cast<int64_t>(seq) * p.H + kvh;
             for (int ti = 0; ti < n_tiles; ++ti, ++it) {
                 const int s = it % NS, r = it / NS;
@@ -800,16 +808,19 @@ decode_splitk_kernel(const DecodeParams p) {
                     break;
                 }
                 if (it == p.skip_tile) continue;  // test hook: never arrive
+                const bool sink = ti >= n_qt + n_wt;
                 const bool window = ti >= n_qt;
-                const int t0 = window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * TILE;
-                const int n = window ? min(p.bf_tile, t_end - t0) : min(TILE, q_end - t0);
+                const int t0 = sink ? 0 : (window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * TILE);
+                const int n = sink ? n_sink : (window ? min(p.bf_tile, t_end - t0) : min(TILE, q_end - t0));
                 if (lane == 0) {
                     hdr->seq = seq;
                     hdr->kvh = kvh;
                     hdr->split = split;
                     hdr->t0 = t0;
                     hdr->n = n;
-                    hdr->flags = (ti == 0 ? kFirst : 0) | (ti == n_tiles - 1 ? kLast : 0) | (window ? kWindow : 0);
+                    hdr->start = window ? 0 : max(0, p.sink_len - t0);
+                    hdr->flags = (ti == 0 ? kFirst : 0) | (ti == n_tiles - 1 ? kLast : 0) |
+                                 (window ? kWindow : 0) | (sink ? kSink : 0);
                 }
                 const uint32_t qb = (ti == 0) ? GQA * kHeadDim * p.q_bytes : 0;
                 if (qb && lane == 31) {  // the item's query rows ride with its first tile
@@ -818,7 +829,15 @@ decode_splitk_kernel(const DecodeParams p) {
                     mbar_expect_tx(bar, qb);
                     bulk_g2s(st + p.off_q, qsrc, qb, bar);
                 }
-                if (window) {
+                if (sink) {
+                    const uint32_t bytes = n * kHeadDim * 2;
+                    const int64_t row = sh * p.sink_len;
+                    if (lane < 2) {
+                        mbar_expect_tx(bar, bytes);
+                        if (lane == 0) bulk_g2s(st, p.k_sink + row * kHeadDim, bytes, bar);
+                        else bulk_g2s(st + p.sink_off_v, p.v_sink + row * kHeadDim, bytes, bar);
+                    }
+                } else if (window) {
                     const uint32_t bytes = n * kHeadDim * 2;
                     const int64_t slot = sh * p.R + (t0 - Tq);
                     if (lane < 2) {
@@ -985,6 +1004,9 @@ decode_splitk_kernel(const DecodeParams p) {
                         }
                     }
                 }
+                if (p.sink_len > 0)
+                    *reinterpret_cast<float4 *>(qs_raw + warp * kHeadDim + 4 * lane) =
+                        make_float4(x[0] * p.qscale, x[1] * p.qscale, x[2] * p.qscale, x[3] * p.qscale);
                 if (p.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
                     const float4 sg = __ldg(reinterpret_cast<const float4 *>(p.signs) + lane);
                     x[0] *= sg.x; x[1] *= sg.y; x[2] *= sg.z; x[3] *= sg.w;
@@ -1050,23 +1072,27 @@ decode_splitk_kernel(const DecodeParams p) {
                 coef = sets + min((warp * TPW) / p.R, nbt - 1) * CBUF;
             }
             constexpr int GKC_T = (KM == K_TOKEN) ? GKC : kHeadDim;
-            if (hdr.n == TILE)
+            if (hdr.n == TILE && hdr.start == 0)
                 process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, true>(
-                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, coef, QHSTR, RG::cstr,
+                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, 0, coef, QHSTR, RG::cstr,
                     coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
             else
                 process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, false>(
-                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, coef, QHSTR, RG::cstr,
-                    coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
+                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, hdr.start, coef, QHSTR,
+                    RG::cstr, coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
         } else if constexpr (KM != K_BF16) {
             if (!folded) {  // first window tile of the item
                 if (VM == V_TOKEN) fold_values();
                 folded = true;
             }
-            // bf16 keys against the plain query rows (coefficients = q)
-            process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, kHeadDim, 0, NVG, false>(
-                sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, qs, kHeadDim, 8, nullptr, p.gk, p.gv, st,
-                wsm, warp, lane);
+            if (hdr.flags & kSink)  // bf16 sink keys against the unrotated query rows
+                process_tile<GQA, K_BF16, V_BF16, 16, 16, kSinkTile / kConsumerWarps, kHeadDim, 0, NVG, false>(
+                    sb, nullptr, sb + p.sink_off_v, nullptr, hdr.n, 0, qs_raw, kHeadDim, 8, nullptr, p.gk,
+                    p.gv, st, wsm, warp, lane);
+            else  // bf16 window keys against the query rows (coefficients = q)
+                process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, kHeadDim, 0, NVG, false>(
+                    sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, 0, qs, kHeadDim, 8, nullptr, p.gk, p.gv, st,
+                    wsm, warp, lane);
         }
 
         if (hdr.flags & kLast) {
@@ -1187,6 +1213,7 @@ StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
         L.bf_tile = kWinTile;
         L.bf_off_v = kWinTile * 256;
         if (d.residual_len > 0) data = std::max(data, 2 * kWinTile * 256);
+        if (d.sink_len > 0) data = std::max(data, 2 * d.sink_len * 256);
     }
     L.off_q = round16(data);
     L.off_hdr = L.off_q + round16(gqa * kHeadDim * q_bytes);
@@ -1226,7 +1253,7 @@ kvq_status launch_variant(DecodeParams p, int max_items, cudaStream_t stream) {
     p.warp_floats = SL.floats;
     p.off_tot = SL.off_tot;
     p.n_sets = (KM == K_CHANNEL) ? 2 * (kTileQ / p.R) : 1;
-    const size_t tail = sizeof(float) * (static_cast<size_t>(GQA) * kHeadDim + static_cast<size_t>(p.n_sets) * cbuf +
+    const size_t tail = sizeof(float) * (2 * static_cast<size_t>(GQA) * kHeadDim + static_cast<size_t>(p.n_sets) * cbuf +
                                          kConsumerWarps * static_cast<size_t>(p.warp_floats)) +
                         sizeof(uint64_t) * 2 * kMaxStages + 16 + sizeof(int) * (2 * p.S + 1);
     // Ring depth: as many stages (2..4) as let the targeted CTAs per SM fit.
@@ -1342,6 +1369,10 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.seq_lens = seq_lens;
     p.q = q;
     p.signs = d.hadamard_block_k > 0 ? d.hadamard_signs : nullptr;
+    p.k_sink = static_cast<const uint16_t *>(d.k_sink);
+    p.v_sink = static_cast<const uint16_t *>(d.v_sink);
+    p.sink_len = d.sink_len;
+    p.sink_off_v = d.sink_len * kHeadDim * 2;
     p.o_part = static_cast<float *>(workspace);
     p.ml = reinterpret_cast<float2 *>(static_cast<uint8_t *>(workspace) + plan.ws_part);
     p.counter = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + plan.ws_part + plan.ws_ml);

@@ -141,6 +141,20 @@ typedef struct {
                                   exact, and (H D)^T (H D) = blk I, so q.k is kept.
                                   Other values give a transform that is not
                                   orthogonal. Requires hadamard_block_k > 0. */
+    void *k_sink, *v_sink;     /* device bf16 [num_seqs][H][sink_len][D], or NULL:
+                                  the attention-sink window of "InnerQ: Hardware-Aware
+                                  Tuning-Free Quantization of KV Cache for Large
+                                  Language Models", Abstract (high-precision windows
+                                  for recent tokens and attention sink tokens). */
+    int32_t sink_len;          /* 0, or 1..64: a sequence's first sink_len tokens
+                                  are kept in k_sink / v_sink as bf16 (the input
+                                  rounded to nearest even) instead of being
+                                  quantized, and attention reads them with the
+                                  unrotated query. Token-wise keys and values
+                                  without the recent window (residual_len == 0),
+                                  contiguous or paged; their quantized rows stay
+                                  unused. */
+    int32_t reserved2;         /* must be 0 */
 } kvq_cache_desc;
 
 /*

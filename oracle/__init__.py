@@ -274,6 +274,32 @@ def decode_attention_gqa(q, khat, vhat, scale, rotate_q_block=0, signs=None):
     return out
 
 
+def decode_attention_gqa_sinks(q, khat, vhat, k_sink, v_sink, scale, rotate_q_block=0, signs=None):
+    """Decode attention of one sequence whose first tokens are attention sinks
+    kept in high precision (InnerQ Abstract: high-precision windows for
+    recent tokens and attention-sink tokens).
+
+    q: [H_q][D]; k_sink, v_sink: [H_kv][n_sink][D] float64, the sink tokens as
+    kept (bf16 values, never rotated); khat, vhat: [H_kv][T - n_sink][D]
+    float64, the dequantized later tokens, keys in the rotated domain. Sink
+    scores take the query as given; the other scores take the query rotated
+    like the keys (randomized with `signs`). One max-shifted softmax over all
+    T tokens, in float64."""
+    q = np.asarray(q, np.float64)
+    H_q, D = q.shape
+    H_kv = khat.shape[0]
+    g = H_q // H_kv
+    qr = rotate_f64(apply_signs(q, signs), rotate_q_block) if rotate_q_block else q
+    out = np.zeros((H_q, D), np.float64)
+    for h in range(H_q):
+        kv = h // g
+        s = np.concatenate([k_sink[kv] @ q[h], khat[kv] @ qr[h]]) * scale
+        e = np.exp(s - s.max())
+        vals = np.concatenate([v_sink[kv], vhat[kv]])
+        out[h] = (e @ vals) / e.sum()
+    return out
+
+
 # --------------------------------------------------------------------------
 # Cache composition for one sequence (the method's steps in order)
 # --------------------------------------------------------------------------

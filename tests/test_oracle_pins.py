@@ -456,3 +456,34 @@ def test_all_plus_signs_quantize_like_the_plain_rotation():
     s = W.hadamard_signs(3)
     c = oracle.quantize_tokens(x, 128, 128, 4, signs=s)
     assert not np.array_equal(c[0], oracle.quantize_tokens(x, 128, 128, 4)[0])
+
+
+# ---------------------------------------------------------------------------
+# Attention-sink window (InnerQ): sink tokens kept in bf16, the rest quantized
+# ---------------------------------------------------------------------------
+
+def test_sink_attention_equals_attention_over_the_concatenated_tokens():
+    import workloads as W
+    g = np.random.default_rng(41)
+    H_kv, H_q, n_sink, T = 2, 8, 4, 37
+    q = g.standard_normal((H_q, RH_D))
+    ks, vs = g.standard_normal((H_kv, n_sink, RH_D)), g.standard_normal((H_kv, n_sink, RH_D))
+    kq, vq = g.standard_normal((H_kv, T - n_sink, RH_D)), g.standard_normal((H_kv, T - n_sink, RH_D))
+    scale = 1.0 / np.sqrt(RH_D)
+    # no rotation: one textbook softmax over sinks followed by the others
+    want = oracle.decode_attention_gqa(q, np.concatenate([ks, kq], 1), np.concatenate([vs, vq], 1), scale)
+    got = oracle.decode_attention_gqa_sinks(q, kq, vq, ks, vs, scale)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-14)
+    # rotated keys: the rotated query against rotated keys equals the plain
+    # query against the keys rotated back (H diag(s) / sqrt(n) is orthogonal)
+    s = W.hadamard_signs(2)
+    kr = oracle.rotate_f64(oracle.apply_signs(kq, s), 128)
+    got = oracle.decode_attention_gqa_sinks(q, kr, vq, ks, vs, scale, rotate_q_block=128, signs=s)
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-12)
+    # a dominant sink logit returns that sink's value row
+    q2 = np.zeros((H_q, RH_D))
+    q2[:, 0] = 1.0
+    ks2 = ks.copy()
+    ks2[:, 1, 0] = 1e4
+    got = oracle.decode_attention_gqa_sinks(q2, kq, vq, ks2, vs, 1.0)
+    assert np.allclose(got[0], vs[0, 1]) and np.allclose(got[-1], vs[1, 1])
