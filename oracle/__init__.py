@@ -313,33 +313,49 @@ def kivi_split(T, R):
     return R * ((T - 1) // R)
 
 
-def quantize_kivi_sequence(k, v, R, bits_k, bits_v, G_v):
+def quantize_kivi_sequence(k, v, R, bits_k, bits_v, G_v, v_per_channel=False):
     """KIVI-style cache of one (sequence, KV head): k, v float32 [T][D].
 
-    Keys in [0, Tq) are quantized per channel over aligned blocks of R tokens,
-    values per token in groups of G_v; tokens in [Tq, T) stay as they are
-    (the bf16 window). Returns dict with codes/sz and the window."""
+    Keys in [0, Tq) are quantized per channel over aligned blocks of R tokens
+    (KIVI Abstract). Values are quantized per token in groups of G_v, or, with
+    v_per_channel, per channel over the same R-token blocks: InnerQ (Abstract)
+    groups each cache matrix along the inner dimension of its product with the
+    attention vector, and for p @ V that dimension is the tokens. Tokens in
+    [Tq, T) stay as they are (the bf16 window). Returns dict with codes/sz and
+    the window; v_sz is [Tq/R][D][2] when v_per_channel, else [Tq][D/G_v][2]."""
     T, D = k.shape
     Tq = kivi_split(T, R)
     nb = Tq // R
-    kc = np.zeros((Tq, D * bits_k // 8), np.uint8)
-    ksz = np.zeros((nb, D, 2), np.uint16)
-    for b in range(nb):
-        kc[b * R:(b + 1) * R], ksz[b] = quantize_channel_block(k[b * R:(b + 1) * R], bits_k)
-    vc, vsz = quantize_tokens(v[:Tq], 0, G_v, bits_v)
+
+    def channel_blocks(x, bits):
+        codes = np.zeros((Tq, D * bits // 8), np.uint8)
+        sz = np.zeros((nb, D, 2), np.uint16)
+        for b in range(nb):
+            codes[b * R:(b + 1) * R], sz[b] = quantize_channel_block(x[b * R:(b + 1) * R], bits)
+        return codes, sz
+
+    kc, ksz = channel_blocks(k, bits_k)
+    if v_per_channel:
+        vc, vsz = channel_blocks(v, bits_v)
+    else:
+        vc, vsz = quantize_tokens(v[:Tq], 0, G_v, bits_v)
     return {"Tq": Tq, "k_codes": kc, "k_sz": ksz, "v_codes": vc, "v_sz": vsz,
             "k_win": np.asarray(k[Tq:], np.float64), "v_win": np.asarray(v[Tq:], np.float64)}
 
 
-def dequant_kivi_sequence(c, R, bits_k, bits_v, G_v):
+def dequant_kivi_sequence(c, R, bits_k, bits_v, G_v, v_per_channel=False):
     """Dequantized [T][D] float64 keys and values of quantize_kivi_sequence."""
     Tq = c["Tq"]
     nb = Tq // R
     D = c["k_win"].shape[1] if c["k_win"].size else c["k_codes"].shape[1] * 8 // bits_k
     kh = np.zeros((Tq, D))
+    vh = np.zeros((Tq, D))
     for b in range(nb):
         kh[b * R:(b + 1) * R] = dequant_channel_block(c["k_codes"][b * R:(b + 1) * R], c["k_sz"][b], bits_k)
-    vh = dequant_tokens(c["v_codes"], c["v_sz"], G_v, bits_v) if Tq else np.zeros((0, D))
+        if v_per_channel:
+            vh[b * R:(b + 1) * R] = dequant_channel_block(c["v_codes"][b * R:(b + 1) * R], c["v_sz"][b], bits_v)
+    if not v_per_channel and Tq:
+        vh = dequant_tokens(c["v_codes"], c["v_sz"], G_v, bits_v)
     return np.concatenate([kh, c["k_win"]]), np.concatenate([vh, c["v_win"]])
 
 

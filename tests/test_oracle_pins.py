@@ -323,6 +323,40 @@ def test_kivi_sequence_window_holds_recent_tokens():
     assert np.array_equal(c["k_codes"][128:256], cb) and np.array_equal(c["k_sz"][1], sb)
 
 
+def test_kivi_values_grouped_along_tokens():
+    # InnerQ (Abstract): V grouped along the inner dimension of p @ V, the
+    # tokens -- one group per (channel, R-token block)
+    g = np.random.default_rng(13)
+    T, D, R = 300, 128, 64
+    k = g.standard_normal((T, D)).astype(np.float32)
+    v = (g.standard_normal((T, D)) * (1 + np.arange(D) / 16)).astype(np.float32)
+    c = oracle.quantize_kivi_sequence(k, v, R, 4, 4, 0, v_per_channel=True)
+    Tq = c["Tq"]
+    assert Tq == 256 and c["v_sz"].shape == (Tq // R, D, 2)
+    # same data on both sides: values quantize exactly like the per-channel keys
+    ck = oracle.quantize_kivi_sequence(v, v, R, 4, 4, 0, v_per_channel=True)
+    assert np.array_equal(ck["v_codes"], ck["k_codes"]) and np.array_equal(ck["v_sz"], ck["k_sz"])
+    # a group is one channel's R tokens of one block
+    q = np.stack([oracle.unpack_codes(c["v_codes"][t], D, 4) for t in range(Tq)])
+    for b, d in ((0, 0), (1, 77), (3, 127)):
+        s, z, qc = oracle.quantize_group(np.ascontiguousarray(v[b * R:(b + 1) * R, d]), 4)
+        assert (s, z) == tuple(c["v_sz"][b, d])
+        assert np.array_equal(q[b * R:(b + 1) * R, d], qc)
+    kh, vh = oracle.dequant_kivi_sequence(c, R, 4, 4, 0, v_per_channel=True)
+    assert np.array_equal(vh[Tq:], v[Tq:])
+    s = c["v_sz"][:, :, 0].view(np.float16).astype(np.float64)  # [nb][D]
+    assert np.all(np.abs(vh[:Tq] - v[:Tq]).reshape(Tq // R, R, D) <= s[:, None, :] * (0.5 + 2.0 ** -17))
+    # the scale and zero of a channel factor out of a block's weighted sum:
+    # sum_t p_t vhat_t = s * sum_t p_t q_t + z * sum_t p_t
+    pw = g.random(Tq)
+    z = c["v_sz"][:, :, 1].view(np.float16).astype(np.float64)
+    for b in range(Tq // R):
+        sl = slice(b * R, (b + 1) * R)
+        want = pw[sl] @ vh[sl]
+        got = s[b] * (pw[sl] @ q[sl]) + z[b] * pw[sl].sum()
+        assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
 def test_effective_bits_match_printed_table():
     with open(os.path.join(GOLDEN, "effective_bits.txt")) as f:
         rows = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
