@@ -483,74 +483,120 @@ def run_long_int2(args, dev):
             "step_GBps": mb / ((statistics.mean(app) + statistics.mean(att)) * 1e-3) / 1e9}
 
 
-def run_rotation_sweep(args, dev):
-    """Accuracy and cost of the key rotation: no rotation, block-diagonal
-    Hadamard with blocks of 32, 64 and 128 channels, each with and without
-    QuaRot's random signs, and the 128 block with a 64-token attention-sink
-    window. 16 seqs x 8 KV heads (32 q heads) x 4096 tokens of
-    the outlier-key recipe, INT4 g128 K and V. The error is that of decode
-    attention over the quantized cache against attention over the same tokens
-    kept in bf16 (the library's bits-16 mode); an orthogonal rotation does not
-    change the latter."""
+def _sweep_setup(dev, seed=6):
+    """Shared data of the accuracy/cost sweeps: 16 seqs x 8 KV heads (32 q
+    heads) x 4096 tokens of the outlier-key recipe, bf16, and decode attention
+    over the same tokens kept in bf16 (the library's bits-16 mode)."""
     import torch
     import bit_kv_cache_21_b200 as K
-    import workloads as W
     S, H, HQ_, T = 16, 8, 32, 4096
-    n_rep = 5
     gen = torch.Generator(device=dev)
-    gen.manual_seed(6)
-    k, v = _synthetic_kv(gen, S * T, H, dev, torch, 6)               # [S*T][H][D]
+    gen.manual_seed(seed)
+    k, v = _synthetic_kv(gen, S * T, H, dev, torch, seed)               # [S*T][H][D]
     q = torch.randn((S, HQ_, D), generator=gen, device=dev).to(torch.bfloat16)
-    kb = k.view(S, T, H, D).permute(0, 2, 1, 3).contiguous()          # [S][H][T][D]
+    kb = k.view(S, T, H, D).permute(0, 2, 1, 3).contiguous()            # [S][H][T][D]
     vb = v.view(S, T, H, D).permute(0, 2, 1, 3).contiguous()
     lens_full = torch.full((S,), T, dtype=torch.int32, device=dev)
     cu = torch.arange(0, (S + 1) * T, T, dtype=torch.int32, device=dev)
     scale = 1.0 / math.sqrt(D)
+    ref = K.decode_attention(K.bf16_cache_desc(kb, vb), q, lens_full, T, scale).double()
+    return dict(S=S, H=H, HQ=HQ_, T=T, k=k, v=v, q=q, lens_full=lens_full, cu=cu, scale=scale, ref=ref)
+
+
+def _sweep_row(spec_kw, d, dev, bytes_per_token_head, n_rep=5):
+    """Append the sweep's tokens into a fresh cache of `spec_kw`, then decode;
+    mean times over n_rep repetitions after one warm-up (L2 flushed before
+    each timed launch), and the error of the attention against bf16."""
+    import torch
+    import bit_kv_cache_21_b200 as K
+    S, H, HQ_, T = d["S"], d["H"], d["HQ"], d["T"]
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ref = K.decode_attention(K.bf16_cache_desc(kb, vb), q, lens_full, T, scale).double()
+    cache = K.KVCache(K.CacheSpec(S, H, capacity_tokens=T, **spec_kw), device=dev)
+    ws = torch.empty(K.decode_workspace_size(cache.desc, S, HQ_, T), dtype=torch.uint8, device=dev)
+    out = torch.empty((S, HQ_, D), dtype=torch.float32, device=dev)
+    app_ms, att_ms = [], []
+    for rep in range(n_rep + 1):
+        lens = torch.zeros(S, dtype=torch.int32, device=dev)
+        flush_l2(flush)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(stream)
+        K.quantize_append(cache.desc, d["k"], d["v"], d["cu"], lens)
+        e[1].record(stream)
+        flush_l2(flush)
+        e[2].record(stream)
+        K.decode_attention(cache.desc, d["q"], d["lens_full"], T, d["scale"], out=out, workspace=ws)
+        e[3].record(stream)
+        torch.cuda.synchronize()
+        if rep > 0:  # the first repetition warms up
+            app_ms.append(e[0].elapsed_time(e[1]))
+            att_ms.append(e[2].elapsed_time(e[3]))
+    assert cache.device_status() == 0
+    diff = out.double() - d["ref"]
+    row = {"attn_rel_l2": float(diff.norm() / d["ref"].norm()),
+           "attn_max_abs": float(diff.abs().max()),
+           "append_ms": statistics.mean(app_ms),
+           "append_tokens_per_s": S * T / (statistics.mean(app_ms) * 1e-3),
+           "decode_ms": statistics.mean(att_ms),
+           "decode_GBps": S * H * T * bytes_per_token_head / (statistics.mean(att_ms) * 1e-3) / 1e9}
+    del cache, ws
+    return row
+
+
+SWEEP_WORKLOAD = ("16 seqs x 8 kv / 32 q heads x 4096 tokens, bf16 K with 4 outlier channels x20; "
+                  "error of decode attention against attention over the same tokens in bf16")
+
+
+def run_rotation_sweep(args, dev):
+    """Accuracy and cost of the key rotation: no rotation, block-diagonal
+    Hadamard with blocks of 32, 64 and 128 channels, each with and without
+    QuaRot's random signs, and the 128 block with a 64-token attention-sink
+    window; INT4 g128 K and V."""
+    import torch
+    import workloads as W
+    d = _sweep_setup(dev)
     signs = torch.from_numpy(W.hadamard_signs(6)).to(dev)
     rows = []
     configs = [(hb, sg, 0) for hb in (0, 32, 64, 128) for sg in ((False, True) if hb else (False,))]
     configs.append((128, False, 64))   # plus InnerQ's attention-sink window of 64 bf16 tokens
     for hb, use_signs, sink in configs:
-        if True:
-            spec = K.CacheSpec(S, H, bits_k=4, bits_v=4, group_k=128, group_v=128, hadamard_block_k=hb,
-                               capacity_tokens=T, hadamard_signs=signs if use_signs else None,
-                               sink_len=sink)
-            cache = K.KVCache(spec, device=dev)
-            ws = torch.empty(K.decode_workspace_size(cache.desc, S, HQ_, T), dtype=torch.uint8, device=dev)
-            out = torch.empty((S, HQ_, D), dtype=torch.float32, device=dev)
-            app_ms, att_ms = [], []
-            for rep in range(n_rep + 1):
-                lens = torch.zeros(S, dtype=torch.int32, device=dev)
-                flush_l2(flush)
-                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-                e[0].record(stream)
-                K.quantize_append(cache.desc, k, v, cu, lens)
-                e[1].record(stream)
-                flush_l2(flush)
-                e[2].record(stream)
-                K.decode_attention(cache.desc, q, lens_full, T, scale, out=out, workspace=ws)
-                e3 = torch.cuda.Event(enable_timing=True)
-                e3.record(stream)
-                torch.cuda.synchronize()
-                if rep > 0:  # the first repetition warms up
-                    app_ms.append(e[0].elapsed_time(e[1]))
-                    att_ms.append(e[2].elapsed_time(e3))
-            assert cache.device_status() == 0
-            d = out.double() - ref
-            rows.append({"hadamard_block": hb, "random_signs": use_signs, "sink_tokens": sink,
-                         "attn_rel_l2": float(d.norm() / ref.norm()),
-                         "attn_max_abs": float(d.abs().max()),
-                         "append_ms": statistics.mean(app_ms),
-                         "append_tokens_per_s": S * T / (statistics.mean(app_ms) * 1e-3),
-                         "decode_ms": statistics.mean(att_ms),
-                         "decode_GBps": S * H * T * BYTES_PER_TOKEN_HEAD / (statistics.mean(att_ms) * 1e-3) / 1e9})
-            del cache, ws
-    return {"workload": "rotation sweep: 16 seqs x 8 kv / 32 q heads x 4096 tokens, bf16 K with 4 "
-                        "outlier channels x20, INT4 g128 K and V; error of decode attention against "
-                        "attention over the same tokens in bf16",
+        kw = dict(bits_k=4, bits_v=4, group_k=128, group_v=128, hadamard_block_k=hb,
+                  hadamard_signs=signs if use_signs else None, sink_len=sink)
+        row = {"hadamard_block": hb, "random_signs": use_signs, "sink_tokens": sink}
+        row.update(_sweep_row(kw, d, dev, BYTES_PER_TOKEN_HEAD))
+        rows.append(row)
+    return {"workload": "rotation sweep: " + SWEEP_WORKLOAD + "; INT4 g128 K and V", "rows": rows}
+
+
+def _layout_bytes(bits, per_channel, G, R):
+    """Stored bytes of one tensor per (token, head): codes plus the share of
+    the 4-byte (scale, zero) pairs (per token: D/G of them; per channel: D per
+    R-token block)."""
+    return D * bits // 8 + (D * 4 // R if per_channel else (D // G) * 4)
+
+
+def run_grouping_sweep(args, dev):
+    """Accuracy and cost of the grouping axes with a 128-token bf16 window, no
+    rotation: token-wise groups for both tensors; KIVI's keys per channel with
+    values per token; InnerQ's keys grouped along channels (per token) with
+    values grouped along tokens (per channel); both per channel. INT4 with
+    128-wide groups and INT2 with 32-wide token groups."""
+    d = _sweep_setup(dev)
+    R = 128
+    rows = []
+    for bits, G in ((4, 128), (2, 32)):
+        for pk, pv, name in ((False, False, "token/token"), (True, False, "KIVI: channel/token"),
+                             (False, True, "InnerQ: token/channel"), (True, True, "channel/channel")):
+            kw = dict(bits_k=bits, bits_v=bits, group_k=R if pk else G, group_v=R if pv else G,
+                      per_channel_k=pk, per_channel_v=pv, residual_len=R)
+            bph = _layout_bytes(bits, pk, G, R) + _layout_bytes(bits, pv, G, R)
+            row = {"bits": bits, "token_group": G, "keys": "channel" if pk else "token",
+                   "values": "channel" if pv else "token", "layout": name,
+                   "bytes_per_token_head": bph}
+            row.update(_sweep_row(kw, d, dev, bph))
+            rows.append(row)
+    return {"workload": "grouping sweep: " + SWEEP_WORKLOAD + "; residual window 128 bf16 tokens; "
+                        "keys / values grouped per token or per channel (128-token blocks)",
             "rows": rows}
 
 
@@ -670,9 +716,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--part", default="all",
-                    choices=["all", "decode", "remat", "long_int2", "paged_mix", "rotation_sweep"],
+                    choices=["all", "decode", "remat", "long_int2", "paged_mix", "rotation_sweep",
+                             "grouping_sweep"],
                     help="run one leg alone: decode (the metric's step), remat, long_int2, "
-                         "paged_mix or rotation_sweep (the last four print their own line)")
+                         "paged_mix, rotation_sweep or grouping_sweep (all but decode print "
+                         "their own line)")
     ap.add_argument("--remat-batch", type=int, default=8)
     ap.add_argument("--remat-steps", type=int, default=10)
     args = ap.parse_args()
@@ -732,14 +780,16 @@ def main():
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
         return
-    if args.part == "rotation_sweep":
+    if args.part in ("rotation_sweep", "grouping_sweep"):
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
-        sw = run_rotation_sweep(args, dev)
+        rot = args.part == "rotation_sweep"
+        sw = (run_rotation_sweep if rot else run_grouping_sweep)(args, dev)
         if rank == 0:
-            print(json.dumps({"metric": "decode-attn error vs bf16 and cost per key rotation",
+            print(json.dumps({"metric": "decode-attn error vs bf16 and cost per " +
+                                        ("key rotation" if rot else "grouping layout"),
                               "n_gpus": world, "data": "synthetic",
-                              "config": {"workload": sw["workload"]}, "rotation_sweep": sw}))
+                              "config": {"workload": sw["workload"]}, args.part: sw}))
         if world > 1:
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
@@ -762,6 +812,7 @@ def main():
     li = run_long_int2(args, torch.device("cuda", local_rank)) if args.part == "all" else None
     pm = run_paged_mix(args, torch.device("cuda", local_rank)) if args.part == "all" else None
     sw = run_rotation_sweep(args, torch.device("cuda", local_rank)) if args.part == "all" else None
+    gs = run_grouping_sweep(args, torch.device("cuda", local_rank)) if args.part == "all" else None
 
     # max over ranks of the device time; bytes summed over ranks
     total_ms, total_bytes, e2e_s, e2e_bytes = res["total_ms"], res["bytes"], res["e2e_s"], res["e2e_bytes"]
@@ -813,6 +864,8 @@ def main():
             line["paged_mix"] = pm
         if sw is not None:
             line["rotation_sweep"] = sw
+        if gs is not None:
+            line["grouping_sweep"] = gs
         print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()

@@ -21,6 +21,7 @@ class CacheSpec:
     group_k: int = 128
     group_v: int = 128
     per_channel_k: bool = False
+    per_channel_v: bool = False    # values grouped along tokens (group_v == residual_len)
     hadamard_block_k: int = 0
     residual_len: int = 0
     capacity_tokens: int = 0      # contiguous layout
@@ -60,7 +61,11 @@ class KVCache:
                 n = rows * (HEAD_DIM // s.group_k)
             self.k_sz = torch.zeros(n * 4, dtype=u8, device=device)
         if s.with_v and s.bits_v != 16:
-            self.v_sz = torch.zeros(rows * (HEAD_DIM // s.group_v) * 4, dtype=u8, device=device)
+            if s.per_channel_v:
+                n = s.num_seqs * s.num_kv_heads * (s.capacity_tokens // s.group_v) * HEAD_DIM
+            else:
+                n = rows * (HEAD_DIM // s.group_v)
+            self.v_sz = torch.zeros(n * 4, dtype=u8, device=device)
         self.k_res = self.v_res = None
         if s.residual_len:
             n = s.num_seqs * s.num_kv_heads * s.residual_len * HEAD_DIM
@@ -85,7 +90,8 @@ class KVCache:
             num_seqs=s.num_seqs, num_kv_heads=s.num_kv_heads, head_dim=HEAD_DIM,
             bits_k=s.bits_k, bits_v=s.bits_v if s.with_v else 0,
             group_k=s.group_k, group_v=s.group_v,
-            axis_k=B.PER_CHANNEL if s.per_channel_k else B.PER_TOKEN, axis_v=B.PER_TOKEN,
+            axis_k=B.PER_CHANNEL if s.per_channel_k else B.PER_TOKEN,
+            axis_v=B.PER_CHANNEL if s.per_channel_v else B.PER_TOKEN,
             hadamard_block_k=s.hadamard_block_k, residual_len=s.residual_len,
             paged=int(s.paged), page_size=s.page_size if s.paged else 0,
             max_pages_per_seq=s.max_pages_per_seq, num_pages=s.num_pages,
@@ -117,7 +123,7 @@ class KVCache:
         G = s.group_k if which == "k" else s.group_v
         import torch
         t16 = t.view(torch.int16)
-        if which == "k" and s.per_channel_k:
+        if (s.per_channel_k if which == "k" else s.per_channel_v):
             return t16.view(s.num_seqs, s.num_kv_heads, s.capacity_tokens // G, HEAD_DIM, 2)
         if s.paged:
             return t16.view(s.num_pages, s.num_kv_heads, s.page_size, HEAD_DIM // G, 2)

@@ -32,18 +32,24 @@ kvq_status validate_desc(const kvq_cache_desc *d, bool need_v) {
         return KVQ_ERR_INVALID_ARG;
     auto bits_ok = [](int b) { return b == 2 || b == 4 || b == 16; };
     if (!bits_ok(d->bits_k) || (need_v && !bits_ok(d->bits_v))) return KVQ_ERR_INVALID_ARG;
-    if (d->axis_v != KVQ_PER_TOKEN) return KVQ_ERR_UNSUPPORTED;
     if (d->axis_k != KVQ_PER_TOKEN && d->axis_k != KVQ_PER_CHANNEL) return KVQ_ERR_INVALID_ARG;
+    if (d->axis_v != KVQ_PER_TOKEN && d->axis_v != KVQ_PER_CHANNEL) return KVQ_ERR_INVALID_ARG;
     const bool bf16_k = d->bits_k == 16, bf16_v = need_v && d->bits_v == 16;
+    const bool chan_v = need_v && d->axis_v == KVQ_PER_CHANNEL;
     if (need_v && bf16_k != bf16_v) return KVQ_ERR_UNSUPPORTED;
     if (bf16_k && (d->paged || d->residual_len || d->hadamard_block_k)) return KVQ_ERR_UNSUPPORTED;
     if (!bf16_k) {
         if (d->axis_k == KVQ_PER_TOKEN && !token_group_ok(d->group_k)) return KVQ_ERR_INVALID_ARG;
-        if (need_v && !token_group_ok(d->group_v)) return KVQ_ERR_INVALID_ARG;
+        if (need_v && !chan_v && !token_group_ok(d->group_v)) return KVQ_ERR_INVALID_ARG;
     }
     if (d->axis_k == KVQ_PER_CHANNEL) {
         if (bf16_k || d->paged || d->hadamard_block_k) return KVQ_ERR_UNSUPPORTED;
         if (d->residual_len != d->group_k) return KVQ_ERR_INVALID_ARG;
+    }
+    if (chan_v) {  // values grouped along tokens: one block of the window at a time
+        if (bf16_v || d->paged || d->hadamard_block_k) return KVQ_ERR_UNSUPPORTED;
+        if (d->residual_len != d->group_v) return KVQ_ERR_INVALID_ARG;
+        if (d->bits_k != d->bits_v) return KVQ_ERR_UNSUPPORTED;
     }
     if (d->residual_len != 0) {
         if (!(d->residual_len == 64 || d->residual_len == 128 || d->residual_len == 256))

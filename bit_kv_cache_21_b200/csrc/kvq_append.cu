@@ -384,7 +384,7 @@ struct WindowParams {
     uint8_t *k_codes, *v_codes;
     __half2 *k_sz, *v_sz;
     int bits_k, bits_v, group_k, group_v;
-    int k_per_channel;
+    int k_per_channel, v_per_channel;
     int R, H, cap;
     const int32_t *cu_new;
     const int32_t *seq_lens;  // lengths before this append
@@ -392,9 +392,43 @@ struct WindowParams {
     int32_t *status;
 };
 
+// Quantize one block of R staged bf16 rows [R][128] per channel (each
+// channel's R values one group; KIVI keys, InnerQ values) into `codes`
+// (R rows packed along channels) and `sz` ([128] half2). Called by the whole
+// CTA; `qk` is [R][128] bytes of scratch.
+__device__ void flush_channel_block(const uint16_t *src, uint8_t *qk, int R, int bits, uint8_t *codes,
+                                    __half2 *sz) {
+    const int L = (1 << bits) - 1;
+    const float Lf = static_cast<float>(L);
+    for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x) {
+        float mn = bf16_bits_to_float(src[d]), mx = mn;
+        for (int t = 1; t < R; ++t) {
+            const float v = bf16_bits_to_float(src[t * kHeadDim + d]);
+            mn = fminf(mn, v);
+            mx = fmaxf(mx, v);
+        }
+        const QParams qp = qparams(mn, mx, L);
+        for (int t = 0; t < R; ++t)
+            qk[t * kHeadDim + d] = static_cast<uint8_t>(qcode(bf16_bits_to_float(src[t * kHeadDim + d]), qp, Lf));
+        sz[d] = qp.sz;
+    }
+    __syncthreads();
+    // Pack along channels: one 32-bit word holds 32/bits channels.
+    const int per_word = 32 / bits;
+    const int words_per_row = kHeadDim / per_word;
+    for (int i = threadIdx.x; i < R * words_per_row; i += blockDim.x) {
+        const int t = i / words_per_row, w = i - t * words_per_row;
+        uint32_t v = 0;
+        for (int j = 0; j < per_word; ++j)
+            v |= static_cast<uint32_t>(qk[t * kHeadDim + w * per_word + j]) << (bits * j);
+        reinterpret_cast<uint32_t *>(codes + static_cast<size_t>(t) * (kHeadDim * bits / 8))[w] = v;
+    }
+    __syncthreads();  // qk is free for the next tensor
+}
+
 // One CTA per (flushed block slot, head, sequence). The block's R tokens come
 // from the old window (positions below the old length) and from the new
-// tokens; keys are quantized per channel (or per token), values per token.
+// tokens; each tensor is quantized per channel or per token.
 __global__ void __launch_bounds__(256) window_flush_kernel(const WindowParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int seq = blockIdx.z, h = blockIdx.y;
@@ -437,36 +471,14 @@ __global__ void __launch_bounds__(256) window_flush_kernel(const WindowParams p)
     const int lane = threadIdx.x & 31, part = lane & 3;
     const int64_t row0 = sh * p.cap + static_cast<int64_t>(b) * R;
 
-    // Keys.
-    if (p.k_per_channel) {
-        const int L = (1 << p.bits_k) - 1;
-        const float Lf = static_cast<float>(L);
-        for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x) {
-            float mn = bf16_bits_to_float(kb[d]), mx = mn;
-            for (int t = 1; t < R; ++t) {
-                const float v = bf16_bits_to_float(kb[t * kHeadDim + d]);
-                mn = fminf(mn, v);
-                mx = fmaxf(mx, v);
-            }
-            const QParams qp = qparams(mn, mx, L);
-            for (int t = 0; t < R; ++t)
-                qk[t * kHeadDim + d] = static_cast<uint8_t>(qcode(bf16_bits_to_float(kb[t * kHeadDim + d]), qp, Lf));
-            p.k_sz[(sh * (p.cap / R) + b) * kHeadDim + d] = qp.sz;
-        }
-        __syncthreads();
-        // Pack along channels: one 32-bit word holds 32/bits channels.
-        const int per_word = 32 / p.bits_k;
-        const int words_per_row = kHeadDim / per_word;
-        for (int i = threadIdx.x; i < R * words_per_row; i += blockDim.x) {
-            const int t = i / words_per_row, w = i - t * words_per_row;
-            uint32_t v = 0;
-            for (int j = 0; j < per_word; ++j)
-                v |= static_cast<uint32_t>(qk[t * kHeadDim + w * per_word + j]) << (p.bits_k * j);
-            reinterpret_cast<uint32_t *>(p.k_codes + (row0 + t) * (kHeadDim * p.bits_k / 8))[w] = v;
-        }
-    }
+    // Per-channel tensors (keys; values grouped along tokens).
+    if (p.k_per_channel) flush_channel_block(kb, qk, R, p.bits_k, p.k_codes + row0 * (kHeadDim * p.bits_k / 8),
+                                             p.k_sz + (sh * (p.cap / R) + b) * kHeadDim);
+    if (p.v_per_channel) flush_channel_block(vb, qk, R, p.bits_v, p.v_codes + row0 * (kHeadDim * p.bits_v / 8),
+                                             p.v_sz + (sh * (p.cap / R) + b) * kHeadDim);
     // Per-token tensors: 8 vectors per warp, 64 per pass.
-    for (int tsel = p.k_per_channel ? 1 : 0; tsel < 2; ++tsel) {
+    for (int tsel = 0; tsel < 2; ++tsel) {
+        if (tsel ? p.v_per_channel : p.k_per_channel) continue;
         const uint16_t *src = tsel ? vb : kb;
         const int bits = tsel ? p.bits_v : p.bits_k;
         const int G = tsel ? p.group_v : p.group_k;
@@ -548,6 +560,7 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
         w.bits_k = d.bits_k; w.bits_v = d.bits_v;
         w.group_k = d.group_k; w.group_v = d.group_v;
         w.k_per_channel = d.axis_k == KVQ_PER_CHANNEL;
+        w.v_per_channel = d.axis_v == KVQ_PER_CHANNEL;
         w.R = d.residual_len; w.H = d.num_kv_heads; w.cap = d.capacity_tokens;
         w.cu_new = cu_new; w.seq_lens = seq_lens;
         w.num_seqs = num_seqs; w.total_tokens = total_new;

@@ -58,7 +58,6 @@ namespace {
 constexpr int kTileQ = 256;        // tokens per quantized tile (64 per warp, 2 per lane)
 constexpr int kTileB = 128;        // tokens per tile of a bf16 cache (32 per warp)
 constexpr int kWinTile = 16;       // tokens per bf16 window tile (quantized caches)
-constexpr int kSinkTile = 64;      // most attention-sink tokens (one bf16 tile)
 constexpr int kMaxStages = 4;      // shared-memory ring depth, chosen on the host
 constexpr int kMaxDevices = 64;    // launch settings cached per device
 constexpr int kConsumerWarps = 4;
@@ -68,7 +67,9 @@ constexpr int kMaxGroups = 8;      // kHeadDim / smallest token-wise group (16)
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum KMode { K_TOKEN = 0, K_CHANNEL = 1, K_BF16 = 2 };
-enum VMode { V_TOKEN = 0, V_BF16 = 2 };
+// V_CHANNEL: values grouped along tokens, one (scale, zero) per channel and
+// R-token block (InnerQ's inner-dimension grouping for p @ V).
+enum VMode { V_TOKEN = 0, V_CHANNEL = 1, V_BF16 = 2 };
 
 // Stage header flags. kWindow marks bf16 tiles; kSink those of the sink window.
 constexpr int kFirst = 1, kLast = 2, kWindow = 4, kDone = 8, kSink = 16;
@@ -87,7 +88,7 @@ struct DecodeParams {
     const void *q;
     const float *signs;  // [128] +-1 applied to the query before its rotation, or null
     const uint16_t *k_sink, *v_sink;  // bf16 [S][H][sink_len][D], or null
-    int sink_len, sink_off_v;          // sink tokens; byte offset of the V rows in a sink tile
+    int sink_len;                      // sink tokens (read in window-sized bf16 tiles)
     float *o_part;  // [S][Hq][n_split][D]
     float2 *ml;     // [S][Hq][n_split]
     int *counter;   // item counter, zeroed before the launch
@@ -279,6 +280,21 @@ __device__ __forceinline__ void value_channels(const float a[8], float W, float 
     }
 }
 
+// The 4-channel half (channels 4h..4h+3 of a slice) of value_channels: INT4
+// channels are independent, and an INT2 byte's planes stay inside one half.
+template <int VBITS>
+__device__ __forceinline__ void value_channels4(const float a[4], float W, float out[4]) {
+    if constexpr (VBITS == 4) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) out[c] = fmaf(256.0f, a[c], -128.0f * W);
+    } else {
+        out[0] = fmaf(256.0f, a[0], -128.0f * W);
+        out[1] = 64.0f * (a[1] - a[0]);
+        out[2] = 16.0f * (a[2] - a[1]);
+        out[3] = fmaf(16.0f, a[3], -8.0f * W) - 4.0f * (a[2] - a[0]);
+    }
+}
+
 // ---- key coefficients -------------------------------------------------------
 // One head's key coefficients, built by one warp from the lane's 4 channels
 // x[0..3] (channels 4*lane..4*lane+3 of the rotated query, scaled to log2
@@ -355,9 +371,19 @@ __device__ __forceinline__ void build_head(const float xin[4], const uint8_t *ch
     }
 }
 
+// Folded value sums of V_CHANNEL kernels (absent from the others, whose state
+// is then exactly what it was without this mode).
+template <int GQA, bool VCH>
+struct FoldedSums {
+    float of[GQA][4];      // folded value sums of earlier tiles, 4 channels per
+                           // lane (half-warp h: channels 4h..4h+3)
+};
+template <int GQA>
+struct FoldedSums<GQA, false> {};
+
 // Per-warp decode state of the current item.
-template <int GQA, int NVG>
-struct WarpState {
+template <int GQA, int NVG, bool VCH>
+struct WarpState : FoldedSums<GQA, VCH> {
     float mref[GQA];       // reference maximum per head (log2 units; warp-uniform)
     float thr[GQA];        // mref + slack: scores above it move the reference
     float l[GQA];          // this lane's tokens: sum of the weights p
@@ -383,15 +409,17 @@ __device__ __forceinline__ float warp_max(float v) {
 //   values: token pairs (p, p + TPW/2); the half-warps take alternate pairs,
 //     16 lanes cover the 128 channels (8 each); the weights of a pair sit
 //     side by side, so one f32x2 FMA serves both tokens.
-// FULL: all 4*TPW tokens are valid. KMT/KB: key mode and bits of this tile
+// FULL: all 4*TPW tokens are valid. SNK: the tile may start at `start` > 0
+// (sink caches; otherwise start is 0). KMT/KB: key mode and bits of this tile
 // (window tiles are bf16). GKC: compile-time key group size (0 = runtime
 // gk_rt); GVC likewise for the values (0 = runtime, NVG groups at most).
-template <int GQA, int KMT, int VMT, int KB, int VBITS, int TPW, int GKC, int GVC, int NVG, bool FULL>
+template <int GQA, int KMT, int VMT, int KB, int VBITS, int TPW, int GKC, int GVC, int NVG, bool FULL,
+          bool SNK, bool VCH>
 __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
                                              const uint8_t *vc, const uint8_t *vs, int n, int start,
                                              const float *coef, int hstr, int cstr,
                                              const float *sums, int gk_rt, int gv_rt,
-                                             WarpState<GQA, NVG> &st, float *wsm, int warp,
+                                             WarpState<GQA, NVG, VCH> &st, float *wsm, int warp,
                                              int lane) {
     using RG = RowGeo<KB>;
     constexpr int TPL = (TPW >= 64) ? 2 : 1;  // key tokens per lane
@@ -403,8 +431,8 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 #pragma unroll
     for (int m = 0; m < TPL; ++m) {
         const int tok = lane + 32 * m;
-        valid[m] = FULL || (tok < TPW && t_warp + tok < n && t_warp + tok >= start);
-        tr[m] = valid[m] ? t_warp + tok : start;  // masked lanes read a staged, valid row
+        valid[m] = FULL || (tok < TPW && t_warp + tok < n && (!SNK || t_warp + tok >= start));
+        tr[m] = valid[m] ? t_warp + tok : (SNK ? start : 0);  // masked lanes read a staged, valid row
     }
 
     // ---- keys: this lane's tokens against every head ----
@@ -563,6 +591,10 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
                 for (int v = 0; v < NVG; ++v) { st.W[g][v] *= alpha; st.Z[g][v] *= alpha; }
 #pragma unroll
                 for (int c = 0; c < 8; ++c) { st.o[g][c].x *= alpha; st.o[g][c].y *= alpha; }
+                if constexpr (VCH) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) st.of[g][c] *= alpha;
+                }
             }
         }
     }
@@ -578,7 +610,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
         }
     }
     // Value weights w = p * s per (token, value group), at their pair slot.
-    const int n_vg = (VMT == V_BF16) ? 1 : (GVC ? kHeadDim / GVC : kHeadDim / gv_rt);
+    const int n_vg = (VMT != V_TOKEN) ? 1 : (GVC ? kHeadDim / GVC : kHeadDim / gv_rt);
     float2 *wsm2 = reinterpret_cast<float2 *>(wsm);
     // pair rows padded by 16 bytes so the lanes' rows start in different bank groups
     const int pstr = n_vg * GQA + 2;
@@ -591,6 +623,14 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
                 for (int m = 0; m < TPL; ++m)
 #pragma unroll
                     for (int g = 0; g < GQA; ++g) w[m][g] = p[m][g];
+            } else if constexpr (VMT == V_CHANNEL) {  // scales come per channel, after the pass
+#pragma unroll
+                for (int m = 0; m < TPL; ++m)
+#pragma unroll
+                    for (int g = 0; g < GQA; ++g) {
+                        w[m][g] = p[m][g];
+                        st.W[g][0] += p[m][g];
+                    }
             } else {
 #pragma unroll
                 for (int m = 0; m < TPL; ++m) {
@@ -617,7 +657,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 
     // ---- values ----
     const int slice = lane & 15, parity = lane >> 4;
-    const int gv_lane = (VMT == V_BF16) ? 0 : (slice * 8) / (GVC ? GVC : gv_rt);
+    const int gv_lane = (VMT != V_TOKEN) ? 0 : (slice * 8) / (GVC ? GVC : gv_rt);
 #pragma unroll 2
     for (int k = 0; k < HALF / 2; ++k) {
         const int pi = 2 * k + parity;
@@ -650,6 +690,42 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 #pragma unroll
             for (int c = 0; c < 8; ++c) ffma2(st.o[g][c], w[g], f[c]);
     }
+    if constexpr (VMT == V_CHANNEL) {
+        // The warp's tokens lie in one R-token block (R >= 64, tiles aligned):
+        // fold this tile's sums with the block's channel scales, sum_t p_t v_t =
+        // s * sum_t p_t c_t + z * sum_t p_t. The halves swap partial sums so
+        // half h owns channels 4h..4h+3 of its slice; vs points at the block's
+        // [128] (scale, zero) pairs. A warp without valid tokens skips (its
+        // block's scales need not be staged).
+        if (FULL || t_warp < n) {
+            const int half = lane >> 4;
+            const uint4 u = lds128(vs + (slice * 8 + 4 * half) * 4);
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+            float2 sz[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sz[j] = __half22float2(*reinterpret_cast<const __half2 *>(&uw[j]));
+#pragma unroll
+            for (int g = 0; g < GQA; ++g) {
+                float Wt = st.W[g][0];
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) Wt += __shfl_xor_sync(0xffffffffu, Wt, m);
+                float a[4], ch[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float lo = st.o[g][j].x + st.o[g][j].y;
+                    const float hi = st.o[g][4 + j].x + st.o[g][4 + j].y;
+                    const float other = __shfl_xor_sync(0xffffffffu, half ? lo : hi, 16);
+                    a[j] = (half ? hi : lo) + other;
+                }
+                value_channels4<VBITS>(a, Wt, ch);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) st.of[g][j] = fmaf(sz[j].x, ch[j], fmaf(sz[j].y, Wt, st.of[g][j]));
+                st.W[g][0] = 0.0f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
+            }
+        }
+    }
     __syncwarp();
 }
 
@@ -677,16 +753,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
 }
 
 // Resident CTAs per SM the register budget targets: two, but one for the
-// generic variants (up to 8 value groups of W/Z per lane) and for bf16 caches
-// (whose 128-token stages take 66 KB each).
-constexpr int decode_min_blocks(int km, int vm, int gvc) {
-    return km == K_BF16 ? 1 : ((vm == V_TOKEN && gvc == 0) ? 1 : 2);
+// generic variants (runtime key group size, or up to 8 value groups of W/Z per
+// lane) and for bf16 caches (whose 128-token stages take 66 KB each).
+constexpr int decode_min_blocks(int km, int vm, int gkc, int gvc) {
+    return (km == K_BF16 || (km == K_TOKEN && gkc == 0) || (vm == V_TOKEN && gvc == 0)) ? 1 : 2;
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int GKC, int GVC>
-__global__ void __launch_bounds__(kThreads, decode_min_blocks(KM, VM, GVC))
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int GKC, int GVC, bool SINK>
+__global__ void __launch_bounds__(kThreads, decode_min_blocks(KM, VM, GKC, GVC))
 decode_splitk_kernel(const DecodeParams p) {
-    constexpr int NVG = (VM == V_BF16) ? 1 : (GVC ? kHeadDim / GVC : kMaxGroups);
+    constexpr int NVG = (VM != V_TOKEN) ? 1 : (GVC ? kHeadDim / GVC : kMaxGroups);
     constexpr int KBF = (KM == K_BF16) ? 16 : KBITS;  // key form of quantized tiles
     constexpr int TILE = (KM == K_BF16) ? kTileB : kTileQ;
     constexpr int TPW = TILE / kConsumerWarps;
@@ -700,8 +776,8 @@ decode_splitk_kernel(const DecodeParams p) {
     uint8_t *stages = smem;
     uint8_t *tail = smem + static_cast<size_t>(NS) * p.stage_bytes;
     float *qs = reinterpret_cast<float *>(tail);                    // [GQA][128]
-    float *qs_raw = qs + GQA * kHeadDim;                             // [GQA][128] unrotated (sinks)
-    float *coefs = qs_raw + GQA * kHeadDim;                          // [n_sets][CBUF], CTA-shared
+    float *qs_raw = qs + GQA * kHeadDim;                             // [GQA][128] unrotated (sinks only)
+    float *coefs = qs_raw + (SINK ? GQA * kHeadDim : 0);             // [n_sets][CBUF], CTA-shared
     float *scratch_all = coefs + p.n_sets * CBUF;                    // [4][warp_floats]
     uint64_t *full = reinterpret_cast<uint64_t *>(scratch_all + kConsumerWarps * p.warp_floats);
     uint64_t *empty = full + kMaxStages;
@@ -768,7 +844,7 @@ decode_splitk_kernel(const DecodeParams p) {
             int item = __shfl_sync(0xffffffffu, next, 0);
             if (lane == 0 && item < n_items) next = atomicAdd(p.counter, 1);
             int seq = 0, kvh = 0, split = 0;
-            int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0, n_sink = 0;
+            int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0, n_sink = 0, n_st = 0;
             if (item < n_items) {
                 item_coords(pref, p.S, p.H, item, seq, kvh, split);
                 const int T = lens[seq];
@@ -776,15 +852,17 @@ decode_splitk_kernel(const DecodeParams p) {
                 t_end = min(T, t_begin + p.chunk);
                 Tq = quantized_len(T, p.R);
                 q_end = min(t_end, Tq);
-                // sink positions [0, sink_len) are read from the sink rows, as the
-                // item's last tile (after the quantized ones, so the value sums
+                // sink positions [0, sink_len) are read from the sink rows, in
+                // window-sized tiles after the quantized ones (so the value sums
                 // are folded first)
-                n_qt = q_end > max(t_begin, p.sink_len) ? (q_end - t_begin + TILE - 1) / TILE : 0;
+                const int q_begin = SINK ? max(t_begin, p.sink_len) : t_begin;
+                n_qt = q_end > q_begin ? (q_end - t_begin + TILE - 1) / TILE : 0;
                 w_begin = max(t_begin, Tq);
                 n_wt = t_end > w_begin ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
-                n_sink = (split == 0 && p.sink_len > 0) ? min(p.sink_len, T) : 0;
+                n_sink = (SINK && split == 0 && p.sink_len > 0) ? min(p.sink_len, T) : 0;
+                n_st = (n_sink + p.bf_tile - 1) / p.bf_tile;
             }
-            const int n_tiles = (item < n_items) ? n_qt + n_wt + (n_sink > 0) : 1;  // 1 = the done marker
+            const int n_tiles = (item < n_items) ? n_qt + n_wt + n_st : 1;  // 1 = the done marker
             const int64_t sh = static_cast<int64_t>(seq) * p.H + kvh;
             for (int ti = 0; ti < n_tiles; ++ti, ++it) {
                 const int s = it % NS, r = it / NS;
@@ -808,17 +886,19 @@ decode_splitk_kernel(const DecodeParams p) {
                     break;
                 }
                 if (it == p.skip_tile) continue;  // test hook: never arrive
-                const bool sink = ti >= n_qt + n_wt;
+                const bool sink = SINK && ti >= n_qt + n_wt;
                 const bool window = ti >= n_qt;
-                const int t0 = sink ? 0 : (window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * TILE);
-                const int n = sink ? n_sink : (window ? min(p.bf_tile, t_end - t0) : min(TILE, q_end - t0));
+                const int t0 = sink ? (ti - n_qt - n_wt) * p.bf_tile
+                                    : (window ? w_begin + (ti - n_qt) * p.bf_tile : t_begin + ti * TILE);
+                const int n = sink ? min(p.bf_tile, n_sink - t0)
+                                   : (window ? min(p.bf_tile, t_end - t0) : min(TILE, q_end - t0));
                 if (lane == 0) {
                     hdr->seq = seq;
                     hdr->kvh = kvh;
                     hdr->split = split;
                     hdr->t0 = t0;
                     hdr->n = n;
-                    hdr->start = window ? 0 : max(0, p.sink_len - t0);
+                    hdr->start = (SINK && !window) ? max(0, p.sink_len - t0) : 0;
                     hdr->flags = (ti == 0 ? kFirst : 0) | (ti == n_tiles - 1 ? kLast : 0) |
                                  (window ? kWindow : 0) | (sink ? kSink : 0);
                 }
@@ -831,11 +911,11 @@ decode_splitk_kernel(const DecodeParams p) {
                 }
                 if (sink) {
                     const uint32_t bytes = n * kHeadDim * 2;
-                    const int64_t row = sh * p.sink_len;
+                    const int64_t row = sh * p.sink_len + t0;
                     if (lane < 2) {
                         mbar_expect_tx(bar, bytes);
                         if (lane == 0) bulk_g2s(st, p.k_sink + row * kHeadDim, bytes, bar);
-                        else bulk_g2s(st + p.sink_off_v, p.v_sink + row * kHeadDim, bytes, bar);
+                        else bulk_g2s(st + p.bf_off_v, p.v_sink + row * kHeadDim, bytes, bar);
                     }
                 } else if (window) {
                     const uint32_t bytes = n * kHeadDim * 2;
@@ -868,6 +948,11 @@ decode_splitk_kernel(const DecodeParams p) {
                         const uint32_t b = (n * ngv * 4 + 15) & ~15;
                         mbar_expect_tx(bar, b);
                         bulk_g2s(st + p.off_vsz, p.v_sz + row * ngv, b, bar);
+                    } else if (lane == 3 && VM == V_CHANNEL) {
+                        const int b0 = t0 / p.R, nb = (t0 + n - 1) / p.R - b0 + 1;
+                        mbar_expect_tx(bar, nb * kHeadDim * 4);
+                        bulk_g2s(st + p.off_vsz, p.v_sz + (sh * (p.cap / p.R) + b0) * kHeadDim,
+                                 nb * kHeadDim * 4, bar);
                     }
                 } else {
                     // Paged (token-wise groups only): one lane per page (or per
@@ -922,7 +1007,8 @@ decode_splitk_kernel(const DecodeParams p) {
     constexpr int RSTR = 132;
     const int slice = lane & 15;
 
-    WarpState<GQA, NVG> st;
+    constexpr bool VCH = VM == V_CHANNEL;
+    WarpState<GQA, NVG, VCH> st;
     bool folded = false;
     // Turn the value accumulators of quantized tiles into plain channel sums
     // (adding the zero-point terms), once: before the first bf16 window tile
@@ -1004,7 +1090,7 @@ decode_splitk_kernel(const DecodeParams p) {
                         }
                     }
                 }
-                if (p.sink_len > 0)
+                if (SINK)
                     *reinterpret_cast<float4 *>(qs_raw + warp * kHeadDim + 4 * lane) =
                         make_float4(x[0] * p.qscale, x[1] * p.qscale, x[2] * p.qscale, x[3] * p.qscale);
                 if (p.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
@@ -1045,6 +1131,10 @@ decode_splitk_kernel(const DecodeParams p) {
                 for (int v = 0; v < NVG; ++v) { st.W[g][v] = 0.0f; st.Z[g][v] = 0.0f; }
 #pragma unroll
                 for (int c = 0; c < 8; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
+                if constexpr (VCH) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) st.of[g][c] = 0.0f;
+                }
             }
             folded = false;
         }
@@ -1072,32 +1162,44 @@ decode_splitk_kernel(const DecodeParams p) {
                 coef = sets + min((warp * TPW) / p.R, nbt - 1) * CBUF;
             }
             constexpr int GKC_T = (KM == K_TOKEN) ? GKC : kHeadDim;
-            if (hdr.n == TILE && hdr.start == 0)
-                process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, true>(
-                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, 0, coef, QHSTR, RG::cstr,
+            // per-channel values: this warp's block among the tile's staged ones
+            const uint8_t *vsz = sb + p.off_vsz;
+            if constexpr (VM == V_CHANNEL)
+                vsz += ((hdr.t0 + warp * TPW) / p.R - hdr.t0 / p.R) * kHeadDim * 4;
+            if (hdr.n == TILE && (!SINK || hdr.start == 0))
+                process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, true, SINK>(
+                    sb, sb + p.off_ksz, sb + p.off_vc, vsz, hdr.n, 0, coef, QHSTR, RG::cstr,
                     coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
             else
-                process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, false>(
-                    sb, sb + p.off_ksz, sb + p.off_vc, sb + p.off_vsz, hdr.n, hdr.start, coef, QHSTR,
+                process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, false, SINK>(
+                    sb, sb + p.off_ksz, sb + p.off_vc, vsz, hdr.n, SINK ? hdr.start : 0, coef, QHSTR,
                     RG::cstr, coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
         } else if constexpr (KM != K_BF16) {
             if (!folded) {  // first window tile of the item
                 if (VM == V_TOKEN) fold_values();
                 folded = true;
             }
-            if (hdr.flags & kSink)  // bf16 sink keys against the unrotated query rows
-                process_tile<GQA, K_BF16, V_BF16, 16, 16, kSinkTile / kConsumerWarps, kHeadDim, 0, NVG, false>(
-                    sb, nullptr, sb + p.sink_off_v, nullptr, hdr.n, 0, qs_raw, kHeadDim, 8, nullptr, p.gk,
-                    p.gv, st, wsm, warp, lane);
-            else  // bf16 window keys against the query rows (coefficients = q)
-                process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, kHeadDim, 0, NVG, false>(
-                    sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, 0, qs, kHeadDim, 8, nullptr, p.gk, p.gv, st,
-                    wsm, warp, lane);
+            // bf16 window keys against the query rows (coefficients = q), or
+            // sink keys against the unrotated ones (one code path for both)
+            const float *qrows = (SINK && (hdr.flags & kSink)) ? qs_raw : qs;
+            process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, kHeadDim, 0, NVG, false, false>(
+                sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, 0, qrows, kHeadDim, 8, nullptr, p.gk, p.gv, st,
+                wsm, warp, lane);
         }
 
         if (hdr.flags & kLast) {
             // ---- item epilogue: merge the four warps, write the partial ----
             if (VM == V_TOKEN && !folded) fold_values();
+            if constexpr (VM == V_CHANNEL) {  // the folded sums join the window's
+                const bool hi = lane >= 16;
+#pragma unroll
+                for (int g = 0; g < GQA; ++g)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        st.o[g][j].x += hi ? 0.0f : st.of[g][j];
+                        st.o[g][4 + j].x += hi ? st.of[g][j] : 0.0f;
+                    }
+            }
             __syncwarp();
 #pragma unroll
             for (int g = 0; g < GQA; ++g) {
@@ -1205,15 +1307,15 @@ StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
         const int vrow = 128 * d.bits_v / 8;
         const int ksz = (d.axis_k == KVQ_PER_CHANNEL) ? (kTileQ / d.residual_len) * 128 * 4
                                                       : kTileQ * (128 / d.group_k) * 4;
-        const int vsz = kTileQ * (128 / d.group_v) * 4;
+        const int vsz = (d.axis_v == KVQ_PER_CHANNEL) ? (kTileQ / d.residual_len) * 128 * 4
+                                                      : kTileQ * (128 / d.group_v) * 4;
         L.off_ksz = round16(kTileQ * krow);
         L.off_vc = L.off_ksz + round16(ksz);
         L.off_vsz = L.off_vc + round16(kTileQ * vrow);
         data = L.off_vsz + round16(vsz);
         L.bf_tile = kWinTile;
         L.bf_off_v = kWinTile * 256;
-        if (d.residual_len > 0) data = std::max(data, 2 * kWinTile * 256);
-        if (d.sink_len > 0) data = std::max(data, 2 * d.sink_len * 256);
+        if (d.residual_len > 0 || d.sink_len > 0) data = std::max(data, 2 * kWinTile * 256);
     }
     L.off_q = round16(data);
     L.off_hdr = L.off_q + round16(gqa * kHeadDim * q_bytes);
@@ -1243,26 +1345,27 @@ int sm_count() {
     return n;
 }
 
-template <int GQA, int KM, int VM, int KBITS, int VBITS, int GKC, int GVC>
+template <int GQA, int KM, int VM, int KBITS, int VBITS, int GKC, int GVC, bool SINK = false>
 kvq_status launch_variant(DecodeParams p, int max_items, cudaStream_t stream) {
     constexpr int KBF = (KM == K_BF16) ? 16 : KBITS;
     constexpr int nch = RowGeo<KBF>::nch;
     constexpr int cbuf = GQA * nch * RowGeo<KBF>::cstr + kMaxGroups * GQA * 2;
-    const int n_vg = (VM == V_BF16) ? 1 : kHeadDim / p.gv;
+    const int n_vg = (VM != V_TOKEN) ? 1 : kHeadDim / p.gv;
     const ScratchLayout SL = scratch_layout(GQA, n_vg);
     p.warp_floats = SL.floats;
     p.off_tot = SL.off_tot;
     p.n_sets = (KM == K_CHANNEL) ? 2 * (kTileQ / p.R) : 1;
-    const size_t tail = sizeof(float) * (2 * static_cast<size_t>(GQA) * kHeadDim + static_cast<size_t>(p.n_sets) * cbuf +
+    const size_t q_rows = (SINK ? 2 : 1) * static_cast<size_t>(GQA) * kHeadDim;  // rotated (+ unrotated)
+    const size_t tail = sizeof(float) * (q_rows + static_cast<size_t>(p.n_sets) * cbuf +
                                          kConsumerWarps * static_cast<size_t>(p.warp_floats)) +
                         sizeof(uint64_t) * 2 * kMaxStages + 16 + sizeof(int) * (2 * p.S + 1);
     // Ring depth: as many stages (2..4) as let the targeted CTAs per SM fit.
-    const int per_sm_target = decode_min_blocks(KM, VM, GVC);
+    const int per_sm_target = decode_min_blocks(KM, VM, GKC, GVC);
     const size_t budget = (232448 - 1024 * per_sm_target) / per_sm_target;
     int ns = static_cast<int>(std::min<size_t>(kMaxStages, (budget > tail ? budget - tail : 0) / p.stage_bytes));
     p.ns = std::max(2, ns);
     const size_t smem = static_cast<size_t>(p.ns) * p.stage_bytes + tail;
-    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, GKC, GVC>;
+    auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, GKC, GVC, SINK>;
     if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;  // too many sequences for one launch
     // The shared-memory opt-in and the occupancy query cost host time on every
     // call; redo them only when this variant's size changes (per device).
@@ -1300,6 +1403,16 @@ kvq_status launch_variant(DecodeParams p, int max_items, cudaStream_t stream) {
 template <int GQA, int KM, int VM, int KBITS, int VBITS>
 kvq_status launch_groups(const kvq_cache_desc &d, const DecodeParams &p, int max_items,
                          cudaStream_t stream) {
+    if constexpr (KM == K_TOKEN && VM == V_TOKEN) {
+        // attention-sink caches: their own instantiations (the sink start
+        // offset and the unrotated query rows), the llama-shaped INT4 one fast
+        if (p.sink_len > 0) {
+            if constexpr (GQA == 4 && KBITS == 4 && VBITS == 4)
+                if (d.group_k == 128 && d.group_v == 128)
+                    return launch_variant<GQA, KM, VM, KBITS, VBITS, 128, 128, true>(p, max_items, stream);
+            return launch_variant<GQA, KM, VM, KBITS, VBITS, 0, 0, true>(p, max_items, stream);
+        }
+    }
     if constexpr (GQA == 4 && VM == V_TOKEN && KM == K_TOKEN && KBITS == 4 && VBITS == 4) {
         if (d.group_k == 128 && d.group_v == 128)  // llama-shaped INT4 caches
             return launch_variant<GQA, KM, VM, KBITS, VBITS, 128, 128>(p, max_items, stream);
@@ -1318,6 +1431,18 @@ kvq_status dispatch_modes(const kvq_cache_desc &d, const DecodeParams &p, int ma
                           cudaStream_t stream) {
     if (d.bits_k == 16 && d.bits_v == 16)
         return launch_variant<GQA, K_BF16, V_BF16, 16, 16, 0, 0>(p, max_items, stream);
+    if (d.axis_v == KVQ_PER_CHANNEL) {  // bits_k == bits_v (validated)
+        if (d.axis_k == KVQ_PER_CHANNEL) {
+            if (d.bits_v == 2) return launch_variant<GQA, K_CHANNEL, V_CHANNEL, 2, 2, 0, 0>(p, max_items, stream);
+            return launch_variant<GQA, K_CHANNEL, V_CHANNEL, 4, 4, 0, 0>(p, max_items, stream);
+        }
+        if (d.group_k == 128) {
+            if (d.bits_v == 2) return launch_variant<GQA, K_TOKEN, V_CHANNEL, 2, 2, 128, 0>(p, max_items, stream);
+            return launch_variant<GQA, K_TOKEN, V_CHANNEL, 4, 4, 128, 0>(p, max_items, stream);
+        }
+        if (d.bits_v == 2) return launch_variant<GQA, K_TOKEN, V_CHANNEL, 2, 2, 0, 0>(p, max_items, stream);
+        return launch_variant<GQA, K_TOKEN, V_CHANNEL, 4, 4, 0, 0>(p, max_items, stream);
+    }
     if (d.axis_k == KVQ_PER_CHANNEL) {
         if (d.bits_k == 2 && d.bits_v == 2) return launch_groups<GQA, K_CHANNEL, V_TOKEN, 2, 2>(d, p, max_items, stream);
         if (d.bits_k == 4 && d.bits_v == 4) return launch_groups<GQA, K_CHANNEL, V_TOKEN, 4, 4>(d, p, max_items, stream);
@@ -1372,7 +1497,6 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.k_sink = static_cast<const uint16_t *>(d.k_sink);
     p.v_sink = static_cast<const uint16_t *>(d.v_sink);
     p.sink_len = d.sink_len;
-    p.sink_off_v = d.sink_len * kHeadDim * 2;
     p.o_part = static_cast<float *>(workspace);
     p.ml = reinterpret_cast<float2 *>(static_cast<uint8_t *>(workspace) + plan.ws_part);
     p.counter = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + plan.ws_part + plan.ws_ml);
@@ -1381,7 +1505,7 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.H = d.num_kv_heads;
     p.Hq = num_q_heads;
     p.gk = (d.bits_k == 16 || d.axis_k == KVQ_PER_CHANNEL) ? kHeadDim : d.group_k;
-    p.gv = (d.bits_v == 16) ? kHeadDim : d.group_v;
+    p.gv = (d.bits_v == 16 || d.axis_v == KVQ_PER_CHANNEL) ? kHeadDim : d.group_v;
     p.hb = d.hadamard_block_k;
     p.hscale = hadamard_scale(d.hadamard_block_k);
     p.qscale = softmax_scale * kLog2e;

@@ -94,6 +94,12 @@ typedef enum {
  *   bits 2 or 4, per-channel key groups (axis_k KVQ_PER_CHANNEL, contiguous only,
  *   requires residual_len == group_k, a multiple of 64):
  *     codes u8 [S][H][Tc][row] (packed along channels)  sz half2 [S][H][Tc/G][D]
+ *   bits 2 or 4, per-channel value groups (axis_v KVQ_PER_CHANNEL): the same
+ *   layout for V, with residual_len == group_v and bits_v == bits_k. InnerQ
+ *   ("InnerQ: Hardware-Aware Tuning-Free Quantization of KV Cache for Large
+ *   Language Models", Abstract) groups each cache matrix along the inner
+ *   dimension of its product with the attention vector: channels for q.K^T,
+ *   tokens for p.V, so V's groups are one channel over an R-token block.
  *   bits 16 (unquantized bf16, contiguous only):
  *     codes bf16 [S][H][Tc][D]; sz unused (may be NULL).
  *   Packing: INT4 element 2i in the low nibble of byte i, 2i+1 in the high
@@ -118,7 +124,7 @@ typedef struct {
     int32_t head_dim;          /* D, must be 128 */
     int32_t bits_k, bits_v;    /* 2, 4 or 16 */
     int32_t group_k, group_v;  /* group sizes (ignored for bits 16) */
-    int32_t axis_k, axis_v;    /* kvq_axis; axis_v must be KVQ_PER_TOKEN */
+    int32_t axis_k, axis_v;    /* kvq_axis of the key and value groups */
     int32_t hadamard_block_k;  /* 0 or power of two <= D */
     int32_t residual_len;      /* 0 or R (bf16 window length) */
     int32_t paged;             /* 0 contiguous, 1 paged */

@@ -68,7 +68,14 @@ def test_append_validation(K):
     assert _append(K, _desc(K, hadamard_signs=FAKE + 4)) == E
     assert _append(K, _desc(K), dtype=7) == E
     assert _append(K, _desc(K), v_new=None) == E          # V cache but no V input
-    assert _append(K, _desc(K, axis_v=1)) == U
+    # values grouped along tokens: per channel over the window's blocks only
+    assert _append(K, _desc(K, axis_v=2)) == E
+    assert _append(K, _desc(K, axis_v=1)) == U                               # rotation
+    assert _append(K, _desc(K, axis_v=1, hadamard_block_k=0)) == E           # no window
+    chan_v = dict(axis_v=1, bits_k=2, bits_v=2, group_k=128, group_v=128, hadamard_block_k=0,
+                  residual_len=128, k_res=FAKE, v_res=FAKE)
+    assert _append(K, _desc(K, **dict(chan_v, group_v=64))) == E             # group != window
+    assert _append(K, _desc(K, **dict(chan_v, bits_v=4))) == U               # mixed widths
     # per-channel keys need the residual window and a contiguous cache
     assert _append(K, _desc(K, axis_k=1, hadamard_block_k=0, residual_len=0)) == E
     assert _append(K, _desc(K, axis_k=1, hadamard_block_k=0, residual_len=128, paged=1,
