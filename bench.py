@@ -54,7 +54,9 @@ def flush_l2(buf):
     kernel's reads would pay for)."""
     buf.zero_()
     buf.amax()
-DECODE_SRC = os.path.join(ROOT, "bit_kv_cache_21_b200", "csrc", "kvq_decode.cu")
+# the timed split-K variant: the kernel template and the unit that instantiates it
+DECODE_SRC = [os.path.join(ROOT, "bit_kv_cache_21_b200", "csrc", f)
+              for f in ("kvq_decode_kernel.cuh", "kvq_decode_plain.cu")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_splitk_llama8b_traffic.json")
 
 
@@ -78,9 +80,12 @@ def tensor_peaks():
         return 1590.0, 1400.0, "fallback"
 
 
-def source_hash(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_hash(paths):
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_per_launch():
