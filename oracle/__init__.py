@@ -68,10 +68,11 @@ def _declare(l):
         "oracle_fwht_f64": (None, [_P, _I]),
         "oracle_rotate_blocks_f64": (None, [_P, _L, _I, _I]),
         "oracle_quantize_group": (None, [_P, _I, _I, _I, _P, _P, _P, _I]),
+        "oracle_quantize_group_hybrid": (None, [_P, _I, _I, _I, _P, _P, _P, _I]),
         "oracle_pack_codes": (None, [_P, _I, _I, _P]),
         "oracle_unpack_codes": (None, [_P, _I, _I, _P]),
-        "oracle_quantize_tokens": (None, [_P, _L, _I, _I, _I, _I, _P, _P]),
-        "oracle_quantize_channel_block": (None, [_P, _I, _I, _I, _P, _P]),
+        "oracle_quantize_tokens": (None, [_P, _L, _I, _I, _I, _I, _I, _P, _P]),
+        "oracle_quantize_channel_block": (None, [_P, _I, _I, _I, _I, _P, _P]),
         "oracle_dequant_tokens": (None, [_P, _P, _L, _I, _I, _I, _P]),
         "oracle_dequant_channel_block": (None, [_P, _P, _I, _I, _I, _P]),
         "oracle_attention": (None, [_P, _I, _P, _P, _L, _I, _D, _P]),
@@ -162,6 +163,21 @@ def quantize_group(x, bits):
     return int(s[0]), int(z[0]), q
 
 
+def quantize_group_hybrid(x, bits):
+    """One group with InnerQ's hybrid choice (Abstract, "(i) hybrid
+    quantization"): the asymmetric min/max candidate or a symmetric one with
+    an exact zero level, whichever reconstructs the group with the smaller
+    squared error (the criterion is this library's reading; oracle.c states
+    it). Returns (s_bits, z_bits, codes)."""
+    a = _c(x, np.float32)
+    s = np.zeros(1, np.uint16)
+    z = np.zeros(1, np.uint16)
+    q = np.zeros(a.size, np.uint8)
+    lib().oracle_quantize_group_hybrid(_ptr(a), a.size, 1, bits, _ptr(s), _ptr(z),
+                                       _ptr(q), 1)
+    return int(s[0]), int(z[0]), q
+
+
 def pack_codes(q, bits):
     q = _c(q, np.uint8)
     out = np.zeros(q.size * bits // 8, np.uint8)
@@ -187,13 +203,14 @@ def apply_signs(x, signs):
     return x * np.asarray(signs, x.dtype)
 
 
-def quantize_tokens(x, hb, G, bits, signs=None):
+def quantize_tokens(x, hb, G, bits, signs=None, hybrid=False):
     """Token-wise group quantization (SAW-INT4 Abstract "token-wise INT4";
     InnerQ Abstract groups along the inner dimension of q.k).
 
     x: float32 [..., D] (bf16 or fp32 values). Each vector is multiplied by
     the random signs (if given), rotated (hb > 0) and split into D/G groups of
-    G consecutive elements.
+    G consecutive elements. hybrid: each group takes the symmetric or the
+    asymmetric candidate (quantize_group_hybrid).
     Returns codes uint8 [..., D*bits/8] and sz uint16 [..., D/G, 2] holding
     the fp16 bit patterns (scale, zero)."""
     a = _c(apply_signs(_c(x, np.float32), signs), np.float32)
@@ -201,11 +218,11 @@ def quantize_tokens(x, hb, G, bits, signs=None):
     n = a.size // D
     codes = np.zeros(a.shape[:-1] + (D * bits // 8,), np.uint8)
     sz = np.zeros(a.shape[:-1] + (D // G, 2), np.uint16)
-    lib().oracle_quantize_tokens(_ptr(a), n, D, hb, G, bits, _ptr(codes), _ptr(sz))
+    lib().oracle_quantize_tokens(_ptr(a), n, D, hb, G, bits, int(hybrid), _ptr(codes), _ptr(sz))
     return codes, sz
 
 
-def quantize_channel_block(x, bits):
+def quantize_channel_block(x, bits, hybrid=False):
     """Channel-wise quantization of one block of R tokens (KIVI keys): each
     channel's R values are one group. x: float32 [R][D].
     Returns codes uint8 [R][D*bits/8] and sz uint16 [D][2]."""
@@ -213,7 +230,7 @@ def quantize_channel_block(x, bits):
     R, D = a.shape
     codes = np.zeros((R, D * bits // 8), np.uint8)
     sz = np.zeros((D, 2), np.uint16)
-    lib().oracle_quantize_channel_block(_ptr(a), R, D, bits, _ptr(codes), _ptr(sz))
+    lib().oracle_quantize_channel_block(_ptr(a), R, D, bits, int(hybrid), _ptr(codes), _ptr(sz))
     return codes, sz
 
 

@@ -301,6 +301,92 @@ void oracle_quantize_group(const float *x, int n, int stride, int bits,
     }
 }
 
+/* Hybrid symmetric/asymmetric choice per group [INQ] "(i) hybrid
+ * quantization ... based on local statistics". The page states no criterion;
+ * this reading takes the candidate with the smaller squared reconstruction
+ * error of the group, ties to the asymmetric one:
+ *   asymmetric: the recipe of oracle_quantize_group above;
+ *   symmetric:  a grid with an exact zero level. Qp = 2^(bits-1) - 1,
+ *     C = 2^(bits-1), m = max(|min|, |max|) (zero extremes as +0),
+ *     s = fp16 rounded toward +inf of fp32(m / Qp), z = -C * s (exact; the
+ *     candidate is dropped when |z| > 65504, the largest fp16),
+ *     s == 0 -> every code is C, else r = fp32(1 / s),
+ *     q = clamp(rint_even(fp32(x * r)), -Qp, Qp) + C.
+ *   Both candidates store (s, z) as fp16 and dequantize as q * s + z, so the
+ *   choice is invisible to the readers of the cache.
+ *   Error of a candidate: e = fp32(x - fma(q, s, z)) per element, squares
+ *   summed with fma in element order over consecutive runs of 32 elements
+ *   (a group of 16 is one run), run sums then added pairwise
+ *   ((r0 + r1) + (r2 + r3)) ...; symmetric iff its sum is smaller. */
+static float run_tree_sse(const float *x, int n, int stride, const uint8_t *q,
+                          int q_stride, float s, float z)
+{
+    float runs[64];
+    int n_runs = 0;
+    for (int r0 = 0; r0 < n; r0 += 32) {
+        int len = (n - r0 < 32) ? n - r0 : 32;
+        float acc = 0.0f;
+        for (int i = r0; i < r0 + len; ++i) {
+            float xh = fmaf((float)q[(int64_t)i * q_stride], s, z);
+            float e = x[(int64_t)i * stride] - xh;
+            acc = fmaf(e, e, acc);
+        }
+        runs[n_runs++] = acc;
+    }
+    for (int w = 1; w < n_runs; w *= 2)
+        for (int i = 0; i + w < n_runs; i += 2 * w)
+            runs[i] = runs[i] + runs[i + w];
+    return runs[0];
+}
+
+void oracle_quantize_group_hybrid(const float *x, int n, int stride, int bits,
+                                  uint16_t *s_out, uint16_t *z_out,
+                                  uint8_t *q_out, int q_stride)
+{
+    uint16_t sa, za;
+    oracle_quantize_group(x, n, stride, bits, &sa, &za, q_out, q_stride);
+    *s_out = sa;
+    *z_out = za;
+    const int C = 1 << (bits - 1), Qp = C - 1;
+    float mn = x[0], mx = x[0];
+    for (int i = 1; i < n; ++i) {
+        float v = x[(int64_t)i * stride];
+        if (v < mn)
+            mn = v;
+        if (v > mx)
+            mx = v;
+    }
+    mn = mn + 0.0f;
+    mx = mx + 0.0f;
+    float m = fabsf(mn) > fabsf(mx) ? fabsf(mn) : fabsf(mx);
+    uint16_t sb = oracle_f32_to_f16(m / (float)Qp, ORACLE_RU);
+    float ss = oracle_f16_to_f32(sb);
+    float zs = -(float)C * ss;
+    if (!(fabsf(zs) <= 65504.0f))
+        return;
+    uint16_t zb = oracle_f32_to_f16(zs, ORACLE_RN);
+    uint8_t *qs = (uint8_t *)calloc((size_t)n, 1);
+    float r = (ss == 0.0f) ? 0.0f : 1.0f / ss;
+    for (int i = 0; i < n; ++i) {
+        float t = rintf(x[(int64_t)i * stride] * r);
+        if (t < -(float)Qp)
+            t = -(float)Qp;
+        if (t > (float)Qp)
+            t = (float)Qp;
+        qs[i] = (uint8_t)(int)(t + (float)C);
+    }
+    float ea = run_tree_sse(x, n, stride, q_out, q_stride, oracle_f16_to_f32(sa),
+                            oracle_f16_to_f32(za));
+    float es = run_tree_sse(x, n, stride, qs, 1, ss, zs);
+    if (es < ea) {
+        *s_out = sb;
+        *z_out = zb;
+        for (int i = 0; i < n; ++i)
+            q_out[(int64_t)i * q_stride] = qs[i];
+    }
+    free(qs);
+}
+
 /* Packing: INT4 puts element 2i in the low nibble of byte i and 2i+1 in the
  * high nibble; INT2 puts element 4i+j in bits 2j..2j+1 of byte i. */
 void oracle_pack_codes(const uint8_t *q, int n, int bits, uint8_t *out)
@@ -327,7 +413,8 @@ void oracle_unpack_codes(const uint8_t *packed, int n, int bits, uint8_t *q)
  * elements along D. codes: [n_vec][D*bits/8], sz: [n_vec][D/G][2] holding
  * the fp16 bit patterns (scale, zero). */
 void oracle_quantize_tokens(const float *x, int64_t n_vec, int D, int hb,
-                            int G, int bits, uint8_t *codes, uint16_t *sz)
+                            int G, int bits, int hybrid, uint8_t *codes,
+                            uint16_t *sz)
 {
     float *tmp = (float *)malloc(sizeof(float) * D);
     uint8_t *q = (uint8_t *)malloc(D);
@@ -339,8 +426,8 @@ void oracle_quantize_tokens(const float *x, int64_t n_vec, int D, int hb,
             oracle_rotate_blocks_f32(tmp, 1, D, hb);
         for (int g = 0; g < ng; ++g) {
             uint16_t *p = sz + (v * ng + g) * 2;
-            oracle_quantize_group(tmp + g * G, G, 1, bits, &p[0], &p[1],
-                                  q + g * G, 1);
+            (hybrid ? oracle_quantize_group_hybrid : oracle_quantize_group)(
+                tmp + g * G, G, 1, bits, &p[0], &p[1], q + g * G, 1);
         }
         oracle_pack_codes(q, D, bits, codes + v * row_bytes);
     }
@@ -352,12 +439,12 @@ void oracle_quantize_tokens(const float *x, int64_t n_vec, int D, int hb,
  * keys): each channel's R values form one group. codes: [R][D*bits/8] packed
  * along channels within each token; sz: [D][2]. */
 void oracle_quantize_channel_block(const float *x, int R, int D, int bits,
-                                   uint8_t *codes, uint16_t *sz)
+                                   int hybrid, uint8_t *codes, uint16_t *sz)
 {
     uint8_t *q = (uint8_t *)malloc((size_t)R * D);
     for (int d = 0; d < D; ++d)
-        oracle_quantize_group(x + d, R, D, bits, &sz[2 * d], &sz[2 * d + 1],
-                              q + d, D);
+        (hybrid ? oracle_quantize_group_hybrid : oracle_quantize_group)(
+            x + d, R, D, bits, &sz[2 * d], &sz[2 * d + 1], q + d, D);
     int row_bytes = D * bits / 8;
     for (int t = 0; t < R; ++t)
         oracle_pack_codes(q + (int64_t)t * D, D, bits, codes + (int64_t)t * row_bytes);

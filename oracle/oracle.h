@@ -27,12 +27,16 @@ void oracle_rotate_blocks_f64(double *x, int64_t n_vec, int D, int hb);
 void oracle_quantize_group(const float *x, int n, int stride, int bits,
                            uint16_t *s_out, uint16_t *z_out, uint8_t *q_out,
                            int q_stride);
+void oracle_quantize_group_hybrid(const float *x, int n, int stride, int bits,
+                                  uint16_t *s_out, uint16_t *z_out,
+                                  uint8_t *q_out, int q_stride);
 void oracle_pack_codes(const uint8_t *q, int n, int bits, uint8_t *out);
 void oracle_unpack_codes(const uint8_t *packed, int n, int bits, uint8_t *q);
 void oracle_quantize_tokens(const float *x, int64_t n_vec, int D, int hb,
-                            int G, int bits, uint8_t *codes, uint16_t *sz);
+                            int G, int bits, int hybrid, uint8_t *codes,
+                            uint16_t *sz);
 void oracle_quantize_channel_block(const float *x, int R, int D, int bits,
-                                   uint8_t *codes, uint16_t *sz);
+                                   int hybrid, uint8_t *codes, uint16_t *sz);
 void oracle_dequant_tokens(const uint8_t *codes, const uint16_t *sz,
                            int64_t n_vec, int D, int G, int bits, double *out);
 void oracle_dequant_channel_block(const uint8_t *codes, const uint16_t *sz,

@@ -521,3 +521,80 @@ def test_sink_attention_equals_attention_over_the_concatenated_tokens():
     ks2[:, 1, 0] = 1e4
     got = oracle.decode_attention_gqa_sinks(q2, kq, vq, ks2, vs, 1.0)
     assert np.allclose(got[0], vs[0, 1]) and np.allclose(got[-1], vs[1, 1])
+
+
+# ---------------------------------------------------------------------------
+# Hybrid symmetric/asymmetric choice per group (InnerQ Abstract, "(i)")
+# ---------------------------------------------------------------------------
+
+def test_hybrid_golden_worked_examples():
+    with open(os.path.join(GOLDEN, "hybrid_sym_asym.txt")) as f:
+        lines = [l for l in f if l.strip() and not l.startswith("#")]
+    assert len(lines) == 4
+    for line in lines:
+        bits, x, sz, q = (part.split() for part in line.split(";"))
+        s, z, codes = oracle.quantize_group_hybrid(np.array([float(t) for t in x], np.float32), int(bits[0]))
+        assert (s, z) == (int(sz[0], 16), int(sz[1], 16)), line
+        assert codes.tolist() == [int(t) for t in q], line
+
+
+def _sym_candidate(x, bits):
+    # the symmetric grid written out independently: s = fp16_ru(max|x| / Qp),
+    # z = -C s, q = clamp(rint(x / s), -Qp, Qp) + C
+    C = 1 << (bits - 1)
+    Qp = C - 1
+    m = np.float32(max(abs(float(x.min())), abs(float(x.max()))))
+    s_bits = int(oracle.f32_to_f16_bits(np.array([m / np.float32(Qp)], np.float32), oracle.ROUND_UP)[0])
+    s = float(oracle.f16_bits_to_f64(np.array([s_bits], np.uint16))[0])
+    if s == 0.0:
+        return s_bits, None, np.full(x.size, C, np.uint8)
+    r = np.float32(1.0) / np.float32(s)
+    q = np.clip(np.rint(x.astype(np.float32) * r), -Qp, Qp) + C
+    z_bits = int(oracle.f32_to_f16_bits(np.array([-C * s], np.float32))[0])
+    return s_bits, z_bits, q.astype(np.uint8)
+
+
+def _sse(x, s_bits, z_bits, q):
+    s, z = oracle.f16_bits_to_f64(np.array([s_bits, z_bits], np.uint16))
+    return float(np.sum((x.astype(np.float64) - (q * s + z)) ** 2))
+
+
+def test_hybrid_takes_one_candidate_and_the_better_one():
+    g = np.random.default_rng(31)
+    picked_sym = 0
+    for trial in range(600):
+        n = (16, 32, 64, 128)[trial % 4]
+        bits = (2, 4)[(trial // 4) % 2]
+        x = (g.standard_t(2, n) if trial % 3 else g.standard_normal(n)).astype(np.float32)
+        s, z, q = oracle.quantize_group_hybrid(x, bits)
+        sa, za, qa = oracle.quantize_group(x, bits)
+        ss, zs, qs = _sym_candidate(x, bits)
+        if (s, z) == (sa, za) and np.array_equal(q, qa):
+            if zs is not None:  # kept the asymmetric one: not worse (float64, fp32 decision slack)
+                assert _sse(x, sa, za, qa) <= _sse(x, ss, zs, qs) * (1 + 1e-5) + 1e-12
+        else:
+            picked_sym += 1
+            assert (s, z) == (ss, zs) and np.array_equal(q, qs)
+            assert _sse(x, ss, zs, qs) <= _sse(x, sa, za, qa) * (1 + 1e-5) + 1e-12
+            # the symmetric grid has an exact zero level
+            sf, zf = oracle.f16_bits_to_f64(np.array([s, z], np.uint16))
+            assert np.all((q * sf + zf)[x == 0] == 0)
+    assert 20 < picked_sym < 580  # both candidates occur on these heavy-tailed groups
+
+
+def test_hybrid_applies_per_group_in_token_and_channel_layouts():
+    g = np.random.default_rng(32)
+    x = g.standard_t(2, (3, 128)).astype(np.float32)
+    for G, bits in ((16, 2), (32, 4), (128, 2)):
+        codes, sz = oracle.quantize_tokens(x, 0, G, bits, hybrid=True)
+        for v in range(3):
+            q = oracle.unpack_codes(codes[v], 128, bits)
+            for grp in range(128 // G):
+                s, z, qg = oracle.quantize_group_hybrid(x[v, grp * G:(grp + 1) * G], bits)
+                assert (s, z) == tuple(sz[v, grp]) and np.array_equal(q[grp * G:(grp + 1) * G], qg)
+    blk = g.standard_t(2, (64, 128)).astype(np.float32)
+    codes, sz = oracle.quantize_channel_block(blk, 2, hybrid=True)
+    q = np.stack([oracle.unpack_codes(codes[t], 128, 2) for t in range(64)])
+    for d in (0, 5, 127):
+        s, z, qg = oracle.quantize_group_hybrid(np.ascontiguousarray(blk[:, d]), 2)
+        assert (s, z) == tuple(sz[d]) and np.array_equal(q[:, d], qg)
