@@ -64,7 +64,7 @@ class CacheDesc(ctypes.Structure):
         ("k_sink", ctypes.c_void_p),
         ("v_sink", ctypes.c_void_p),
         ("sink_len", ctypes.c_int32),
-        ("reserved2", ctypes.c_int32),
+        ("hybrid", ctypes.c_int32),
     ]
 
 

@@ -32,6 +32,7 @@ class CacheSpec:
     with_v: bool = True
     hadamard_signs: object = None  # device float32 [128] of +-1 (randomized Hadamard), or None
     sink_len: int = 0              # attention-sink tokens kept in bf16
+    hybrid: bool = False           # per-group symmetric/asymmetric choice
 
 
 def _row_bytes(bits: int) -> int:
@@ -99,7 +100,8 @@ class KVCache:
             k_codes=p(self.k_codes), v_codes=p(self.v_codes), k_sz=p(self.k_sz), v_sz=p(self.v_sz),
             k_res=p(self.k_res), v_res=p(self.v_res), block_table=p(self.block_table),
             status=p(self.status), hadamard_signs=p(s.hadamard_signs),
-            k_sink=p(self.k_sink), v_sink=p(self.v_sink), sink_len=s.sink_len, reserved2=0)
+            k_sink=p(self.k_sink), v_sink=p(self.v_sink), sink_len=s.sink_len,
+            hybrid=int(s.hybrid))
 
     def device_status(self) -> int:
         return int(self.status[0].item())

@@ -75,7 +75,7 @@ kvq_status validate_desc(const kvq_cache_desc *d, bool need_v) {
     if (d->status != nullptr && (reinterpret_cast<uintptr_t>(d->status) & 3u)) return KVQ_ERR_INVALID_ARG;
     if (d->hadamard_signs != nullptr && (d->hadamard_block_k == 0 || !aligned16(d->hadamard_signs)))
         return KVQ_ERR_INVALID_ARG;
-    if (d->reserved2 != 0 || d->sink_len < 0 || d->sink_len > 64) return KVQ_ERR_INVALID_ARG;
+    if ((d->hybrid != 0 && d->hybrid != 1) || d->sink_len < 0 || d->sink_len > 64) return KVQ_ERR_INVALID_ARG;
     if (d->sink_len > 0) {
         if (!need_v || bf16_k || d->axis_k != KVQ_PER_TOKEN || d->residual_len != 0) return KVQ_ERR_UNSUPPORTED;
         if (d->k_sink == nullptr || d->v_sink == nullptr || !aligned16(d->k_sink) || !aligned16(d->v_sink))

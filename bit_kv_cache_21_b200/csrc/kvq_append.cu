@@ -170,6 +170,7 @@ __device__ __forceinline__ void fwht_lane(float x[32], int hb, int part, float c
 
 struct QParams {
     __half2 sz;   // {scale, zero}
+    float sf;     // scale as fp32
     float zf;     // zero as fp32
     float r;      // fp32(1/scale), 0 when scale == 0
 };
@@ -185,6 +186,7 @@ __device__ __forceinline__ QParams qparams(float mn, float mx, int L) {
     const float sf = __half2float(s);
     QParams p;
     p.sz = __halves2half2(s, z);
+    p.sf = sf;
     p.zf = zf;
     p.r = (sf == 0.0f) ? 0.0f : __frcp_rn(sf);
     return p;
@@ -195,6 +197,47 @@ __device__ __forceinline__ uint32_t qcode(float x, const QParams &p, float Lf) {
     const float t = __fmul_rn(__fsub_rn(x, p.zf), p.r);
     const float q = fminf(fmaxf(rintf(t), 0.0f), Lf);
     return static_cast<uint32_t>(q);
+}
+
+// ---- hybrid symmetric/asymmetric choice (InnerQ, Abstract, "(i)") ---------
+// The symmetric candidate: Qp = 2^(bits-1) - 1, C = 2^(bits-1),
+// s = fp16_ru(fp32(max|x| / Qp)), z = -C s (exact in fp32; the candidate is
+// dropped when |z| exceeds the largest fp16), q = clamp(rint(x / s), -Qp, Qp) + C
+// with x / s taken as fp32(x * fp32(1/s)). It has an exact zero level. A group
+// takes it when its squared reconstruction error is smaller than the
+// asymmetric one's: fp32 e = x - fma(q, s, z), squares summed with fma in
+// element order over runs of 32 elements, run sums added pairwise.
+struct SymParams {
+    __half2 sz;
+    float sf, zf, r;
+    bool ok;
+};
+
+__device__ __forceinline__ SymParams sym_params(float mn, float mx, int bits) {
+    const int C = 1 << (bits - 1);
+    mn = __fadd_rn(mn, 0.0f);
+    mx = __fadd_rn(mx, 0.0f);
+    const float m = fmaxf(fabsf(mn), fabsf(mx));
+    const __half s = __float2half_ru(__fdiv_rn(m, static_cast<float>(C - 1)));
+    SymParams p;
+    p.sf = __half2float(s);
+    p.zf = -static_cast<float>(C) * p.sf;
+    p.ok = fabsf(p.zf) <= 65504.0f;
+    p.sz = __halves2half2(s, __float2half_rn(p.zf));
+    p.r = (p.sf == 0.0f) ? 0.0f : __frcp_rn(p.sf);
+    return p;
+}
+
+__device__ __forceinline__ uint32_t sym_code(float x, const SymParams &p, int bits) {
+    const float C = static_cast<float>(1 << (bits - 1));
+    const float t = fminf(fmaxf(rintf(__fmul_rn(x, p.r)), 1.0f - C), C - 1.0f);
+    return static_cast<uint32_t>(__fadd_rn(t, C));
+}
+
+// Squared error of one run of codes (plain integers) against x.
+__device__ __forceinline__ float sq_err(float x, uint32_t q, float s, float z, float acc) {
+    const float e = __fsub_rn(x, __fmaf_rn(static_cast<float>(q), s, z));
+    return __fmaf_rn(e, e, acc);
 }
 
 // Codes of n consecutive elements (n even) of one group:
@@ -220,11 +263,29 @@ __device__ __forceinline__ void qcodes(const float *x, int n, const QParams &p, 
 // when G > 32) and pack them. Returns the scale/zero pairs of the groups that
 // start in this lane (n_sz of them) and the packed words (4 for INT4, 2 for
 // INT2).
-template <int BITS>
+template <int BITS, bool HYB = false>
 __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32_t words[4],
                                                 __half2 sz[2], int &n_sz, int part) {
     constexpr int L = (1 << BITS) - 1;
     uint32_t q[32];  // 0x4B00000q
+    // hybrid: replace the asymmetric codes of elements [j0, j0 + n) by the
+    // symmetric ones when the group's error sum `es` is below `ea`
+    auto choose = [&](int j0, int n, const SymParams &ps, float ea, float es, __half2 &out_sz) {
+        if (ps.ok && es < ea) {
+#pragma unroll
+            for (int j = j0; j < j0 + n; ++j) q[j] = 0x4B000000u | sym_code(x[j], ps, BITS);
+            out_sz = ps.sz;
+        }
+    };
+    auto run_errs = [&](int j0, int n, const QParams &p, const SymParams &ps, float &ea, float &es) {
+        ea = 0.0f;
+        es = 0.0f;
+#pragma unroll
+        for (int j = j0; j < j0 + n; ++j) {
+            ea = sq_err(x[j], q[j] - 0x4B000000u, p.sf, p.zf, ea);
+            es = sq_err(x[j], sym_code(x[j], ps, BITS), ps.sf, ps.zf, es);
+        }
+    };
     if (G >= 32) {
         float mn = x[0], mx = x[0];
 #pragma unroll
@@ -236,6 +297,17 @@ __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32
         const QParams p = qparams(mn, mx, L);
         qcodes(x, 32, p, q);
         sz[0] = p.sz;
+        if constexpr (HYB) {
+            const SymParams ps = sym_params(mn, mx, BITS);
+            float ea, es;
+            run_errs(0, 32, p, ps, ea, es);
+            // the group's runs (one per lane) added pairwise: (r0 + r1) + (r2 + r3)
+            for (int m = 1; m < G / 32; m <<= 1) {
+                ea += __shfl_xor_sync(0xffffffffu, ea, m);
+                es += __shfl_xor_sync(0xffffffffu, es, m);
+            }
+            choose(0, 32, ps, ea, es, sz[0]);
+        }
         n_sz = ((part * 32) % G == 0) ? 1 : 0;
     } else {  // G == 16: two groups in the lane
 #pragma unroll
@@ -246,6 +318,12 @@ __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32
             const QParams p = qparams(mn, mx, L);
             qcodes(x + 16 * g, 16, p, q + 16 * g);
             sz[g] = p.sz;
+            if constexpr (HYB) {
+                const SymParams ps = sym_params(mn, mx, BITS);
+                float ea, es;
+                run_errs(16 * g, 16, p, ps, ea, es);
+                choose(16 * g, 16, ps, ea, es, sz[g]);
+            }
         }
         n_sz = 2;
     }
@@ -317,7 +395,7 @@ __device__ __forceinline__ bool dest_row(const AppendParams &p, int s, int pos, 
 
 // ---- kernel: per-token append ----------------------------------------------
 // grid.x: blocks of 64 vectors; grid.y: 0 = keys, 1 = values.
-template <int DT>
+template <int DT, bool HYB>
 __global__ void __launch_bounds__(256) append_tokens_kernel(const AppendParams p) {
     pdl_launch_dependents();  // the length advance may be scheduled; it waits for us
     const AppendTensor &T = p.t[blockIdx.y];
@@ -343,8 +421,8 @@ __global__ void __launch_bounds__(256) append_tokens_kernel(const AppendParams p
     uint32_t words[4];
     __half2 s[2];
     int n_sz = 0;
-    if (T.bits == 4) quant_pack_lane<4>(x, T.group, words, s, n_sz, part);
-    else quant_pack_lane<2>(x, T.group, words, s, n_sz, part);
+    if (T.bits == 4) quant_pack_lane<4, HYB>(x, T.group, words, s, n_sz, part);
+    else quant_pack_lane<2, HYB>(x, T.group, words, s, n_sz, part);
     if (!active) return;
 
     const int tok = static_cast<int>(v / p.H);
@@ -385,6 +463,7 @@ struct WindowParams {
     __half2 *k_sz, *v_sz;
     int bits_k, bits_v, group_k, group_v;
     int k_per_channel, v_per_channel;
+    int hybrid;
     int R, H, cap;
     const int32_t *cu_new;
     const int32_t *seq_lens;  // lengths before this append
@@ -394,10 +473,12 @@ struct WindowParams {
 
 // Quantize one block of R staged bf16 rows [R][128] per channel (each
 // channel's R values one group; KIVI keys, InnerQ values) into `codes`
-// (R rows packed along channels) and `sz` ([128] half2). Called by the whole
-// CTA; `qk` is [R][128] bytes of scratch.
-__device__ void flush_channel_block(const uint16_t *src, uint8_t *qk, int R, int bits, uint8_t *codes,
-                                    __half2 *sz) {
+// (R rows packed along channels) and `sz` ([128] half2). With `hybrid`, each
+// group takes the symmetric candidate when its squared error is smaller (runs
+// of 32 tokens, run sums added pairwise). Called by the whole CTA; `qk` is
+// [R][128] bytes of scratch.
+__device__ void flush_channel_block(const uint16_t *src, uint8_t *qk, int R, int bits, int hybrid,
+                                    uint8_t *codes, __half2 *sz) {
     const int L = (1 << bits) - 1;
     const float Lf = static_cast<float>(L);
     for (int d = threadIdx.x; d < kHeadDim; d += blockDim.x) {
@@ -408,9 +489,34 @@ __device__ void flush_channel_block(const uint16_t *src, uint8_t *qk, int R, int
             mx = fmaxf(mx, v);
         }
         const QParams qp = qparams(mn, mx, L);
-        for (int t = 0; t < R; ++t)
-            qk[t * kHeadDim + d] = static_cast<uint8_t>(qcode(bf16_bits_to_float(src[t * kHeadDim + d]), qp, Lf));
-        sz[d] = qp.sz;
+        bool use_sym = false;
+        SymParams ps{};
+        if (hybrid) {
+            ps = sym_params(mn, mx, bits);
+            float ra[8], rs[8];  // R <= 256: at most 8 runs of 32 tokens
+            const int n_runs = R / 32;
+            for (int r = 0; r < n_runs; ++r) {
+                float ea = 0.0f, es = 0.0f;
+                for (int t = 32 * r; t < 32 * r + 32; ++t) {
+                    const float v = bf16_bits_to_float(src[t * kHeadDim + d]);
+                    ea = sq_err(v, qcode(v, qp, Lf), qp.sf, qp.zf, ea);
+                    es = sq_err(v, sym_code(v, ps, bits), ps.sf, ps.zf, es);
+                }
+                ra[r] = ea;
+                rs[r] = es;
+            }
+            for (int w = 1; w < n_runs; w *= 2)
+                for (int r = 0; r + w < n_runs; r += 2 * w) {
+                    ra[r] = __fadd_rn(ra[r], ra[r + w]);
+                    rs[r] = __fadd_rn(rs[r], rs[r + w]);
+                }
+            use_sym = ps.ok && rs[0] < ra[0];
+        }
+        for (int t = 0; t < R; ++t) {
+            const float v = bf16_bits_to_float(src[t * kHeadDim + d]);
+            qk[t * kHeadDim + d] = static_cast<uint8_t>(use_sym ? sym_code(v, ps, bits) : qcode(v, qp, Lf));
+        }
+        sz[d] = use_sym ? ps.sz : qp.sz;
     }
     __syncthreads();
     // Pack along channels: one 32-bit word holds 32/bits channels.
@@ -472,9 +578,9 @@ __global__ void __launch_bounds__(256) window_flush_kernel(const WindowParams p)
     const int64_t row0 = sh * p.cap + static_cast<int64_t>(b) * R;
 
     // Per-channel tensors (keys; values grouped along tokens).
-    if (p.k_per_channel) flush_channel_block(kb, qk, R, p.bits_k, p.k_codes + row0 * (kHeadDim * p.bits_k / 8),
+    if (p.k_per_channel) flush_channel_block(kb, qk, R, p.bits_k, p.hybrid, p.k_codes + row0 * (kHeadDim * p.bits_k / 8),
                                              p.k_sz + (sh * (p.cap / R) + b) * kHeadDim);
-    if (p.v_per_channel) flush_channel_block(vb, qk, R, p.bits_v, p.v_codes + row0 * (kHeadDim * p.bits_v / 8),
+    if (p.v_per_channel) flush_channel_block(vb, qk, R, p.bits_v, p.hybrid, p.v_codes + row0 * (kHeadDim * p.bits_v / 8),
                                              p.v_sz + (sh * (p.cap / R) + b) * kHeadDim);
     // Per-token tensors: 8 vectors per warp, 64 per pass.
     for (int tsel = 0; tsel < 2; ++tsel) {
@@ -494,10 +600,12 @@ __global__ void __launch_bounds__(256) window_flush_kernel(const WindowParams p)
             __half2 s[2];
             int n_sz = 0;
             if (bits == 4) {
-                quant_pack_lane<4>(x, G, words, s, n_sz, part);
+                if (p.hybrid) quant_pack_lane<4, true>(x, G, words, s, n_sz, part);
+                else quant_pack_lane<4, false>(x, G, words, s, n_sz, part);
                 store_lane<4>(codes, sz, row0 + t, G, part, words, s, n_sz);
             } else {
-                quant_pack_lane<2>(x, G, words, s, n_sz, part);
+                if (p.hybrid) quant_pack_lane<2, true>(x, G, words, s, n_sz, part);
+                else quant_pack_lane<2, false>(x, G, words, s, n_sz, part);
                 store_lane<2>(codes, sz, row0 + t, G, part, words, s, n_sz);
             }
         }
@@ -561,6 +669,7 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
         w.group_k = d.group_k; w.group_v = d.group_v;
         w.k_per_channel = d.axis_k == KVQ_PER_CHANNEL;
         w.v_per_channel = d.axis_v == KVQ_PER_CHANNEL;
+        w.hybrid = d.hybrid;
         w.R = d.residual_len; w.H = d.num_kv_heads; w.cap = d.capacity_tokens;
         w.cu_new = cu_new; w.seq_lens = seq_lens;
         w.num_seqs = num_seqs; w.total_tokens = total_new;
@@ -595,9 +704,18 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
         const int64_t n_vec = static_cast<int64_t>(total_new) * d.num_kv_heads;
         const dim3 grid(static_cast<unsigned>((n_vec + 63) / 64), has_v ? 2 : 1);
         switch (dtype) {
-            case KVQ_BF16: append_tokens_kernel<KVQ_BF16><<<grid, 256, 0, stream>>>(p); break;
-            case KVQ_FP16: append_tokens_kernel<KVQ_FP16><<<grid, 256, 0, stream>>>(p); break;
-            default: append_tokens_kernel<KVQ_FP32><<<grid, 256, 0, stream>>>(p); break;
+            case KVQ_BF16:
+                if (d.hybrid) append_tokens_kernel<KVQ_BF16, true><<<grid, 256, 0, stream>>>(p);
+                else append_tokens_kernel<KVQ_BF16, false><<<grid, 256, 0, stream>>>(p);
+                break;
+            case KVQ_FP16:
+                if (d.hybrid) append_tokens_kernel<KVQ_FP16, true><<<grid, 256, 0, stream>>>(p);
+                else append_tokens_kernel<KVQ_FP16, false><<<grid, 256, 0, stream>>>(p);
+                break;
+            default:
+                if (d.hybrid) append_tokens_kernel<KVQ_FP32, true><<<grid, 256, 0, stream>>>(p);
+                else append_tokens_kernel<KVQ_FP32, false><<<grid, 256, 0, stream>>>(p);
+                break;
         }
         if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     }

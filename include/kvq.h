@@ -160,7 +160,19 @@ typedef struct {
                                   without the recent window (residual_len == 0),
                                   contiguous or paged; their quantized rows stay
                                   unused. */
-    int32_t reserved2;         /* must be 0 */
+    int32_t hybrid;            /* 0, or 1: every quantized group of K and V takes
+                                  the symmetric or the asymmetric grid, whichever
+                                  reconstructs it with the smaller squared error
+                                  (InnerQ, Abstract, "(i) hybrid quantization ...
+                                  based on local statistics"; the page states no
+                                  criterion, this is the library's). Symmetric:
+                                  Qp = 2^(bits-1) - 1, C = 2^(bits-1),
+                                  s = fp16_ru(max|x| / Qp), z = -C s, q =
+                                  clamp(rint(x / s), -Qp, Qp) + C, so zero is a level.
+                                  Error: fp32 e = x - fma(q, s, z), squares summed
+                                  with fma over runs of 32 elements in order, runs
+                                  added pairwise; ties keep the asymmetric grid.
+                                  Readers of the cache see (s, z) pairs as always. */
 } kvq_cache_desc;
 
 /*

@@ -80,9 +80,10 @@ def gather_tokens(cache: K.KVCache, which: str, seq: int, head: int, T: int):
     return c.cpu().numpy(), z.cpu().numpy().view(np.uint16)
 
 
-def expected_tokens(x_hist: np.ndarray, head: int, hb: int, G: int, bits: int, signs=None):
+def expected_tokens(x_hist: np.ndarray, head: int, hb: int, G: int, bits: int, signs=None, hybrid=False):
     """Oracle codes and scale/zero for one head of a [T][H][D] history."""
-    return oracle.quantize_tokens(np.ascontiguousarray(x_hist[:, head, :]), hb, G, bits, signs=signs)
+    return oracle.quantize_tokens(np.ascontiguousarray(x_hist[:, head, :]), hb, G, bits, signs=signs,
+                                  hybrid=hybrid)
 
 
 def oracle_decode_tokens(k_hist, v_hist, q, spec: K.CacheSpec, scale=SCALE, signs=None):
@@ -95,9 +96,9 @@ def oracle_decode_tokens(k_hist, v_hist, q, spec: K.CacheSpec, scale=SCALE, sign
     vh = np.zeros((H, T, D))
     for h in range(H):
         kc, ksz = oracle.quantize_tokens(np.ascontiguousarray(k_hist[:, h]), spec.hadamard_block_k,
-                                         spec.group_k, spec.bits_k, signs=signs)
+                                         spec.group_k, spec.bits_k, signs=signs, hybrid=spec.hybrid)
         vc, vsz = oracle.quantize_tokens(np.ascontiguousarray(v_hist[:, h]), 0, spec.group_v,
-                                         spec.bits_v)
+                                         spec.bits_v, hybrid=spec.hybrid)
         kh[h] = oracle.dequant_tokens(kc, ksz, spec.group_k, spec.bits_k)
         vh[h] = oracle.dequant_tokens(vc, vsz, spec.group_v, spec.bits_v)
     return oracle.decode_attention_gqa(q, kh, vh, scale, rotate_q_block=spec.hadamard_block_k,

@@ -63,6 +63,7 @@ def test_append_validation(K):
     assert _append(K, _desc(K, k_codes=FAKE + 4)) == E
     assert _append(K, _desc(K, capacity_tokens=1000)) == E
     assert _append(K, _desc(K, reserved=1)) == E
+    assert _append(K, _desc(K, hybrid=2)) == E          # hybrid is 0 or 1
     # randomized-Hadamard signs need a rotation and 16-byte alignment
     assert _append(K, _desc(K, hadamard_block_k=0, hadamard_signs=FAKE)) == E
     assert _append(K, _desc(K, hadamard_signs=FAKE + 4)) == E

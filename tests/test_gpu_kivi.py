@@ -19,18 +19,18 @@ def _spec(S, H, cap, bits=2, G_v=32, R=128, per_channel=True, per_channel_v=Fals
                        per_channel_v=per_channel_v, residual_len=R, capacity_tokens=cap)
 
 
-def _oracle_tensor(x, Tq, R, bits, G, per_channel):
+def _oracle_tensor(x, Tq, R, bits, G, per_channel, hybrid=False):
     """Codes, scale/zero bit patterns and dequantized rows of x[:Tq] (one head):
     per channel over R-token blocks, or per token in groups of G."""
     if not per_channel:
-        c, z = oracle.quantize_tokens(np.ascontiguousarray(x[:Tq]), 0, G, bits)
+        c, z = oracle.quantize_tokens(np.ascontiguousarray(x[:Tq]), 0, G, bits, hybrid=hybrid)
         return c, z, (oracle.dequant_tokens(c, z, G, bits) if Tq else np.zeros((0, D)))
     codes = np.zeros((Tq, D * bits // 8), np.uint8)
     sz = np.zeros((Tq // R, D, 2), np.uint16)
     xh = np.zeros((Tq, D))
     for b in range(Tq // R):
         sl = slice(b * R, (b + 1) * R)
-        codes[sl], sz[b] = oracle.quantize_channel_block(np.ascontiguousarray(x[sl]), bits)
+        codes[sl], sz[b] = oracle.quantize_channel_block(np.ascontiguousarray(x[sl]), bits, hybrid=hybrid)
         xh[sl] = oracle.dequant_channel_block(codes[sl], sz[b], bits)
     return codes, sz, xh
 
@@ -44,7 +44,7 @@ def _check_state(cache, k, v, T, s, h):
     sp = cache.spec
     R = sp.residual_len
     Tq = oracle.kivi_split(T, R)
-    if sp.per_channel_k and not sp.per_channel_v:  # the KIVI composition of the oracle
+    if sp.per_channel_k and not sp.per_channel_v and not sp.hybrid:  # the oracle's KIVI composition
         want = oracle.quantize_kivi_sequence(np.ascontiguousarray(k[:T, h]), np.ascontiguousarray(v[:T, h]),
                                              R, sp.bits_k, sp.bits_v, sp.group_v)
         assert want["Tq"] == Tq
@@ -52,7 +52,7 @@ def _check_state(cache, k, v, T, s, h):
         assert np.array_equal(cache.sz_view("k")[s, h, :Tq // R].cpu().numpy().view(np.uint16), want["k_sz"])
     for which, G, bits, pc in _tensors(sp):
         x = k if which == "k" else v
-        ec, ez, _ = _oracle_tensor(x[:, h], Tq, R, bits, G, pc)
+        ec, ez, _ = _oracle_tensor(x[:, h], Tq, R, bits, G, pc, sp.hybrid)
         n_sz = Tq // R if pc else Tq
         assert np.array_equal(cache.codes_view(which)[s, h, :Tq].cpu().numpy(), ec), (which, s, h, T)
         assert np.array_equal(cache.sz_view(which)[s, h, :n_sz].cpu().numpy().view(np.uint16), ez), (which, s, h, T)
@@ -63,7 +63,7 @@ def _check_state(cache, k, v, T, s, h):
 
 
 def _oracle_decode(k, v, q, spec):
-    if spec.per_channel_k and not spec.per_channel_v:
+    if spec.per_channel_k and not spec.per_channel_v and not spec.hybrid:
         return oracle_decode_kivi(k, v, q, spec)
     H, T = k.shape[1], k.shape[0]
     R = spec.residual_len
@@ -72,7 +72,7 @@ def _oracle_decode(k, v, q, spec):
     vh = np.zeros((H, T, D))
     for h in range(H):
         for (which, G, bits, pc), dst, x in zip(_tensors(spec), (kh, vh), (k, v)):
-            dst[h, :Tq] = _oracle_tensor(x[:, h], Tq, R, bits, G, pc)[2]
+            dst[h, :Tq] = _oracle_tensor(x[:, h], Tq, R, bits, G, pc, spec.hybrid)[2]
             dst[h, Tq:] = x[Tq:, h]
     return oracle.decode_attention_gqa(q, kh, vh, SCALE)
 
