@@ -488,6 +488,66 @@ def run_long_int2(args, dev):
             "step_GBps": mb / ((statistics.mean(app) + statistics.mean(att)) * 1e-3) / 1e9}
 
 
+def run_long_int2_sharded(args, dev, rank, world):
+    """The long_int2 cache split by token range over the ranks (one GPU each):
+    rank r holds its run of 256-token blocks of the 131072-token sequence in
+    its own KIVI INT2 cache. A step is the sharded decode: split-K and partial
+    merge on every rank, one NCCL all-gather of the partials (130 floats per
+    query head), the cross-rank merge. Strong scaling: the sequence is fixed,
+    each rank reads 1/world of it. Time = max over ranks of the mean step."""
+    import torch
+    import bit_kv_cache_21_b200 as K
+    from bit_kv_cache_21_b200.sharded import decode_attention_sharded, shard_token_range
+    H, HQ_, T_END, R = 8, 32, 131072, 128
+    n_steps, n_warm = 20, 3
+    lo, hi = shard_token_range(T_END, world, rank, 256)
+    T_loc = hi - lo
+    cap = max(256, -(-T_loc // 256) * 256)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3 + rank)
+    spec = K.CacheSpec(1, H, bits_k=2, bits_v=2, group_k=R, group_v=32, per_channel_k=True,
+                       residual_len=R, capacity_tokens=cap)
+    cache = K.KVCache(spec, device=dev)
+    lens = torch.zeros(1, dtype=torch.int32, device=dev)
+    if T_loc:
+        k, v = _synthetic_kv(gen, T_loc, H, dev, torch, 3)
+        K.quantize_append(cache.desc, k, v, torch.tensor([0, T_loc], dtype=torch.int32, device=dev), lens)
+        del k, v
+    qgen = torch.Generator(device=dev)
+    qgen.manual_seed(33)  # the same query on every rank
+    q = torch.randn((1, HQ_, D), generator=qgen, device=dev).to(torch.bfloat16)
+    ws = torch.empty(K.decode_workspace_size(cache.desc, 1, HQ_, cap), dtype=torch.uint8, device=dev)
+    out = torch.empty((1, HQ_, D), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = 1.0 / math.sqrt(D)
+    times = []
+    for i in range(n_warm + n_steps):
+        flush_l2(flush)
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        decode_attention_sharded(cache.desc, q, lens, cap, scale, out=out, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= n_warm:
+            times.append(e0.elapsed_time(e1))
+    assert cache.device_status() == 0
+    Tq = R * ((T_loc - 1) // R) if T_loc else 0
+    nbytes = H * (Tq * (32 + 32 + 16) + (Tq // R) * D * 4 + (T_loc - Tq) * 2 * D * 2)
+    ms = statistics.mean(times)
+    if world > 1:
+        t = torch.tensor([ms, float(nbytes)], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t[:1], op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(t[1:], op=torch.distributed.ReduceOp.SUM)
+        ms, nbytes = float(t[0]), float(t[1])
+    return {"workload": "long_int2 sharded by token range over %d GPU(s): 1 seq x 131072 tokens, "
+                        "32 q / 8 kv heads, KIVI INT2, 128-token bf16 window on each rank" % world,
+            "steps": n_steps, "bytes_per_step": nbytes, "attention_ms": ms,
+            "attention_GBps": nbytes / (ms * 1e-3) / 1e9}
+
+
 def _sweep_setup(dev, seed=6):
     """Shared data of the accuracy/cost sweeps: 16 seqs x 8 KV heads (32 q
     heads) x 4096 tokens of the outlier-key recipe, bf16, and decode attention
@@ -537,6 +597,15 @@ def _sweep_row(spec_kw, d, dev, bytes_per_token_head, n_rep=5):
             app_ms.append(e[0].elapsed_time(e[1]))
             att_ms.append(e[2].elapsed_time(e[3]))
     assert cache.device_status() == 0
+    sym_fraction = None
+    if spec_kw.get("hybrid"):
+        # groups that took the symmetric grid store z = -2^(bits-1) s exactly
+        n_sym = n_all = 0
+        for t, bits in ((cache.k_sz, spec_kw["bits_k"]), (cache.v_sz, spec_kw["bits_v"])):
+            sz = t.view(torch.float16).view(-1, 2).float()
+            n_sym += int(((sz[:, 1] == -(1 << (bits - 1)) * sz[:, 0]) & (sz[:, 0] != 0)).sum())
+            n_all += sz.shape[0]
+        sym_fraction = n_sym / n_all
     diff = out.double() - d["ref"]
     row = {"attn_rel_l2": float(diff.norm() / d["ref"].norm()),
            "attn_max_abs": float(diff.abs().max()),
@@ -544,6 +613,8 @@ def _sweep_row(spec_kw, d, dev, bytes_per_token_head, n_rep=5):
            "append_tokens_per_s": S * T / (statistics.mean(app_ms) * 1e-3),
            "decode_ms": statistics.mean(att_ms),
            "decode_GBps": S * H * T * bytes_per_token_head / (statistics.mean(att_ms) * 1e-3) / 1e9}
+    if sym_fraction is not None:
+        row["symmetric_group_fraction"] = sym_fraction
     del cache, ws
     return row
 
@@ -585,18 +656,23 @@ def run_grouping_sweep(args, dev):
     rotation: token-wise groups for both tensors; KIVI's keys per channel with
     values per token; InnerQ's keys grouped along channels (per token) with
     values grouped along tokens (per channel); both per channel. INT4 with
-    128-wide groups and INT2 with 32-wide token groups."""
+    128-wide groups and INT2 with 32-wide token groups. The KIVI and InnerQ
+    layouts also run with InnerQ's hybrid symmetric/asymmetric groups."""
     d = _sweep_setup(dev)
     R = 128
     rows = []
     for bits, G in ((4, 128), (2, 32)):
-        for pk, pv, name in ((False, False, "token/token"), (True, False, "KIVI: channel/token"),
-                             (False, True, "InnerQ: token/channel"), (True, True, "channel/channel")):
+        for pk, pv, hyb, name in ((False, False, False, "token/token"),
+                                  (True, False, False, "KIVI: channel/token"),
+                                  (True, False, True, "KIVI: channel/token, hybrid"),
+                                  (False, True, False, "InnerQ: token/channel"),
+                                  (False, True, True, "InnerQ: token/channel, hybrid"),
+                                  (True, True, False, "channel/channel")):
             kw = dict(bits_k=bits, bits_v=bits, group_k=R if pk else G, group_v=R if pv else G,
-                      per_channel_k=pk, per_channel_v=pv, residual_len=R)
+                      per_channel_k=pk, per_channel_v=pv, residual_len=R, hybrid=hyb)
             bph = _layout_bytes(bits, pk, G, R) + _layout_bytes(bits, pv, G, R)
             row = {"bits": bits, "token_group": G, "keys": "channel" if pk else "token",
-                   "values": "channel" if pv else "token", "layout": name,
+                   "values": "channel" if pv else "token", "hybrid": hyb, "layout": name,
                    "bytes_per_token_head": bph}
             row.update(_sweep_row(kw, d, dev, bph))
             rows.append(row)
@@ -722,10 +798,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--part", default="all",
                     choices=["all", "decode", "remat", "long_int2", "paged_mix", "rotation_sweep",
-                             "grouping_sweep"],
+                             "grouping_sweep", "long_int2_sharded"],
                     help="run one leg alone: decode (the metric's step), remat, long_int2, "
-                         "paged_mix, rotation_sweep or grouping_sweep (all but decode print "
-                         "their own line)")
+                         "paged_mix, rotation_sweep, grouping_sweep or long_int2_sharded (all "
+                         "but decode print their own line)")
     ap.add_argument("--remat-batch", type=int, default=8)
     ap.add_argument("--remat-steps", type=int, default=10)
     args = ap.parse_args()
@@ -772,6 +848,19 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    if args.part == "long_int2_sharded":
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        leg = run_long_int2_sharded(args, dev, rank, world)
+        if rank == 0:
+            print(json.dumps({"metric": "decode-attn packed-KV GB/s (token-range sharded)",
+                              "value": leg["attention_GBps"], "unit": "GB/s", "n_gpus": world,
+                              "higher_is_better": True, "scaling": "strong", "data": "synthetic",
+                              "config": {"workload": leg["workload"]}, args.part: leg}))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.part in ("long_int2", "paged_mix"):
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)

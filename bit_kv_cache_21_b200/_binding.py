@@ -81,6 +81,8 @@ _SIGNATURES = {
     "kvq_decode_splitk": (_I, [_DESC, _P, _I, _I, _P, _I, _I, ctypes.c_float, _P, _S, _P]),
     "kvq_decode_attention_static": (_I, [_DESC, _P, _I, _I, _P, _I, _I, ctypes.c_float, _P, _P]),
     "kvq_decode_merge": (_I, [_DESC, _I, _P, _I, _I, _P, _P, _S, _P]),
+    "kvq_decode_merge_partial": (_I, [_DESC, _I, _P, _I, _I, _P, _P, _P, _S, _P]),
+    "kvq_merge_partials": (_I, [_P, _I, _I, _I, _P, _P]),
     "kvq_remat_kv": (_I, [_DESC, _P, _I, _P, _P, _I, _I, _P, _P, _P]),
     "kvq_rope_tables": (_I, [_P, _P, _I, _I, ctypes.c_double, _P]),
     "kvq_status_string": (ctypes.c_char_p, [_I]),
@@ -233,6 +235,49 @@ def decode_merge(desc: CacheDesc, num_q_heads: int, seq_lens, max_seq_len: int, 
                                 max_seq_len, _ptr(out), _ptr(workspace), workspace.numel(),
                                 _stream_handle(stream))
     check(st, "kvq_decode_merge")
+
+
+def decode_merge_partial(desc: CacheDesc, num_q_heads: int, seq_lens, max_seq_len: int, o_part, ml,
+                         workspace, stream=None) -> None:
+    """kvq_decode_merge_partial: this cache's unnormalized partial o_part fp32
+    [S][Hq][128] and its (m, l) pairs ml fp32 [S][Hq][2]."""
+    import torch
+    for t, name in ((o_part, "o_part"), (ml, "ml")):
+        if t is None or not t.is_cuda or t.dtype != torch.float32:
+            raise ValueError("%s must be a CUDA fp32 tensor" % name)
+    st = lib().kvq_decode_merge_partial(ctypes.byref(desc), num_q_heads, _ptr(seq_lens), o_part.shape[0],
+                                        max_seq_len, _ptr(o_part), _ptr(ml), _ptr(workspace),
+                                        workspace.numel(), _stream_handle(stream))
+    check(st, "kvq_decode_merge_partial")
+
+
+def partial_buffer(num_seqs: int, num_q_heads: int, device, n_part: int = 1):
+    """fp32 [n_part][S*Hq*130]: per part the o rows [S][Hq][128], then the
+    (m, l) pairs [S][Hq][2] (the layout kvq_merge_partials reads)."""
+    import torch
+    return torch.empty((n_part, num_seqs * num_q_heads * 130), dtype=torch.float32, device=device)
+
+
+def partial_views(buf, num_seqs: int, num_q_heads: int):
+    """o_part [S][Hq][128] and ml [S][Hq][2] views of one part of partial_buffer."""
+    rows = num_seqs * num_q_heads
+    return buf[:rows * 128].view(num_seqs, num_q_heads, 128), buf[rows * 128:].view(num_seqs, num_q_heads, 2)
+
+
+def merge_partials(parts, num_seqs: int, num_q_heads: int, out=None, stream=None):
+    """kvq_merge_partials: parts fp32 [n_part][S*Hq*130] (partial_buffer's
+    layout) -> out fp32 [S][Hq][128]."""
+    import torch
+    _require(parts, "parts", torch.float32)
+    if parts.dim() != 2 or parts.shape[1] != num_seqs * num_q_heads * 130:
+        raise ValueError("parts must be [n_part][num_seqs * num_q_heads * 130]")
+    if out is None:
+        out = torch.empty((num_seqs, num_q_heads, 128), dtype=torch.float32, device=parts.device)
+    _require(out, "out", torch.float32)
+    st = lib().kvq_merge_partials(_ptr(parts), parts.shape[0], num_seqs, num_q_heads, _ptr(out),
+                                  _stream_handle(stream))
+    check(st, "kvq_merge_partials")
+    return out
 
 
 def remat_kv(x_desc: CacheDesc, w_kv, n_kv_heads: int, rope_cos, rope_sin, batch: int,

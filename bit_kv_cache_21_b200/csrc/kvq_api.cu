@@ -169,7 +169,34 @@ kvq_status kvq_decode_merge(const kvq_cache_desc *desc, int32_t num_q_heads,
     if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < plan.ws_total)
         return workspace == nullptr || !aligned16(workspace) ? KVQ_ERR_INVALID_ARG : KVQ_ERR_CAPACITY;
     return launch_decode_merge(*desc, plan, num_q_heads, seq_lens, num_seqs, max_seq_len, out,
+                               nullptr, workspace, static_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_decode_merge_partial(const kvq_cache_desc *desc, int32_t num_q_heads,
+                                    const int32_t *seq_lens, int32_t num_seqs, int32_t max_seq_len,
+                                    float *o_part, float *ml, const void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+    kvq_status s = validate_desc(desc, true);
+    if (s != KVQ_OK) return s;
+    if (o_part == nullptr || ml == nullptr || !aligned16(o_part) || (reinterpret_cast<uintptr_t>(ml) & 7u) ||
+        seq_lens == nullptr || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)
+        return KVQ_ERR_INVALID_ARG;
+    DecodePlan plan;
+    if (!plan_decode(*desc, num_seqs, num_q_heads, max_seq_len, &plan)) return KVQ_ERR_INVALID_ARG;
+    if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < plan.ws_total)
+        return workspace == nullptr || !aligned16(workspace) ? KVQ_ERR_INVALID_ARG : KVQ_ERR_CAPACITY;
+    return launch_decode_merge(*desc, plan, num_q_heads, seq_lens, num_seqs, max_seq_len, o_part, ml,
                                workspace, static_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_merge_partials(const float *parts, int32_t n_part, int32_t num_seqs, int32_t num_q_heads,
+                              float *out, void *stream) {
+    if (parts == nullptr || out == nullptr || !aligned16(parts) || n_part <= 0 || num_seqs <= 0 ||
+        num_q_heads <= 0 || num_seqs > 65535 || num_q_heads > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(num_seqs) * num_q_heads * (kHeadDim + 2) * n_part > (int64_t(1) << 40))
+        return KVQ_ERR_INVALID_ARG;
+    return launch_merge_partials(parts, n_part, num_seqs, num_q_heads, out, static_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_decode_attention(const kvq_cache_desc *desc, const void *q, kvq_dtype q_dtype,

@@ -8,38 +8,74 @@ namespace kvq {
 using namespace dec;
 
 namespace {
-// One CTA of 128 threads per (query head, sequence): combine the splits.
-// Launched as a programmatic dependent of the split-K pass: its CTAs may start
-// while that pass drains and wait here until its partials are complete.
+// Log-sum-exp combination of n partials (o_j, m_j, l_j) of one (sequence,
+// query head) by a CTA of 128 threads (channel d each): partial j's o row at
+// o_part + o0 + j * o_step (kHeadDim floats), its (m, l) at ml[m0 + j * m_step].
+// o = sum_j e_j o_j, l = sum_j e_j l_j with e_j = 2^(m_j - M), M = max_j m_j
+// (log2 units). Partials with m = -inf (no tokens) weigh 0.
+__device__ __forceinline__ void combine_partials(const float *o_part, const float2 *ml, int64_t o0,
+                                                 int64_t o_step, int64_t m0, int64_t m_step, int n,
+                                                 float *s_max, float &M, float &o, float &l) {
+    const int d = threadIdx.x;
+    if (d < 32) {  // maximum over the partials, one warp
+        float m = -INFINITY;
+        for (int j = d; j < n; j += 32) m = fmaxf(m, ml[m0 + j * m_step].x);
+#pragma unroll
+        for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
+        if (d == 0) *s_max = m;
+    }
+    __syncthreads();
+    M = *s_max;
+    o = 0.0f;
+    l = 0.0f;
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) {
+        const float2 v = ml[m0 + j * m_step];
+        const float e = (v.x == -INFINITY) ? 0.0f : fast_exp2(v.x - M);
+        o = fmaf(e, o_part[o0 + j * o_step + d], o);
+        l = fmaf(e, v.y, l);
+    }
+}
+
+// One CTA of 128 threads per (query head, sequence): combine the splits into
+// the output, or (PARTIAL) into this cache's unnormalized partial (o, m, l)
+// for a merge with the partials of other caches that hold other token ranges
+// of the same sequences. Launched as a programmatic dependent of the split-K
+// pass: its CTAs may start while that pass drains and wait here until its
+// partials are complete.
+template <bool PARTIAL>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const float *o_part, const float2 *ml,
                                                            const int32_t *seq_lens, float *out,
-                                                           int Hq, int n_split, int chunk,
-                                                           int max_seq_len) {
+                                                           float2 *out_ml, int Hq, int n_split,
+                                                           int chunk, int max_seq_len) {
     __shared__ float s_max;
     pdl_wait_prior_grid();
     const int hq = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
     const int T = min(__ldg(seq_lens + seq), max_seq_len);
     const int nv = T > 0 ? (T + chunk - 1) / chunk : 0;
-    const int64_t base = (static_cast<int64_t>(seq) * Hq + hq) * n_split;
-    if (d < 32) {  // maximum over the splits, one warp
-        float m = -INFINITY;
-        for (int j = d; j < nv; j += 32) m = fmaxf(m, ml[base + j].x);
-#pragma unroll
-        for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
-        if (d == 0) s_max = m;
+    const int64_t row = static_cast<int64_t>(seq) * Hq + hq;
+    float M, o, l;
+    combine_partials(o_part, ml, row * n_split * kHeadDim, kHeadDim, row * n_split, 1, nv, &s_max, M, o, l);
+    if constexpr (PARTIAL) {
+        out[row * kHeadDim + d] = o;
+        if (d == 0) out_ml[row] = make_float2(M, l);
+    } else {
+        out[row * kHeadDim + d] = (l > 0.0f) ? o / l : 0.0f;
     }
-    __syncthreads();
-    const float M = s_max;
-    float o = 0.0f, l = 0.0f;
-    const float *op = o_part + base * kHeadDim + d;
-#pragma unroll 4
-    for (int j = 0; j < nv; ++j) {
-        const float2 v = ml[base + j];
-        const float e = (v.x == -INFINITY) ? 0.0f : fast_exp2(v.x - M);
-        o = fmaf(e, op[static_cast<int64_t>(j) * kHeadDim], o);
-        l = fmaf(e, v.y, l);
-    }
-    out[(static_cast<int64_t>(seq) * Hq + hq) * kHeadDim + d] = (l > 0.0f) ? o / l : 0.0f;
+}
+
+// One CTA of 128 threads per (query head, sequence): the output from n_part
+// partials, part j = `rows` o rows of kHeadDim floats then `rows` (m, l)
+// pairs, parts back to back (rows * (kHeadDim + 2) floats each).
+__global__ void __launch_bounds__(128) merge_partials_kernel(const float *parts, int n_part, int rows,
+                                                             float *out) {
+    __shared__ float s_max;
+    const int64_t row = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+    const int64_t part = static_cast<int64_t>(rows) * (kHeadDim + 2);  // floats per part
+    const float2 *ml = reinterpret_cast<const float2 *>(parts + static_cast<int64_t>(rows) * kHeadDim);
+    float M, o, l;
+    combine_partials(parts, ml, row * kHeadDim, part, row, part / 2, n_part, &s_max, M, o, l);
+    out[row * kHeadDim + threadIdx.x] = (l > 0.0f) ? o / l : 0.0f;
 }
 
 }  // namespace
@@ -129,7 +165,7 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
 
 kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, int num_q_heads,
                                const int32_t *seq_lens, int num_seqs, int max_seq_len,
-                               float *out, const void *workspace, cudaStream_t stream) {
+                               float *out, float *out_ml, const void *workspace, cudaStream_t stream) {
     (void)d;
     const float *o_part = static_cast<const float *>(workspace);
     const float2 *ml =
@@ -145,10 +181,20 @@ kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const int n_split = plan.n_split, chunk = plan.chunk;
-    return cudaLaunchKernelEx(&cfg, decode_merge_kernel, o_part, ml, seq_lens, out, num_q_heads,
-                              n_split, chunk, max_seq_len) == cudaSuccess
-               ? KVQ_OK
-               : KVQ_ERR_CUDA;
+    float2 *oml = reinterpret_cast<float2 *>(out_ml);
+    const cudaError_t e =
+        out_ml ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<true>, o_part, ml, seq_lens, out, oml,
+                                    num_q_heads, n_split, chunk, max_seq_len)
+               : cudaLaunchKernelEx(&cfg, decode_merge_kernel<false>, o_part, ml, seq_lens, out, oml,
+                                    num_q_heads, n_split, chunk, max_seq_len);
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status launch_merge_partials(const float *parts, int n_part, int num_seqs, int num_q_heads, float *out,
+                                 cudaStream_t stream) {
+    merge_partials_kernel<<<dim3(num_q_heads, num_seqs), 128, 0, stream>>>(parts, n_part, num_seqs * num_q_heads,
+                                                                           out);
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 }  // namespace kvq

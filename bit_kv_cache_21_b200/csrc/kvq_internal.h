@@ -35,9 +35,13 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
                                 kvq_dtype q_dtype, int num_q_heads, const int32_t *seq_lens,
                                 int num_seqs, int max_seq_len, float softmax_scale,
                                 void *workspace, cudaStream_t stream);
+// out_ml == nullptr: normalized output; else this cache's unnormalized
+// partial into out and its (m, l) pairs into out_ml.
 kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, int num_q_heads,
                                const int32_t *seq_lens, int num_seqs, int max_seq_len,
-                               float *out, const void *workspace, cudaStream_t stream);
+                               float *out, float *out_ml, const void *workspace, cudaStream_t stream);
+kvq_status launch_merge_partials(const float *parts, int n_part, int num_seqs, int num_q_heads, float *out,
+                                 cudaStream_t stream);
 
 kvq_status launch_remat(const kvq_cache_desc &x, const void *w_kv, int n_kv_heads,
                         const float *rope_cos, const float *rope_sin, int batch, int ctx_len,

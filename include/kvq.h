@@ -247,6 +247,43 @@ KVQ_API kvq_status kvq_decode_merge(const kvq_cache_desc *desc, int32_t num_q_he
                             void *stream);
 
 /*
+ * Token-range sharding of long sequences over several caches (one per GPU):
+ * each cache holds a disjoint, contiguous token range of the same sequences
+ * (lengths local to the cache), and softmax attention over the union is the
+ * log-sum-exp combination of the per-cache partials, the same identity the
+ * split-K merge uses inside one cache. A decode step is then kvq_decode_splitk
+ * and kvq_decode_merge_partial on every cache, one all-gather of the partials
+ * (e.g. NCCL; 130 floats per query head per cache), and kvq_merge_partials.
+ *
+ * kvq_decode_merge_partial -- as kvq_decode_merge, but writes this cache's
+ * unnormalized partial: o_part fp32 [num_seqs][num_q_heads][D] holds
+ * sum_t 2^(x_t - m) v^_t and ml fp32 [num_seqs][num_q_heads][2] holds (m, l),
+ * with x_t = log2(e) * softmax_scale * q~ . k^_t, l = sum_t 2^(x_t - m) and m
+ * a reference score: max_t x_t up to the kernel's lazy rescaling (m may sit
+ * below the maximum by at most 8, so every weight stays <= 2^8). Only
+ * o / l and l * 2^m carry meaning. A sequence with no tokens here gives
+ * (-inf, 0) and zeros. o_part 16-byte and ml 8-byte aligned.
+ */
+KVQ_API kvq_status kvq_decode_merge_partial(const kvq_cache_desc *desc, int32_t num_q_heads,
+                                            const int32_t *seq_lens, int32_t num_seqs,
+                                            int32_t max_seq_len, float *o_part, float *ml,
+                                            const void *workspace, size_t workspace_bytes,
+                                            void *stream);
+
+/*
+ * kvq_merge_partials -- out[s][h] = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r
+ * over n_part partials (M = max_r m_r; zeros when every l_r is 0). `parts`:
+ * device fp32, the n_part partials back to back, each num_seqs * num_q_heads
+ * o rows [num_seqs][num_q_heads][D] followed by their (m, l) pairs
+ * [num_seqs][num_q_heads][2] -- what an all-gather of one buffer per cache
+ * gives when kvq_decode_merge_partial wrote o_part at its start and ml right
+ * after the o rows. 16-byte aligned. out: device fp32 [num_seqs][num_q_heads][D].
+ * num_seqs and num_q_heads at most 65535.
+ */
+KVQ_API kvq_status kvq_merge_partials(const float *parts, int32_t n_part, int32_t num_seqs,
+                                      int32_t num_q_heads, float *out, void *stream);
+
+/*
  * kvq_decode_attention_static -- kvq_decode_attention without a workspace
  * argument, for callers that cannot allocate device memory: a plain C program
  * or a plugin running inside a runtime that owns every device allocation, or a

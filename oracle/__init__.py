@@ -321,6 +321,40 @@ def decode_attention_gqa_sinks(q, khat, vhat, k_sink, v_sink, scale, rotate_q_bl
 # Cache composition for one sequence (the method's steps in order)
 # --------------------------------------------------------------------------
 
+def attention_partial(q, k, v, scale):
+    """Unnormalized softmax attention of query rows q [n][D] over one range of
+    tokens k, v [T][D], in float64 and log2 units: x_t = log2(e) * scale *
+    q . k_t, m = max_t x_t, l = sum_t 2^(x_t - m), o = sum_t 2^(x_t - m) v_t.
+    No tokens: m = -inf, l = 0, o = 0. Returns (o [n][D], m [n], l [n])."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    n, D = q.shape
+    if k.shape[0] == 0:
+        return np.zeros((n, D)), np.full(n, -np.inf), np.zeros(n)
+    x = (q @ k.T) * (scale * np.log2(np.e))
+    m = x.max(axis=1)
+    p = np.exp2(x - m[:, None])
+    return p @ v, m, p.sum(axis=1)
+
+
+def merge_partials(parts):
+    """Attention output from partials (o, m, l) of disjoint token ranges
+    (attention_partial's form): sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r,
+    M = max_r m_r; zeros where every range is empty."""
+    M = np.max(np.stack([m for _, m, _ in parts]), axis=0)
+    o = np.zeros_like(parts[0][0])
+    l = np.zeros_like(parts[0][2])
+    for o_r, m_r, l_r in parts:
+        live = ~np.isneginf(m_r)  # an empty range weighs 0
+        e = np.zeros_like(l_r)
+        e[live] = np.exp2(m_r[live] - M[live])
+        o = o + e[:, None] * o_r
+        l = l + e * l_r
+    with np.errstate(invalid="ignore", divide="ignore"):
+        return np.where(l[:, None] > 0, o / np.where(l > 0, l, 1.0)[:, None], 0.0)
+
+
 def kivi_split(T, R):
     """Number of quantized tokens when the most recent tokens stay in a
     full-precision window of capacity R that is flushed as one block only

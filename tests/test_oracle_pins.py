@@ -598,3 +598,25 @@ def test_hybrid_applies_per_group_in_token_and_channel_layouts():
     for d in (0, 5, 127):
         s, z, qg = oracle.quantize_group_hybrid(np.ascontiguousarray(blk[:, d]), 2)
         assert (s, z) == tuple(sz[d]) and np.array_equal(q[:, d], qg)
+
+
+# ---------------------------------------------------------------------------
+# Partials of disjoint token ranges (the sharded decode's merge)
+# ---------------------------------------------------------------------------
+
+def test_partials_of_any_token_split_merge_to_attention():
+    g = np.random.default_rng(41)
+    q = g.standard_normal((4, 16))
+    k = g.standard_normal((37, 16)) * 3
+    v = g.standard_normal((37, 16))
+    want = scipy.special.softmax(q @ k.T * 0.25, axis=1) @ v
+    for cuts in ([0, 37], [0, 1, 37], [0, 10, 10, 37], [0, 5, 20, 36, 37]):
+        parts = [oracle.attention_partial(q, k[a:b], v[a:b], 0.25) for a, b in zip(cuts[:-1], cuts[1:])]
+        assert np.allclose(oracle.merge_partials(parts), want, atol=1e-13)
+    # one range: o / l is the attention, and m is the largest log2-unit score
+    o, m, l = oracle.attention_partial(q, k, v, 0.25)
+    assert np.allclose(o / l[:, None], want, atol=1e-13)
+    assert np.allclose(m, (q @ k.T).max(axis=1) * 0.25 / np.log(2), atol=1e-12)
+    # every range empty -> zeros
+    e = oracle.attention_partial(q, k[:0], v[:0], 0.25)
+    assert np.array_equal(oracle.merge_partials([e, e]), np.zeros((4, 16)))
