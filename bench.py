@@ -390,6 +390,23 @@ def run_remat(args, dev):
     assert cache.device_status() == 0 and int(status[0]) == 0
     remat_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # the fused path: remat GEMM with attention in its epilogue (K/V never stored)
+    fws = torch.empty(int(K.lib().kvq_remat_attention_workspace_size(B, XQ_HQ, T)), dtype=torch.uint8,
+                      device=dev)
+    fout = torch.empty_like(out)
+    fused_ms = []
+    for i in range(args.warmup + args.remat_steps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        K.remat_attention(cache.desc, w, H, cos, sin, B, T, q, scale, out=fout, workspace=fws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            fused_ms.append(e0.elapsed_time(e1))
+    assert cache.device_status() == 0
+    fused_diff = float((fout - out).abs().max())
+    fused = statistics.mean(fused_ms)
     flops = 2.0 * B * T * (2 * H * D) * hidden
     kv_bytes = 2.0 * B * H * T * D * 2
     peak_b, peak_s, kind = tensor_peaks()
@@ -404,6 +421,11 @@ def run_remat(args, dev):
                       "frac_of_sustained": tflops / peak_s},
             "attention_bf16": {"ms": attn_ms, "bytes": kv_bytes,
                                "GBps": kv_bytes / (attn_ms * 1e-3) / 1e9},
+            "fused_remat_attention": {"kernel": "remat_kernel<FUSED> + remat_merge_kernel", "ms": fused,
+                                      "achieved": flops / (fused * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                      "frac": flops / (fused * 1e-3) / 1e12 / peak_b,
+                                      "speedup_vs_unfused": (remat_ms + attn_ms) / fused,
+                                      "max_abs_diff_vs_unfused": fused_diff},
             "gpu_launches_per_step": 4}
 
 

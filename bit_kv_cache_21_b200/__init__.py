@@ -13,6 +13,6 @@ from ._binding import (  # noqa: F401
     CacheDesc, KvqError, lib, header_symbols, status_string, check,
     quantize_append, decode_workspace_size, decode_attention, decode_attention_static,
     decode_splitk, decode_merge, decode_merge_partial, merge_partials, partial_buffer, partial_views,
-    remat_kv, rope_tables, debug_set, version,
+    remat_kv, remat_attention, rope_tables, debug_set, version,
 )
 from .cache import CacheSpec, KVCache, bf16_cache_desc, sink_view  # noqa: F401

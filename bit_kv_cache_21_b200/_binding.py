@@ -85,6 +85,8 @@ _SIGNATURES = {
     "kvq_merge_partials": (_I, [_P, _I, _I, _I, _P, _P]),
     "kvq_remat_kv": (_I, [_DESC, _P, _I, _P, _P, _I, _I, _P, _P, _P]),
     "kvq_rope_tables": (_I, [_P, _P, _I, _I, ctypes.c_double, _P]),
+    "kvq_remat_attention_workspace_size": (_S, [_I, _I, _I]),
+    "kvq_remat_attention": (_I, [_DESC, _P, _I, _P, _P, _I, _I, _P, _I, _I, ctypes.c_float, _P, _P, _S, _P]),
     "kvq_status_string": (ctypes.c_char_p, [_I]),
     "kvq_debug_set": (_I, [_I, ctypes.c_int64]),
     "kvq_version": (_I, []),
@@ -293,6 +295,27 @@ def remat_kv(x_desc: CacheDesc, w_kv, n_kv_heads: int, rope_cos, rope_sin, batch
                             _ptr(rope_sin), batch, ctx_len, _ptr(k_out), _ptr(v_out),
                             _stream_handle(stream))
     check(st, "kvq_remat_kv")
+
+
+def remat_attention(x_desc: CacheDesc, w_kv, n_kv_heads: int, rope_cos, rope_sin, batch: int,
+                    ctx_len: int, q, softmax_scale: float, out=None, workspace=None, stream=None):
+    """kvq_remat_attention: decode attention of q [batch][Hq][128] over K, V
+    rematerialized from the X cache on the fly -> out fp32 [batch][Hq][128]."""
+    import torch
+    _require(w_kv, "w_kv", torch.bfloat16)
+    _require(q, "q")
+    num_q_heads = q.shape[1]
+    if workspace is None:
+        need = int(lib().kvq_remat_attention_workspace_size(batch, num_q_heads, ctx_len))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((batch, num_q_heads, 128), dtype=torch.float32, device=q.device)
+    _require(out, "out", torch.float32)
+    st = lib().kvq_remat_attention(ctypes.byref(x_desc), _ptr(w_kv), n_kv_heads, _ptr(rope_cos), _ptr(rope_sin),
+                                   batch, ctx_len, _ptr(q), dtype_code(q), num_q_heads, float(softmax_scale),
+                                   _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    check(st, "kvq_remat_attention")
+    return out
 
 
 def rope_tables(n_pos: int, head_dim: int = 128, theta: float = 500000.0, device="cuda", stream=None):

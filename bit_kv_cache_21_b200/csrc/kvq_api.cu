@@ -231,6 +231,37 @@ kvq_status kvq_remat_kv(const kvq_cache_desc *x_cache, const void *w_kv, int32_t
                         v_out, static_cast<cudaStream_t>(stream));
 }
 
+size_t kvq_remat_attention_workspace_size(int32_t batch, int32_t num_q_heads, int32_t ctx_len) {
+    if (batch <= 0 || num_q_heads <= 0 || ctx_len <= 0 || ctx_len % 128 != 0) return 0;
+    return remat_attention_workspace(batch, num_q_heads, ctx_len);
+}
+
+kvq_status kvq_remat_attention(const kvq_cache_desc *x_cache, const void *w_kv, int32_t n_kv_heads,
+                               const float *rope_cos, const float *rope_sin, int32_t batch, int32_t ctx_len,
+                               const void *q, kvq_dtype q_dtype, int32_t num_q_heads, float softmax_scale,
+                               float *out, void *workspace, size_t workspace_bytes, void *stream) {
+    kvq_status s = validate_desc(x_cache, false);
+    if (s != KVQ_OK) return s;
+    if (x_cache->paged || x_cache->bits_k != 4 || x_cache->group_k != 128 ||
+        x_cache->axis_k != KVQ_PER_TOKEN || x_cache->hadamard_block_k != 0 ||
+        x_cache->residual_len != 0 || x_cache->sink_len != 0)
+        return KVQ_ERR_UNSUPPORTED;
+    if (w_kv == nullptr || rope_cos == nullptr || rope_sin == nullptr || q == nullptr || out == nullptr ||
+        !aligned16(w_kv) || !aligned16(rope_cos) || !aligned16(rope_sin) || !aligned16(q) || !aligned16(out) ||
+        !dtype_ok(q_dtype))
+        return KVQ_ERR_INVALID_ARG;
+    if (n_kv_heads <= 0 || batch <= 0 || batch > x_cache->num_seqs || ctx_len <= 0 || ctx_len % 128 != 0 ||
+        ctx_len > x_cache->capacity_tokens || num_q_heads <= 0 || num_q_heads % n_kv_heads != 0 ||
+        batch > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    const int gqa = num_q_heads / n_kv_heads;
+    if (gqa != 1 && gqa != 2 && gqa != 4) return KVQ_ERR_UNSUPPORTED;
+    if (workspace == nullptr || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
+    if (workspace_bytes < remat_attention_workspace(batch, num_q_heads, ctx_len)) return KVQ_ERR_CAPACITY;
+    return launch_remat_attention(*x_cache, w_kv, n_kv_heads, rope_cos, rope_sin, batch, ctx_len, q, q_dtype,
+                                  num_q_heads, softmax_scale, out, workspace, static_cast<cudaStream_t>(stream));
+}
+
 kvq_status kvq_rope_tables(float *rope_cos, float *rope_sin, int32_t n_pos, int32_t head_dim,
                            double theta, void *stream) {
     if (rope_cos == nullptr || rope_sin == nullptr || n_pos <= 0 || head_dim <= 0 ||

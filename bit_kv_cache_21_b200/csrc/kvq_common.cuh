@@ -169,4 +169,33 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// Log-sum-exp combination of n partials (o_j, m_j, l_j) of one (sequence,
+// query head) by a CTA of 128 threads (channel d each): partial j's o row at
+// o_part + o0 + j * o_step (kHeadDim floats), its (m, l) at ml[m0 + j * m_step].
+// o = sum_j e_j o_j, l = sum_j e_j l_j with e_j = 2^(m_j - M), M = max_j m_j
+// (log2 units). Partials with m = -inf (no tokens) weigh 0.
+__device__ __forceinline__ void combine_partials(const float *o_part, const float2 *ml, int64_t o0,
+                                                 int64_t o_step, int64_t m0, int64_t m_step, int n,
+                                                 float *s_max, float &M, float &o, float &l) {
+    const int d = threadIdx.x;
+    if (d < 32) {  // maximum over the partials, one warp
+        float m = -INFINITY;
+        for (int j = d; j < n; j += 32) m = fmaxf(m, ml[m0 + j * m_step].x);
+#pragma unroll
+        for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
+        if (d == 0) *s_max = m;
+    }
+    __syncthreads();
+    M = *s_max;
+    o = 0.0f;
+    l = 0.0f;
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) {
+        const float2 v = ml[m0 + j * m_step];
+        const float e = (v.x == -INFINITY) ? 0.0f : fast_exp2(v.x - M);
+        o = fmaf(e, o_part[o0 + j * o_step + d], o);
+        l = fmaf(e, v.y, l);
+    }
+}
+
 }  // namespace kvq

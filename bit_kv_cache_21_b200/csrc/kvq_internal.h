@@ -48,5 +48,10 @@ kvq_status launch_remat(const kvq_cache_desc &x, const void *w_kv, int n_kv_head
                         void *k_out, void *v_out, cudaStream_t stream);
 kvq_status launch_rope_tables(float *c, float *s, int n_pos, int head_dim, double theta,
                               cudaStream_t stream);
+size_t remat_attention_workspace(int batch, int num_q_heads, int ctx_len);
+kvq_status launch_remat_attention(const kvq_cache_desc &x, const void *w_kv, int n_kv_heads,
+                                  const float *rope_cos, const float *rope_sin, int batch, int ctx_len,
+                                  const void *q, kvq_dtype q_dtype, int num_q_heads, float softmax_scale,
+                                  float *out, void *workspace, cudaStream_t stream);
 
 }  // namespace kvq

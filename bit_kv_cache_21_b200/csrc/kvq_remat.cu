@@ -89,6 +89,14 @@ static_assert(kCStages % kDeqGroups == 0, "a codes slot always goes to the same 
 
 struct RematParams {
     const __half2 *x_sz;   // [S][XH][Tc] (one group of 128 channels per row)
+    // fused attention (remat_kernel<true>): the tile of head h holds its K
+    // (accumulator columns 0..127) and V (128..255); per tile a partial
+    // (o, m, l) of the GQA query heads over its 128 tokens.
+    const void *q;         // [B][Hq][128] of q_dtype
+    int q_dtype, gqa;      // gqa = Hq / H (1, 2 or 4)
+    float qscale;          // softmax scale * log2(e)
+    float *o_part;         // [B][Hq][n_blk][128]
+    float2 *ml;            // [B][Hq][n_blk]
     const float *rope_cos; // [T][64]
     const float *rope_sin;
     uint16_t *k_out;       // bf16 [B][H][T][128]
@@ -229,6 +237,11 @@ __device__ __forceinline__ void bulk_wait_read() {
 // Wait until the issued bulk stores have completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// x rounded to the nearest bf16 (ties to even), as a float.
+__device__ __forceinline__ float bf16_round(float x) {
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -334,6 +347,11 @@ __device__ __forceinline__ TileCoord tile_coord(const RematParams &p, int tile) 
     return c;
 }
 
+// FUSED: decode attention over the rematerialized tile instead of storing
+// it (K and V never reach HBM): W's B tile is head h's 128 K rows then its 128
+// V rows (two TMA boxes of tm_w, 64 x 128), and the epilogue scores the tile's
+// 128 tokens against the GQA query rows.
+template <bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     remat_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -416,7 +434,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&w_full[s], kBBytes);
-                    tma_load_2d(w_ring + s * kBBytes, &tm_w, kb * kBK, c.n * kBN, &w_full[s]);
+                    if constexpr (FUSED) {  // head c.n: its K rows, then its V rows
+                        tma_load_2d(w_ring + s * kBBytes, &tm_w, kb * kBK, c.n * kHeadDim, &w_full[s]);
+                        tma_load_2d(w_ring + s * kBBytes + kBBytes / 2, &tm_w, kb * kBK,
+                                    (p.H + c.n) * kHeadDim, &w_full[s]);
+                    } else {
+                        tma_load_2d(w_ring + s * kBBytes, &tm_w, kb * kBK, c.n * kBN, &w_full[s]);
+                    }
                 }
             }
             drain(w_full, kWStages, it);
@@ -534,6 +558,149 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&a_full[sa]);
             }
         }
+    } else if constexpr (FUSED) {
+        // --------------------------- attention epilogue ---------------------------
+        // Thread `row` owns token c.t0 + row (its TMEM lane). K and V are
+        // rounded to bf16 as the unfused path stores them; scores, softmax and
+        // P V of the tile in fp32; the partial (o, m, l) per query head goes
+        // to the workspace for the merge over the tiles.
+        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+        const int row = quarter * 32 + lane;
+        float *q_s = reinterpret_cast<float *>(out_stage);              // [4][128] scaled queries
+        float *p_s = q_s + 4 * kHeadDim;                                // [128][4] weights
+        float *red = p_s + kBM * 4;                                     // [4 warps][4] max, then sums
+        uint16_t *v_s = reinterpret_cast<uint16_t *>(red + 32);         // bf16 [128][kVStride]
+        constexpr int kVStride = kHeadDim + 8;  // padded rows: 8 consecutive rows hit distinct banks
+        const int n_blk = p.T / kBM;
+        int lt = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < n_total; tile += gridDim.x, ++lt) {
+            ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(acc_full, lt & 1, p.timeout_ns,
+                                                                 p.status, abort_flag));
+            tc_fence_after();
+            if (!ok) {  // take every barrier of the tile so no epilogue warp is left waiting
+                named_sync(1, 128);
+                named_sync(1, 128);
+                named_sync(1, 128);
+                named_sync(1, 128);
+                continue;
+            }
+            const TileCoord c = tile_coord(p, tile);
+            const int t = c.t0 + row;
+            const int hq0 = c.n * p.gqa;
+            const int Hq = p.H * p.gqa;
+            // (A) the tile's query rows, scaled, zero for heads past gqa
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int idx = i * kBM + row;  // [g][channel]
+                const int g = idx / kHeadDim, ch = idx - g * kHeadDim;
+                float v = 0.0f;
+                if (g < p.gqa) {
+                    const int64_t qi = (static_cast<int64_t>(c.b) * Hq + hq0 + g) * kHeadDim + ch;
+                    if (p.q_dtype == KVQ_FP32) v = static_cast<const float *>(p.q)[qi];
+                    else if (p.q_dtype == KVQ_BF16) v = bf16_bits_to_float(static_cast<const uint16_t *>(p.q)[qi]);
+                    else v = __half2float(static_cast<const __half *>(p.q)[qi]);
+                }
+                q_s[idx] = v * p.qscale;
+            }
+            named_sync(1, 128);
+            // (B) scores of this token: RoPE on K (pairs i, i + 64), bf16, dot with q
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+            float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+            for (int c32 = 0; c32 < 64; c32 += 32) {
+                float a[32], bv[32];
+                tmem_ld32x2(tbase + c32, tbase + 64 + c32, a, bv);
+                const float4 *cs = reinterpret_cast<const float4 *>(p.rope_cos + static_cast<int64_t>(t) * 64 + c32);
+                const float4 *sn = reinterpret_cast<const float4 *>(p.rope_sin + static_cast<int64_t>(t) * 64 + c32);
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 cv = __ldg(cs + i4), sv = __ldg(sn + i4);
+                    const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+                    const float ss[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = i4 * 4 + e;
+                        const float x0 = a[i], x1 = bv[i];
+                        a[i] = bf16_round(__fmaf_rn(x0, cc[e], -__fmul_rn(x1, ss[e])));
+                        bv[i] = bf16_round(__fmaf_rn(x1, cc[e], __fmul_rn(x0, ss[e])));
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const float *qg = q_s + g * kHeadDim + c32;
+                    float acc = sc[g];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc = fmaf(qg[i], a[i], fmaf(qg[64 + i], bv[i], acc));
+                    sc[g] = acc;
+                }
+            }
+            // V rows to shared memory as bf16
+#pragma unroll 1
+            for (int c32 = 0; c32 < 64; c32 += 32) {
+                float a[32], bv[32];
+                tmem_ld32x2(tbase + kHeadDim + c32, tbase + kHeadDim + 64 + c32, a, bv);
+                uint4 *va = reinterpret_cast<uint4 *>(v_s + row * kVStride + c32);
+                uint4 *vb = reinterpret_cast<uint4 *>(v_s + row * kVStride + 64 + c32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    va[v] = make_uint4(pack_bf16x2(a[8 * v + 0], a[8 * v + 1]), pack_bf16x2(a[8 * v + 2], a[8 * v + 3]),
+                                       pack_bf16x2(a[8 * v + 4], a[8 * v + 5]), pack_bf16x2(a[8 * v + 6], a[8 * v + 7]));
+                    vb[v] = make_uint4(pack_bf16x2(bv[8 * v + 0], bv[8 * v + 1]), pack_bf16x2(bv[8 * v + 2], bv[8 * v + 3]),
+                                       pack_bf16x2(bv[8 * v + 4], bv[8 * v + 5]), pack_bf16x2(bv[8 * v + 6], bv[8 * v + 7]));
+                }
+            }
+            // Accumulator read out: the next tile's MMAs may start.
+            tc_fence_before();
+            mbar_arrive(acc_empty);
+            // (C) the tile's maximum and weights per head
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float m = sc[g];
+#pragma unroll
+                for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
+                if (lane == 0) red[quarter * 4 + g] = m;
+            }
+            named_sync(1, 128);
+            float M[4], pw[4];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                M[g] = fmaxf(fmaxf(red[g], red[4 + g]), fmaxf(red[8 + g], red[12 + g]));
+                pw[g] = fast_exp2(sc[g] - M[g]);
+            }
+            *reinterpret_cast<float4 *>(p_s + row * 4) = make_float4(pw[0], pw[1], pw[2], pw[3]);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float l = pw[g];
+#pragma unroll
+                for (int k = 16; k > 0; k >>= 1) l += __shfl_xor_sync(0xffffffffu, l, k);
+                if (lane == 0) red[16 + quarter * 4 + g] = l;
+            }
+            named_sync(1, 128);
+            // (D) thread `row` takes channel `row`: o[g] = sum_t p[t][g] v[t][row]
+            float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 8
+            for (int tt = 0; tt < kBM; ++tt) {
+                const float4 pv = *reinterpret_cast<const float4 *>(p_s + tt * 4);
+                const float v = bf16_bits_to_float(v_s[tt * kVStride + row]);
+                o[0] = fmaf(pv.x, v, o[0]);
+                o[1] = fmaf(pv.y, v, o[1]);
+                o[2] = fmaf(pv.z, v, o[2]);
+                o[3] = fmaf(pv.w, v, o[3]);
+            }
+            const int blk = c.t0 / kBM;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                if (g >= p.gqa) break;
+                const int64_t pi = (static_cast<int64_t>(c.b) * Hq + hq0 + g) * n_blk + blk;
+                p.o_part[pi * kHeadDim + row] = o[g];
+                if (row == 0) {
+                    const float L = (red[16 + g] + red[20 + g]) + (red[24 + g] + red[28 + g]);
+                    p.ml[pi] = make_float2(M[g], L);
+                }
+            }
+            named_sync(1, 128);  // q_s, p_s, v_s are free for the next tile
+        }
     } else {
         // ------------------------------ epilogue ----------------------------------
         // Drain the accumulator into a swizzled bf16 staging tile (RoPE on K
@@ -634,6 +801,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// One CTA of 128 threads per (query head, sequence): the fused kernel's
+// per-tile partials combined into the output.
+__global__ void __launch_bounds__(128) remat_merge_kernel(const float *o_part, const float2 *ml, int n_blk,
+                                                          float *out) {
+    __shared__ float s_max;
+    const int64_t row = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+    float M, o, l;
+    combine_partials(o_part, ml, row * n_blk * kHeadDim, kHeadDim, row * n_blk, 1, n_blk, &s_max, M, o, l);
+    out[row * kHeadDim + threadIdx.x] = (l > 0.0f) ? o / l : 0.0f;
+}
+
 // cos/sin(p * theta^(-2i/D)) in float64, rounded once to fp32.
 __global__ void rope_tables_kernel(float *c, float *s, int n_pos, int half, double theta) {
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -676,6 +854,28 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uin
     return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+namespace {
+
+// One persistent CTA per SM (at most one per tile).
+template <bool FUSED>
+kvq_status launch_remat_grid(const CUtensorMap &tm_w, const CUtensorMap &tm_x, const CUtensorMap &tm_k,
+                             const CUtensorMap &tm_v, const RematParams &p, cudaStream_t stream) {
+    if (cudaFuncSetAttribute(remat_kernel<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+    if (tiles >= (1LL << 31)) return KVQ_ERR_UNSUPPORTED;
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+    remat_kernel<FUSED><<<grid, kThreads, kSmemBytes, stream>>>(tm_w, tm_x, tm_k, tm_v, p);
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 }  // namespace
@@ -727,17 +927,55 @@ kvq_status launch_remat(const kvq_cache_desc &x, const void *w_kv, int n_kv_head
     p.n_tiles = n_kv_heads;
     p.timeout_ns = debug_hooks().wait_timeout_ns;
     p.status = x.status;
-    if (cudaFuncSetAttribute(remat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+    return launch_remat_grid<false>(tm_w, tm_x, tm_k, tm_v, p, stream);
+}
+
+size_t remat_attention_workspace(int batch, int num_q_heads, int ctx_len) {
+    const size_t rows = static_cast<size_t>(batch) * num_q_heads * (ctx_len / kBM);
+    return rows * (kHeadDim * sizeof(float) + sizeof(float2));
+}
+
+kvq_status launch_remat_attention(const kvq_cache_desc &x, const void *w_kv, int n_kv_heads,
+                                  const float *rope_cos, const float *rope_sin, int batch, int ctx_len,
+                                  const void *q, kvq_dtype q_dtype, int num_q_heads, float softmax_scale,
+                                  float *out, void *workspace, cudaStream_t stream) {
+    const int XH = x.num_kv_heads;
+    const int64_t hidden = static_cast<int64_t>(XH) * kHeadDim;
+    const int64_t n_rows = 2LL * n_kv_heads * kHeadDim;
+    const int64_t code_rows = static_cast<int64_t>(x.num_seqs) * XH * x.capacity_tokens;
+    if (code_rows >= (1LL << 31) || n_rows >= (1LL << 31)) return KVQ_ERR_UNSUPPORTED;
+    // W in boxes of 64 hidden channels x 128 rows: a head's K rows and its V
+    // rows make one 256-row B tile.
+    CUtensorMap tm_w, tm_x;
+    if (!make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_kv, hidden, n_rows, hidden * 2,
+                     kBK, kHeadDim, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, x.k_codes, kHeadDim / 2, code_rows,
+                     kHeadDim / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
         return KVQ_ERR_CUDA;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return KVQ_ERR_CUDA;
-    const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
-    if (tiles >= (1LL << 31)) return KVQ_ERR_UNSUPPORTED;
-    const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
-    remat_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_w, tm_x, tm_k, tm_v, p);
+    RematParams p{};
+    p.x_sz = static_cast<const __half2 *>(x.k_sz);
+    p.rope_cos = rope_cos;
+    p.rope_sin = rope_sin;
+    p.XH = XH;
+    p.H = n_kv_heads;
+    p.Tc = x.capacity_tokens;
+    p.T = ctx_len;
+    p.m_tiles = batch * (ctx_len / kBM);
+    p.n_tiles = n_kv_heads;
+    p.timeout_ns = debug_hooks().wait_timeout_ns;
+    p.status = x.status;
+    p.q = q;
+    p.q_dtype = q_dtype;
+    p.gqa = num_q_heads / n_kv_heads;
+    p.qscale = softmax_scale * 1.4426950408889634f;
+    const int n_blk = ctx_len / kBM;
+    const size_t rows = static_cast<size_t>(batch) * num_q_heads * n_blk;
+    p.o_part = static_cast<float *>(workspace);
+    p.ml = reinterpret_cast<float2 *>(static_cast<uint8_t *>(workspace) + rows * kHeadDim * sizeof(float));
+    // the store maps are unused by the fused kernel; any valid map fills the slots
+    kvq_status s = launch_remat_grid<true>(tm_w, tm_x, tm_w, tm_w, p, stream);
+    if (s != KVQ_OK) return s;
+    remat_merge_kernel<<<dim3(num_q_heads, batch), 128, 0, stream>>>(p.o_part, p.ml, n_blk, out);
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

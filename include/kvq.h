@@ -24,6 +24,10 @@
  *                         X with a tensor-core GEMM, RoPE on K. "XQuant:
  *                         Breaking the Memory Wall for LLM Inference with KV
  *                         Cache Rematerialization", Abstract.
+ * and their compositions: kvq_remat_attention (the remat GEMM with decode
+ * attention in its epilogue, K and V never stored), kvq_decode_merge_partial
+ * and kvq_merge_partials (decode over token ranges held by several caches,
+ * e.g. one per GPU).
  *
  * Conventions for every call:
  *   - The caller owns all memory. Pointers named d_* or documented "device" are
@@ -326,6 +330,31 @@ KVQ_API kvq_status kvq_remat_kv(const kvq_cache_desc *x_cache, const void *w_kv,
                         int32_t n_kv_heads, const float *rope_cos,
                         const float *rope_sin, int32_t batch, int32_t ctx_len,
                         void *k_out, void *v_out, void *stream);
+
+/*
+ * kvq_remat_attention -- rematerialization fused with decode attention
+ * ("XQuant: Breaking the Memory Wall for LLM Inference with KV Cache
+ * Rematerialization", Abstract: K and V are recomputed from the cached X
+ * instead of being cached). Same arguments and requirements as kvq_remat_kv
+ * for the X cache, W and the RoPE tables, and K, V are the same values
+ * (fp32 accumulation, RoPE on K, rounded to bf16), but they never leave the
+ * chip: each 128-token tile of a head's K and V, held in tensor memory, is
+ * scored against the head's GQA query rows at once, and
+ *     out[b][h] = sum_t softmax_t(softmax_scale * q[b][h] . k_t) v_t
+ * over all t < ctx_len (no rotation; queries as given). q: device
+ * [batch][num_q_heads][128] of q_dtype, num_q_heads / n_kv_heads in {1, 2, 4}.
+ * out: device fp32 [batch][num_q_heads][128]. workspace: device, at least
+ * kvq_remat_attention_workspace_size(batch, num_q_heads, ctx_len) bytes
+ * (per 128-token tile and query head a partial of 130 floats), else
+ * KVQ_ERR_CAPACITY. ctx_len a multiple of 128; batch <= 65535.
+ */
+KVQ_API size_t kvq_remat_attention_workspace_size(int32_t batch, int32_t num_q_heads, int32_t ctx_len);
+KVQ_API kvq_status kvq_remat_attention(const kvq_cache_desc *x_cache, const void *w_kv,
+                                       int32_t n_kv_heads, const float *rope_cos,
+                                       const float *rope_sin, int32_t batch, int32_t ctx_len,
+                                       const void *q, kvq_dtype q_dtype, int32_t num_q_heads,
+                                       float softmax_scale, float *out, void *workspace,
+                                       size_t workspace_bytes, void *stream);
 
 /* kvq_rope_tables -- cos and sin tables fp32 [n_pos][head_dim/2]:
  * fp32 of cos/sin(p * theta^(-2i/head_dim)) evaluated in float64 on the

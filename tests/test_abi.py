@@ -128,6 +128,20 @@ def test_remat_and_rope_validation(K):
     assert call(ctypes.byref(_desc(K, num_kv_heads=32, hadamard_block_k=128, v_codes=None)),
                 FAKE, 8, FAKE, FAKE, 2, 128, FAKE, FAKE, None) == K.ERR_UNSUPPORTED
     assert call(ctypes.byref(x), None, 8, FAKE, FAKE, 2, 128, FAKE, FAKE, None) == K.ERR_INVALID_ARG
+    fused = K.lib().kvq_remat_attention
+    ws = K.lib().kvq_remat_attention_workspace_size(2, 32, 1024)
+    assert ws == 2 * 32 * 8 * (128 * 4 + 8)
+    assert K.lib().kvq_remat_attention_workspace_size(2, 32, 1000) == 0
+    args = lambda **kw: [kw.get(n, d) for n, d in (("w", FAKE), ("h", 8), ("c", FAKE), ("s", FAKE), ("b", 2),
+                                                  ("t", 1024), ("q", FAKE), ("qd", 0), ("hq", 32),
+                                                  ("sc", 0.088), ("o", FAKE), ("ws", FAKE), ("wb", ws))]
+    xb = _desc(K, num_kv_heads=32, hadamard_block_k=0, v_codes=None, v_sz=None, bits_v=0, capacity_tokens=1024)
+    assert fused(ctypes.byref(xb), *args(t=1000), None) == K.ERR_INVALID_ARG        # not whole tiles
+    assert fused(ctypes.byref(xb), *args(hq=24), None) == K.ERR_UNSUPPORTED         # GQA 3
+    assert fused(ctypes.byref(xb), *args(hq=30), None) == K.ERR_INVALID_ARG         # not a multiple
+    assert fused(ctypes.byref(xb), *args(q=None), None) == K.ERR_INVALID_ARG
+    assert fused(ctypes.byref(xb), *args(qd=7), None) == K.ERR_INVALID_ARG
+    assert fused(ctypes.byref(xb), *args(wb=ws - 1), None) == K.ERR_CAPACITY
     assert K.lib().kvq_rope_tables(FAKE, FAKE, 0, 128, 500000.0, None) == K.ERR_INVALID_ARG
     assert K.lib().kvq_rope_tables(FAKE, FAKE, 16, 127, 500000.0, None) == K.ERR_INVALID_ARG
 

@@ -195,6 +195,34 @@ def test_attention_over_rematerialized_kv():
         assert_close(out[b], want, "seq %d" % b)
 
 
+@pytest.mark.parametrize("HQ,q_dtype", [(32, "bf16"), (16, "fp32"), (8, "fp16")])
+def test_fused_remat_attention(HQ, q_dtype):
+    # K and V rematerialized in tensor memory and attended in the GEMM's
+    # epilogue, never stored: the oracle's attention over its own
+    # rematerialized, bf16-rounded K/V, and the unfused path's output
+    B, T, hidden, H = 2, 1024, 1024, 8
+    xs, w = _inputs(31 + HQ, B, T, hidden, H)
+    cache = _x_cache(xs, T)
+    g = np.random.default_rng(32 + HQ)
+    q = W.finish(W.normal(g, (B, HQ, D)), q_dtype)
+    cos, sin = K.rope_tables(T, D, THETA)
+    wd = dev(w, "bf16")
+    qd = dev(q, q_dtype)
+    out = K.remat_attention(cache.desc, wd, H, cos, sin, B, T, qd, SCALE).cpu().numpy()
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    k_out, v_out = _remat(cache, w, H, B, T)
+    unfused = K.decode_attention(K.bf16_cache_desc(k_out, v_out), qd, lens_tensor([T] * B), T,
+                                 SCALE).cpu().numpy()
+    for b in range(B):
+        ek, ev, _, _ = _oracle_kv(xs[b], w, H, np.arange(T))
+        kh = _to_bf16(ek).transpose(1, 0, 2)
+        vh = _to_bf16(ev).transpose(1, 0, 2)
+        want = oracle.decode_attention_gqa(q[b].astype(np.float64), kh, vh, SCALE)
+        assert_close(out[b], want, "fused seq %d" % b)
+        assert_close(out[b], unfused[b], "fused vs unfused seq %d" % b)
+
+
 def test_xquant_full_size_sampled():
     # 8 sequences x 16384 positions, hidden 4096 (32 X heads), 8 KV heads:
     # the full GEMM runs; sampled tokens are compared channel by channel, and
