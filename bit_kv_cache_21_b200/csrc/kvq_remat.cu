@@ -604,13 +604,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 q_s[idx] = v * p.qscale;
             }
             named_sync(1, 128);
-            // (B) scores of this token: RoPE on K (pairs i, i + 64), bf16, dot with q
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+            // V rows to shared memory as bf16 (first, so the accumulator is
+            // released right after the last K load)
+#pragma unroll 1
+            for (int c32 = 0; c32 < 64; c32 += 32) {
+                float a[32], bv[32];
+                tmem_ld32x2(tbase + kHeadDim + c32, tbase + kHeadDim + 64 + c32, a, bv);
+                uint4 *va = reinterpret_cast<uint4 *>(v_s + row * kVStride + c32);
+                uint4 *vb = reinterpret_cast<uint4 *>(v_s + row * kVStride + 64 + c32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    va[v] = make_uint4(pack_bf16x2(a[8 * v + 0], a[8 * v + 1]), pack_bf16x2(a[8 * v + 2], a[8 * v + 3]),
+                                       pack_bf16x2(a[8 * v + 4], a[8 * v + 5]), pack_bf16x2(a[8 * v + 6], a[8 * v + 7]));
+                    vb[v] = make_uint4(pack_bf16x2(bv[8 * v + 0], bv[8 * v + 1]), pack_bf16x2(bv[8 * v + 2], bv[8 * v + 3]),
+                                       pack_bf16x2(bv[8 * v + 4], bv[8 * v + 5]), pack_bf16x2(bv[8 * v + 6], bv[8 * v + 7]));
+                }
+            }
+            // (B) scores of this token: RoPE on K (pairs i, i + 64), bf16, dot with q
             float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
             for (int c32 = 0; c32 < 64; c32 += 32) {
                 float a[32], bv[32];
                 tmem_ld32x2(tbase + c32, tbase + 64 + c32, a, bv);
+                if (c32 == 32) {  // the last tensor-memory read: the next tile's MMAs may start
+                    tc_fence_before();
+                    mbar_arrive(acc_empty);
+                }
                 const float4 *cs = reinterpret_cast<const float4 *>(p.rope_cos + static_cast<int64_t>(t) * 64 + c32);
                 const float4 *sn = reinterpret_cast<const float4 *>(p.rope_sin + static_cast<int64_t>(t) * 64 + c32);
 #pragma unroll
@@ -635,24 +655,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sc[g] = acc;
                 }
             }
-            // V rows to shared memory as bf16
-#pragma unroll 1
-            for (int c32 = 0; c32 < 64; c32 += 32) {
-                float a[32], bv[32];
-                tmem_ld32x2(tbase + kHeadDim + c32, tbase + kHeadDim + 64 + c32, a, bv);
-                uint4 *va = reinterpret_cast<uint4 *>(v_s + row * kVStride + c32);
-                uint4 *vb = reinterpret_cast<uint4 *>(v_s + row * kVStride + 64 + c32);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    va[v] = make_uint4(pack_bf16x2(a[8 * v + 0], a[8 * v + 1]), pack_bf16x2(a[8 * v + 2], a[8 * v + 3]),
-                                       pack_bf16x2(a[8 * v + 4], a[8 * v + 5]), pack_bf16x2(a[8 * v + 6], a[8 * v + 7]));
-                    vb[v] = make_uint4(pack_bf16x2(bv[8 * v + 0], bv[8 * v + 1]), pack_bf16x2(bv[8 * v + 2], bv[8 * v + 3]),
-                                       pack_bf16x2(bv[8 * v + 4], bv[8 * v + 5]), pack_bf16x2(bv[8 * v + 6], bv[8 * v + 7]));
-                }
-            }
-            // Accumulator read out: the next tile's MMAs may start.
-            tc_fence_before();
-            mbar_arrive(acc_empty);
             // (C) the tile's maximum and weights per head
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
