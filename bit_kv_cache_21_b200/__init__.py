@@ -16,3 +16,4 @@ from ._binding import (  # noqa: F401
     remat_kv, remat_attention, rope_tables, debug_set, version,
 )
 from .cache import CacheSpec, KVCache, bf16_cache_desc, sink_view  # noqa: F401
+from .graph import DecodeStep  # noqa: F401

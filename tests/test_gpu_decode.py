@@ -206,3 +206,43 @@ def test_decode_randomized_hadamard(hb, gqa):
     assert cache.device_status() == 0
     for s_, T in enumerate(lens):
         assert_close(out[s_], oracle_decode_tokens(ks[s_], vs[s_], q[s_], spec, signs=signs), "seq %d" % s_)
+
+
+def test_decode_step_graph_replays_the_eager_step():
+    # the CUDA-graph step (uploads, append, decode, download) gives the eager
+    # calls' results bit for bit, step after step, and advances the lengths
+    import workloads as W
+    S, H, Hq, T0, steps = 3, 2, 8, 300, 4
+    g = np.random.default_rng(77)
+    ch = W.outlier_channels(g)
+    hist_k = W.finish(W.keys(g, (S, T0 + steps, H, D), ch), "bf16")
+    hist_v = W.finish(W.normal(g, (S, T0 + steps, H, D)), "bf16")
+    qs = W.finish(W.normal(g, (steps, S, Hq, D)), "bf16")
+    caches, lens = [], []
+    for _ in range(2):
+        c = K.KVCache(K.CacheSpec(S, H, bits_k=4, bits_v=4, group_k=128, group_v=128, hadamard_block_k=128,
+                                  capacity_tokens=384))
+        sl = lens_tensor([0] * S)
+        append(c, [hist_k[s, :T0] for s in range(S)], [hist_v[s, :T0] for s in range(S)], sl)
+        caches.append(c)
+        lens.append(sl)
+    cu_one = torch.arange(0, S + 1, dtype=torch.int32, device="cuda")
+    hk = torch.empty((S, H, D), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    hq = torch.empty((S, Hq, D), dtype=torch.bfloat16).pin_memory()
+    step = K.DecodeStep(caches[1].desc, lens[1], cu_one, 384, SCALE, hk, hv, hq)
+    for i in range(steps):
+        kk = torch.from_numpy(hist_k[:, T0 + i]).to(torch.bfloat16)
+        vv = torch.from_numpy(hist_v[:, T0 + i]).to(torch.bfloat16)
+        qq = torch.from_numpy(qs[i]).to(torch.bfloat16)
+        K.quantize_append(caches[0].desc, kk.cuda(), vv.cuda(), cu_one, lens[0])
+        want = K.decode_attention(caches[0].desc, qq.cuda(), lens[0], 384, SCALE).cpu()
+        hk.copy_(kk)
+        hv.copy_(vv)
+        hq.copy_(qq)
+        step.run()
+        torch.cuda.synchronize()
+        assert torch.equal(step.out_host, want), i
+        assert lens[1].tolist() == [T0 + i + 1] * S
+    assert torch.equal(caches[0].k_codes, caches[1].k_codes) and torch.equal(caches[0].v_sz, caches[1].v_sz)
+    assert caches[1].device_status() == 0
