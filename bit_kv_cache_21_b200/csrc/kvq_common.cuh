@@ -170,31 +170,61 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // Log-sum-exp combination of n partials (o_j, m_j, l_j) of one (sequence,
-// query head) by a CTA of 128 threads (channel d each): partial j's o row at
-// o_part + o0 + j * o_step (kHeadDim floats), its (m, l) at ml[m0 + j * m_step].
-// o = sum_j e_j o_j, l = sum_j e_j l_j with e_j = 2^(m_j - M), M = max_j m_j
-// (log2 units). Partials with m = -inf (no tokens) weigh 0.
+// query head) by a CTA of 128 * NG threads: thread t takes channel t % 128
+// and the partials j = t / 128 (mod NG), so NG groups walk the partials side
+// by side. Partial j's o row is at o_part + o0 + j * o_step (kHeadDim floats),
+// its (m, l) at ml[m0 + j * m_step]. o = sum_j e_j o_j, l = sum_j e_j l_j with
+// e_j = 2^(m_j - M), M = max_j m_j (log2 units); partials with m = -inf (no
+// tokens) weigh 0. The groups' sums are added in group order. Results are
+// valid in the threads of group 0 (t < 128).
+template <int NG>
+struct CombineSmem {
+    float o[NG][kHeadDim];
+    float l[NG];
+    float red[NG * 4];
+    float max;
+};
+
+template <int NG>
 __device__ __forceinline__ void combine_partials(const float *o_part, const float2 *ml, int64_t o0,
                                                  int64_t o_step, int64_t m0, int64_t m_step, int n,
-                                                 float *s_max, float &M, float &o, float &l) {
-    const int d = threadIdx.x;
-    if (d < 32) {  // maximum over the partials, one warp
-        float m = -INFINITY;
-        for (int j = d; j < n; j += 32) m = fmaxf(m, ml[m0 + j * m_step].x);
+                                                 CombineSmem<NG> &sm, float &M, float &o, float &l) {
+    const int t = threadIdx.x, d = t & (kHeadDim - 1), grp = t / kHeadDim;
+    float m = -INFINITY;
+    for (int j = t; j < n; j += NG * kHeadDim) m = fmaxf(m, ml[m0 + j * m_step].x);
 #pragma unroll
-        for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
-        if (d == 0) *s_max = m;
+    for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
+    if ((t & 31) == 0) sm.red[t >> 5] = m;
+    __syncthreads();
+    if (t == 0) {
+        float mm = sm.red[0];
+        for (int w = 1; w < NG * 4; ++w) mm = fmaxf(mm, sm.red[w]);
+        sm.max = mm;
     }
     __syncthreads();
-    M = *s_max;
-    o = 0.0f;
-    l = 0.0f;
+    M = sm.max;
+    float oo = 0.0f, ll = 0.0f;
 #pragma unroll 4
-    for (int j = 0; j < n; ++j) {
+    for (int j = grp; j < n; j += NG) {
         const float2 v = ml[m0 + j * m_step];
         const float e = (v.x == -INFINITY) ? 0.0f : fast_exp2(v.x - M);
-        o = fmaf(e, o_part[o0 + j * o_step + d], o);
-        l = fmaf(e, v.y, l);
+        oo = fmaf(e, o_part[o0 + j * o_step + d], oo);
+        ll = fmaf(e, v.y, ll);
+    }
+    if constexpr (NG == 1) {
+        o = oo;
+        l = ll;
+    } else {
+        sm.o[grp][d] = oo;
+        if (d == 0) sm.l[grp] = ll;
+        __syncthreads();
+        o = sm.o[0][d];
+        l = sm.l[0];
+#pragma unroll
+        for (int g = 1; g < NG; ++g) {
+            o += sm.o[g][d];
+            l += sm.l[g];
+        }
     }
 }
 

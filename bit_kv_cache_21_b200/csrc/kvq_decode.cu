@@ -14,19 +14,23 @@ namespace {
 // of the same sequences. Launched as a programmatic dependent of the split-K
 // pass: its CTAs may start while that pass drains and wait here until its
 // partials are complete.
+constexpr int kMergeGroups = 4;  // partial groups per merge CTA (128 threads each)
+
 template <bool PARTIAL>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const float *o_part, const float2 *ml,
+__global__ void __launch_bounds__(128 * kMergeGroups) decode_merge_kernel(const float *o_part, const float2 *ml,
                                                            const int32_t *seq_lens, float *out,
                                                            float2 *out_ml, int Hq, int n_split,
                                                            int chunk, int max_seq_len) {
-    __shared__ float s_max;
+    __shared__ CombineSmem<kMergeGroups> sm;
     pdl_wait_prior_grid();
     const int hq = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
     const int T = min(__ldg(seq_lens + seq), max_seq_len);
     const int nv = T > 0 ? (T + chunk - 1) / chunk : 0;
     const int64_t row = static_cast<int64_t>(seq) * Hq + hq;
     float M, o, l;
-    combine_partials(o_part, ml, row * n_split * kHeadDim, kHeadDim, row * n_split, 1, nv, &s_max, M, o, l);
+    combine_partials<kMergeGroups>(o_part, ml, row * n_split * kHeadDim, kHeadDim, row * n_split, 1, nv, sm, M,
+                                   o, l);
+    if (d >= kHeadDim) return;
     if constexpr (PARTIAL) {
         out[row * kHeadDim + d] = o;
         if (d == 0) out_ml[row] = make_float2(M, l);
@@ -40,12 +44,12 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *o_part, 
 // pairs, parts back to back (rows * (kHeadDim + 2) floats each).
 __global__ void __launch_bounds__(128) merge_partials_kernel(const float *parts, int n_part, int rows,
                                                              float *out) {
-    __shared__ float s_max;
+    __shared__ CombineSmem<1> sm;
     const int64_t row = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
     const int64_t part = static_cast<int64_t>(rows) * (kHeadDim + 2);  // floats per part
     const float2 *ml = reinterpret_cast<const float2 *>(parts + static_cast<int64_t>(rows) * kHeadDim);
     float M, o, l;
-    combine_partials(parts, ml, row * kHeadDim, part, row, part / 2, n_part, &s_max, M, o, l);
+    combine_partials<1>(parts, ml, row * kHeadDim, part, row, part / 2, n_part, sm, M, o, l);
     out[row * kHeadDim + threadIdx.x] = (l > 0.0f) ? o / l : 0.0f;
 }
 
@@ -143,7 +147,7 @@ kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, 
         reinterpret_cast<const float2 *>(static_cast<const uint8_t *>(workspace) + plan.ws_part);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(num_q_heads, num_seqs);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(128 * kMergeGroups);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

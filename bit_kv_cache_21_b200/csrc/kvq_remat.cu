@@ -805,13 +805,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // One CTA of 128 threads per (query head, sequence): the fused kernel's
 // per-tile partials combined into the output.
-__global__ void __launch_bounds__(128) remat_merge_kernel(const float *o_part, const float2 *ml, int n_blk,
+__global__ void __launch_bounds__(512) remat_merge_kernel(const float *o_part, const float2 *ml, int n_blk,
                                                           float *out) {
-    __shared__ float s_max;
+    __shared__ CombineSmem<4> sm;
     const int64_t row = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
     float M, o, l;
-    combine_partials(o_part, ml, row * n_blk * kHeadDim, kHeadDim, row * n_blk, 1, n_blk, &s_max, M, o, l);
-    out[row * kHeadDim + threadIdx.x] = (l > 0.0f) ? o / l : 0.0f;
+    combine_partials<4>(o_part, ml, row * n_blk * kHeadDim, kHeadDim, row * n_blk, 1, n_blk, sm, M, o, l);
+    if (threadIdx.x < kHeadDim) out[row * kHeadDim + threadIdx.x] = (l > 0.0f) ? o / l : 0.0f;
 }
 
 // cos/sin(p * theta^(-2i/D)) in float64, rounded once to fp32.
@@ -977,7 +977,7 @@ kvq_status launch_remat_attention(const kvq_cache_desc &x, const void *w_kv, int
     // the store maps are unused by the fused kernel; any valid map fills the slots
     kvq_status s = launch_remat_grid<true>(tm_w, tm_x, tm_w, tm_w, p, stream);
     if (s != KVQ_OK) return s;
-    remat_merge_kernel<<<dim3(num_q_heads, batch), 128, 0, stream>>>(p.o_part, p.ml, n_blk, out);
+    remat_merge_kernel<<<dim3(num_q_heads, batch), 512, 0, stream>>>(p.o_part, p.ml, n_blk, out);
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
