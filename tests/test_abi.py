@@ -112,6 +112,22 @@ def test_decode_validation(K):
     assert _decode(K, d, scale=float("nan")) == K.ERR_INVALID_ARG
 
 
+def test_partial_merge_validation(K):
+    d = _desc(K)
+    mp = K.lib().kvq_decode_merge_partial
+    ws = K.decode_workspace_size(d, 2, 32, 512)
+    assert mp(ctypes.byref(d), 32, FAKE, 2, 512, None, FAKE, FAKE, ws, None) == K.ERR_INVALID_ARG
+    assert mp(ctypes.byref(d), 32, FAKE, 2, 512, FAKE, FAKE + 4, FAKE, ws, None) == K.ERR_INVALID_ARG
+    assert mp(ctypes.byref(d), 32, FAKE, 2, 512, FAKE, FAKE, FAKE, 16, None) == K.ERR_CAPACITY
+    assert mp(ctypes.byref(d), 0, FAKE, 2, 512, FAKE, FAKE, FAKE, ws, None) == K.ERR_INVALID_ARG
+    mg = K.lib().kvq_merge_partials
+    assert mg(None, 2, 2, 32, FAKE, None) == K.ERR_INVALID_ARG
+    assert mg(FAKE + 8, 2, 2, 32, FAKE, None) == K.ERR_INVALID_ARG         # parts not 16-byte aligned
+    assert mg(FAKE, 0, 2, 32, FAKE, None) == K.ERR_INVALID_ARG
+    assert mg(FAKE, 2, 70000, 32, FAKE, None) == K.ERR_INVALID_ARG         # grid limit on sequences
+    assert mg(FAKE, 2, 2, 32, None, None) == K.ERR_INVALID_ARG
+
+
 def test_workspace_size(K):
     d = _desc(K)
     ws = K.decode_workspace_size(d, 2, 32, 512)
