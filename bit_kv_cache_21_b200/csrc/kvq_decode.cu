@@ -1,6 +1,12 @@
 // kvq_decode.cu -- decode attention entry: the split plan, the choice of the
-// split-K variant family, and the log-sum-exp merge of the splits. The split-K
-// kernel itself is kvq_decode_kernel.cuh, instantiated by kvq_decode_*.cu.
+// split-K variant family, and the log-sum-exp merges (of the splits, and of
+// partials from caches that hold other token ranges of the same sequences).
+// The split-K kernel itself is kvq_decode_kernel.cuh, a template over GQA, the
+// key mode (token-wise groups, KIVI's per-channel blocks, bf16), the value
+// mode (token-wise groups, groups along tokens = one scale/zero per channel
+// and R-token block, bf16), the code widths, compile-time group sizes and the
+// item's bf16 tail (none, the recent window, the attention sinks); each family
+// is instantiated in its own unit (kvq_decode_plain/window/innerq/sink.cu).
 #include "kvq_decode_kernel.cuh"
 
 namespace kvq {

@@ -26,6 +26,10 @@
 //               fp32 on K, round to bf16 into a swizzled shared staging tile,
 //               release the accumulator; one thread stores the tile to
 //               [B][H][T][128] with TMA while the next tile's main loop runs.
+// The fused variant (remat_kernel<true>, kvq_remat_attention) builds each
+// tile from one head's K rows and V rows and replaces the stores by decode
+// attention of the head's GQA query rows over the tile's 128 tokens, writing
+// one (o, m, l) partial per tile; remat_merge_kernel combines the tiles.
 // Every mbarrier wait is bounded; on expiry the kernel sets KVQ_DEV_TIMEOUT,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
 #include <cuda.h>
