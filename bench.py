@@ -569,6 +569,41 @@ def run_long_int2_sharded(args, dev, rank, world):
             "attention_GBps": nbytes / (ms * 1e-3) / 1e9}
 
 
+def run_append_hybrid(args, dev):
+    """Bulk append of the llama8b-layer prefill (16 x 8192 tokens x 8 KV heads,
+    K and V, bf16, INT4 g128, Hadamard(128) on K, x20 outlier key channels),
+    plain and with InnerQ's hybrid groups; the mean of 3 timed appends after
+    one warm-up, CUDA events."""
+    import torch
+    import bit_kv_cache_21_b200 as K
+    S, H, T = 16, 8, 8192
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2)
+    k, v = _synthetic_kv(gen, S * T, H, dev, torch, 2)
+    cu = torch.arange(0, (S + 1) * T, T, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for hyb in (False, True):
+        cache = K.KVCache(K.CacheSpec(S, H, bits_k=4, bits_v=4, group_k=128, group_v=128,
+                                      hadamard_block_k=128, capacity_tokens=T, hybrid=hyb), device=dev)
+        ms = []
+        for rep in range(4):
+            lens = torch.zeros(S, dtype=torch.int32, device=dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            K.quantize_append(cache.desc, k, v, cu, lens)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if rep > 0:
+                ms.append(e0.elapsed_time(e1))
+        assert cache.device_status() == 0
+        res["hybrid" if hyb else "plain"] = {"ms": statistics.mean(ms),
+                                             "tokens_per_s": S * T / (statistics.mean(ms) * 1e-3)}
+        del cache
+    return {"workload": "bulk prefill 16 x 8192 tokens x 8 KV heads, K and V, bf16, INT4 g128, "
+                        "Hadamard(128) K, plain and hybrid groups", **res}
+
+
 def _sweep_setup(dev, seed=6):
     """Shared data of the accuracy/cost sweeps: 16 seqs x 8 KV heads (32 q
     heads) x 4096 tokens of the outlier-key recipe, bf16, and decode attention
@@ -819,10 +854,10 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--part", default="all",
                     choices=["all", "decode", "remat", "long_int2", "paged_mix", "rotation_sweep",
-                             "grouping_sweep", "long_int2_sharded"],
+                             "grouping_sweep", "long_int2_sharded", "append_hybrid"],
                     help="run one leg alone: decode (the metric's step), remat, long_int2, "
-                         "paged_mix, rotation_sweep, grouping_sweep or long_int2_sharded (all "
-                         "but decode print their own line)")
+                         "paged_mix, rotation_sweep, grouping_sweep, long_int2_sharded or "
+                         "append_hybrid (all but decode print their own line)")
     ap.add_argument("--remat-batch", type=int, default=8)
     ap.add_argument("--remat-steps", type=int, default=10)
     args = ap.parse_args()
@@ -869,6 +904,19 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    if args.part == "append_hybrid":
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        leg = run_append_hybrid(args, dev)
+        if rank == 0:
+            print(json.dumps({"metric": "quantize-append tokens/s", "value": leg["hybrid"]["tokens_per_s"],
+                              "unit": "tokens/s", "n_gpus": world, "higher_is_better": True,
+                              "data": "synthetic", "config": {"workload": leg["workload"]},
+                              args.part: leg}))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.part == "long_int2_sharded":
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
