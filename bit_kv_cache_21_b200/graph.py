@@ -49,7 +49,9 @@ class DecodeStep:
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream(dev))
         self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph, stream=side):
+        # thread-local capture: other threads of the process (a process group's
+        # watchdog, for one) may keep making CUDA calls meanwhile
+        with torch.cuda.graph(self.graph, stream=side, capture_error_mode="thread_local"):
             self._body()
         torch.cuda.current_stream(dev).wait_stream(side)
 
