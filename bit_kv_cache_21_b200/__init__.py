@@ -1,9 +1,13 @@
 """B200 (sm_100a) low-bit KV cache: INT4/INT2 quantize-append with Hadamard
-rotation, split-K decode attention over the packed cache, and XQuant-style
-K/V rematerialization on the tensor cores.
+rotation (KIVI per-channel keys, values grouped along tokens, attention sinks,
+hybrid symmetric/asymmetric groups as options), split-K decode attention over
+the packed cache (also over token ranges sharded across GPUs), and XQuant-style
+K/V rematerialization on the tensor cores, alone or fused with attention.
 
 The compute lives in libkvq.so (C ABI, include/kvq.h); this package is its
-ctypes binding plus helpers that allocate the cache buffers with torch.
+ctypes binding plus helpers that allocate the cache buffers with torch
+(`cache`), run the sharded exchange (`sharded`) and capture a decode step as a
+CUDA graph (`graph`).
 """
 from ._binding import (  # noqa: F401
     BF16, FP16, FP32, PER_TOKEN, PER_CHANNEL,
