@@ -204,9 +204,9 @@ __device__ __forceinline__ uint32_t qcode(float x, const QParams &p, float Lf) {
 // s = fp16_ru(fp32(max|x| / Qp)), z = -C s (exact in fp32; the candidate is
 // dropped when |z| exceeds the largest fp16), q = clamp(rint(x / s), -Qp, Qp) + C
 // with x / s taken as fp32(x * fp32(1/s)). It has an exact zero level. A group
-// takes it when its squared reconstruction error is smaller than the
-// asymmetric one's: fp32 e = x - fma(q, s, z), squares summed with fma in
-// element order over runs of 32 elements, run sums added pairwise.
+// takes it when its largest reconstruction error is smaller than the
+// asymmetric one's: |e| with fp32 e = x - fma(q, s, z), the maximum over the
+// group (exact, so the lanes may visit the elements in any order).
 struct SymParams {
     __half2 sz;
     float sf, zf, r;
@@ -234,10 +234,9 @@ __device__ __forceinline__ uint32_t sym_code(float x, const SymParams &p, int bi
     return static_cast<uint32_t>(__fadd_rn(t, C));
 }
 
-// Squared error of one run of codes (plain integers) against x.
-__device__ __forceinline__ float sq_err(float x, uint32_t q, float s, float z, float acc) {
-    const float e = __fsub_rn(x, __fmaf_rn(static_cast<float>(q), s, z));
-    return __fmaf_rn(e, e, acc);
+// Largest reconstruction error so far, with the element x of code q.
+__device__ __forceinline__ float max_err(float x, uint32_t q, float s, float z, float m) {
+    return fmaxf(m, fabsf(__fsub_rn(x, __fmaf_rn(static_cast<float>(q), s, z))));
 }
 
 // Codes of n consecutive elements (n even) of one group:
@@ -269,7 +268,7 @@ __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32
     constexpr int L = (1 << BITS) - 1;
     uint32_t q[32];  // 0x4B00000q
     // hybrid: replace the asymmetric codes of elements [j0, j0 + n) by the
-    // symmetric ones when the group's error sum `es` is below `ea`
+    // symmetric ones when the group's largest error `es` is below `ea`
     auto choose = [&](int j0, int n, const SymParams &ps, float ea, float es, __half2 &out_sz) {
         if (ps.ok && es < ea) {
 #pragma unroll
@@ -282,8 +281,8 @@ __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32
         es = 0.0f;
 #pragma unroll
         for (int j = j0; j < j0 + n; ++j) {
-            ea = sq_err(x[j], q[j] - 0x4B000000u, p.sf, p.zf, ea);
-            es = sq_err(x[j], sym_code(x[j], ps, BITS), ps.sf, ps.zf, es);
+            ea = max_err(x[j], q[j] - 0x4B000000u, p.sf, p.zf, ea);
+            es = max_err(x[j], sym_code(x[j], ps, BITS), ps.sf, ps.zf, es);
         }
     };
     if (G >= 32) {
@@ -301,10 +300,10 @@ __device__ __forceinline__ void quant_pack_lane(const float x[32], int G, uint32
             const SymParams ps = sym_params(mn, mx, BITS);
             float ea, es;
             run_errs(0, 32, p, ps, ea, es);
-            // the group's runs (one per lane) added pairwise: (r0 + r1) + (r2 + r3)
+            // the group's largest errors over its lanes
             for (int m = 1; m < G / 32; m <<= 1) {
-                ea += __shfl_xor_sync(0xffffffffu, ea, m);
-                es += __shfl_xor_sync(0xffffffffu, es, m);
+                ea = fmaxf(ea, __shfl_xor_sync(0xffffffffu, ea, m));
+                es = fmaxf(es, __shfl_xor_sync(0xffffffffu, es, m));
             }
             choose(0, 32, ps, ea, es, sz[0]);
         }
@@ -474,9 +473,8 @@ struct WindowParams {
 // Quantize one block of R staged bf16 rows [R][128] per channel (each
 // channel's R values one group; KIVI keys, InnerQ values) into `codes`
 // (R rows packed along channels) and `sz` ([128] half2). With `hybrid`, each
-// group takes the symmetric candidate when its squared error is smaller (runs
-// of 32 tokens, run sums added pairwise). Called by the whole CTA; `qk` is
-// [R][128] bytes of scratch.
+// group takes the symmetric candidate when its largest error is smaller.
+// Called by the whole CTA; `qk` is [R][128] bytes of scratch.
 __device__ void flush_channel_block(const uint16_t *src, uint8_t *qk, int R, int bits, int hybrid,
                                     uint8_t *codes, __half2 *sz) {
     const int L = (1 << bits) - 1;
@@ -493,24 +491,13 @@ __device__ void flush_channel_block(const uint16_t *src, uint8_t *qk, int R, int
         SymParams ps{};
         if (hybrid) {
             ps = sym_params(mn, mx, bits);
-            float ra[8], rs[8];  // R <= 256: at most 8 runs of 32 tokens
-            const int n_runs = R / 32;
-            for (int r = 0; r < n_runs; ++r) {
-                float ea = 0.0f, es = 0.0f;
-                for (int t = 32 * r; t < 32 * r + 32; ++t) {
-                    const float v = bf16_bits_to_float(src[t * kHeadDim + d]);
-                    ea = sq_err(v, qcode(v, qp, Lf), qp.sf, qp.zf, ea);
-                    es = sq_err(v, sym_code(v, ps, bits), ps.sf, ps.zf, es);
-                }
-                ra[r] = ea;
-                rs[r] = es;
+            float ea = 0.0f, es = 0.0f;
+            for (int t = 0; t < R; ++t) {
+                const float v = bf16_bits_to_float(src[t * kHeadDim + d]);
+                ea = max_err(v, qcode(v, qp, Lf), qp.sf, qp.zf, ea);
+                es = max_err(v, sym_code(v, ps, bits), ps.sf, ps.zf, es);
             }
-            for (int w = 1; w < n_runs; w *= 2)
-                for (int r = 0; r + w < n_runs; r += 2 * w) {
-                    ra[r] = __fadd_rn(ra[r], ra[r + w]);
-                    rs[r] = __fadd_rn(rs[r], rs[r + w]);
-                }
-            use_sym = ps.ok && rs[0] < ra[0];
+            use_sym = ps.ok && es < ea;
         }
         for (int t = 0; t < R; ++t) {
             const float v = bf16_bits_to_float(src[t * kHeadDim + d]);

@@ -167,8 +167,8 @@ def quantize_group_hybrid(x, bits):
     """One group with InnerQ's hybrid choice (Abstract, "(i) hybrid
     quantization"): the asymmetric min/max candidate or a symmetric one with
     an exact zero level, whichever reconstructs the group with the smaller
-    squared error (the criterion is this library's reading; oracle.c states
-    it). Returns (s_bits, z_bits, codes)."""
+    largest absolute error, ties to the asymmetric one (the criterion is this
+    library's reading; oracle.c states it). Returns (s_bits, z_bits, codes)."""
     a = _c(x, np.float32)
     s = np.zeros(1, np.uint16)
     z = np.zeros(1, np.uint16)

@@ -303,7 +303,7 @@ void oracle_quantize_group(const float *x, int n, int stride, int bits,
 
 /* Hybrid symmetric/asymmetric choice per group [INQ] "(i) hybrid
  * quantization ... based on local statistics". The page states no criterion;
- * this reading takes the candidate with the smaller squared reconstruction
+ * this reading takes the candidate with the smaller worst-case reconstruction
  * error of the group, ties to the asymmetric one:
  *   asymmetric: the recipe of oracle_quantize_group above;
  *   symmetric:  a grid with an exact zero level. Qp = 2^(bits-1) - 1,
@@ -314,29 +314,21 @@ void oracle_quantize_group(const float *x, int n, int stride, int bits,
  *     q = clamp(rint_even(fp32(x * r)), -Qp, Qp) + C.
  *   Both candidates store (s, z) as fp16 and dequantize as q * s + z, so the
  *   choice is invisible to the readers of the cache.
- *   Error of a candidate: e = fp32(x - fma(q, s, z)) per element, squares
- *   summed with fma in element order over consecutive runs of 32 elements
- *   (a group of 16 is one run), run sums then added pairwise
- *   ((r0 + r1) + (r2 + r3)) ...; symmetric iff its sum is smaller. */
-static float run_tree_sse(const float *x, int n, int stride, const uint8_t *q,
-                          int q_stride, float s, float z)
+ *   Error of a candidate: the largest |e| over the group with
+ *   e = fp32(x - fma(q, s, z)) per element; a maximum is exact, so the choice
+ *   does not depend on the order the elements are visited in. Symmetric iff
+ *   its largest error is smaller. */
+static float max_abs_err(const float *x, int n, int stride, const uint8_t *q,
+                         int q_stride, float s, float z)
 {
-    float runs[64];
-    int n_runs = 0;
-    for (int r0 = 0; r0 < n; r0 += 32) {
-        int len = (n - r0 < 32) ? n - r0 : 32;
-        float acc = 0.0f;
-        for (int i = r0; i < r0 + len; ++i) {
-            float xh = fmaf((float)q[(int64_t)i * q_stride], s, z);
-            float e = x[(int64_t)i * stride] - xh;
-            acc = fmaf(e, e, acc);
-        }
-        runs[n_runs++] = acc;
+    float m = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float xh = fmaf((float)q[(int64_t)i * q_stride], s, z);
+        float e = fabsf(x[(int64_t)i * stride] - xh);
+        if (e > m)
+            m = e;
     }
-    for (int w = 1; w < n_runs; w *= 2)
-        for (int i = 0; i + w < n_runs; i += 2 * w)
-            runs[i] = runs[i] + runs[i + w];
-    return runs[0];
+    return m;
 }
 
 void oracle_quantize_group_hybrid(const float *x, int n, int stride, int bits,
@@ -375,9 +367,9 @@ void oracle_quantize_group_hybrid(const float *x, int n, int stride, int bits,
             t = (float)Qp;
         qs[i] = (uint8_t)(int)(t + (float)C);
     }
-    float ea = run_tree_sse(x, n, stride, q_out, q_stride, oracle_f16_to_f32(sa),
-                            oracle_f16_to_f32(za));
-    float es = run_tree_sse(x, n, stride, qs, 1, ss, zs);
+    float ea = max_abs_err(x, n, stride, q_out, q_stride, oracle_f16_to_f32(sa),
+                           oracle_f16_to_f32(za));
+    float es = max_abs_err(x, n, stride, qs, 1, ss, zs);
     if (es < ea) {
         *s_out = sb;
         *z_out = zb;

@@ -15,12 +15,21 @@ from gpu_common import (D, SCALE, append, assert_close, assign_pages, dev, expec
 pytestmark = pytest.mark.gpu
 
 
+def _mixed(g, shape, df, scale):
+    # half the token rows heavy-tailed (Student t), half sparse values on a
+    # coarse grid (multiples of 1/3, half of them exact zeros): the symmetric
+    # grid, with its exact zero level, wins some groups of the second kind
+    cont = g.standard_t(df, shape)
+    grid = np.round(g.standard_normal(shape) * 3) / 3 * (g.random(shape) < 0.5)
+    pick = (g.random(shape[:-1]) < 0.5)[..., None]
+    return (np.where(pick, grid, cont) * scale).astype(np.float32)
+
+
 def _heavy(g, T, H, dtype, df=2, scale=1.0):
-    # heavy-tailed rows (Student t), so that both grids win some groups;
     # channels 0..3 of the keys carry x20 outliers as usual
     out = np.where(np.arange(D) < 4, 20, 1).astype(np.float32)
-    k = W.finish(g.standard_t(df, (T, H, D)).astype(np.float32) * np.float32(scale) * out, dtype)
-    v = W.finish(g.standard_t(df, (T, H, D)).astype(np.float32) * np.float32(scale), dtype)
+    k = W.finish(_mixed(g, (T, H, D), df, scale) * out, dtype)
+    v = W.finish(_mixed(g, (T, H, D), df, scale), dtype)
     return k, v
 
 
