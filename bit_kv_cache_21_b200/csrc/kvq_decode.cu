@@ -123,12 +123,11 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.q_dtype = q_dtype;
     p.q_bytes = (q_dtype == KVQ_FP32) ? 4 : 2;
     const int gqa = num_q_heads / d.num_kv_heads;
-    const StageLayout L = stage_layout(d, gqa, p.q_bytes);
+    const StageLayout L = stage_layout(d);
     p.stage_bytes = L.bytes;
     p.off_ksz = L.off_ksz;
     p.off_vc = L.off_vc;
     p.off_vsz = L.off_vsz;
-    p.off_q = L.off_q;
     p.off_hdr = L.off_hdr;
     p.bf_tile = L.bf_tile;
     p.bf_off_v = L.bf_off_v;

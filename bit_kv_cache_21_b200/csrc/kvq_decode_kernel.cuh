@@ -12,20 +12,25 @@
 // the keys' orthogonal transform, so q~ . k~ = q . k.
 //
 // Work items are (sequence, KV head, split of `chunk` tokens). The kernel is
-// persistent: each CTA (4 consumer warps + 1 producer warp) runs until a
-// global item counter is exhausted. The producer warp claims items and streams
-// every item's tiles (K codes, K scale/zero, V codes, V scale/zero; bf16 rows
-// for the recent-token window; the item's query rows with its first tile) into
-// a shared-memory ring with 1-D bulk copies (TMA engine, mbarrier
-// complete_tx); its lanes issue the copies of a tile in parallel, one page per
-// lane for paged caches. Each stage carries a small header, so the consumers
-// follow the stream without further coordination and the ring never drains
-// between items.
+// persistent: each CTA (4 consumer warps, 1 producer warp, 1 helper warp)
+// runs until a global item counter is exhausted. The producer warp claims
+// items and streams every item's tiles (K codes, K scale/zero, V codes, V
+// scale/zero; bf16 rows for the recent-token window) into a shared-memory ring
+// with 1-D bulk copies (TMA engine, mbarrier complete_tx); its lanes issue the
+// copies of a tile in parallel, one page per lane for paged caches. Each stage
+// carries a small header, so the consumers follow the stream without further
+// coordination and the ring never drains between items. The helper warp
+// rotates each item's query rows and builds its key coefficients one item
+// ahead, and merges the four consumer warps' states into the split's partial
+// once they have deposited them, so the consumers never wait for each other.
 //
-// The path is bound by the FP32 pipe, not by the tensor cores: every cached
-// element meets GQA query heads, one multiply-add each, and on sm_100a the
-// packed f32x2 FMA issues at half rate. So the consumers spend as few issue
-// slots as possible besides those multiply-adds:
+// Every cached element meets GQA query heads, one multiply-add each, on the
+// CUDA cores (each cached element meets only GQA = 4 query rows, too thin a
+// contraction for the tensor cores). The consumers are bound by instruction
+// issue: besides the packed f32x2 multiply-adds (16 warp instructions per
+// token and KV head at INT4, GQA 4) they convert codes, load coefficients and
+// run the softmax. So they spend as few issue slots as possible besides the
+// multiply-adds:
 //   * keys: one lane per token. A lane walks its token's code row in 16-byte
 //     chunks and multiplies each code with the GQA heads' query coefficients,
 //     which every lane reads with the same broadcast shared-memory load. No
@@ -45,8 +50,8 @@
 //   * values: 16 lanes cover the 128 channels (8 each) for all GQA heads; the
 //     two half-warps take alternate tokens; the weights p*s come from the key
 //     lanes through shared memory, already duplicated into f32x2 pairs.
-// The four warps' states are merged once per item; the merge kernel combines
-// the splits.
+// The four warps' states are merged once per item by the helper warp; the
+// merge kernel combines the splits.
 #pragma once
 
 #include <algorithm>
@@ -65,7 +70,11 @@ constexpr int kMaxStages = 4;      // shared-memory ring depth, chosen on the ho
 constexpr int kMaxDevices = 64;    // launch settings cached per device
 constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;
+constexpr int kProducerWarp = kConsumerWarps;      // streams the tiles
+constexpr int kHelperWarp = kConsumerWarps + 1;    // query rows, coefficients, item merges
+constexpr int kThreads = kConsumers + 64;
+constexpr int kItemSlots = 2;      // items in flight per CTA (query rows and coefficients)
+constexpr int kDepStride = 132;    // floats per (warp, head) deposit: o[128], (m, l), pad
 constexpr int kMaxGroups = 8;      // kHeadDim / smallest token-wise group (16)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -83,8 +92,13 @@ enum TailMode { kTailNone = 0, kTailWindow = 1, kTailSink = 2 };
 constexpr int kFirst = 1, kLast = 2, kWindow = 4, kDone = 8, kSink = 16;
 
 struct TileHdr {
-    int seq, kvh, split, t0;
-    int n, flags, start, pad1;  // tokens [start, n) of the tile are attended
+    int t0, n, flags, start;  // tokens [start, n) of the tile are attended
+    int item, pad[3];         // the CTA's item ordinal (its slot: item % kItemSlots)
+};
+
+// Coordinates of an item, posted by the producer for the helper warp.
+struct ItemInfo {
+    int seq, kvh, split, done;
 };
 
 struct DecodeParams {
@@ -112,12 +126,16 @@ struct DecodeParams {
     int ns;                // ring depth (stages), <= kMaxStages
     int q_dtype, q_bytes;  // element type and bytes of q
     // shared-memory stage layout (bytes)
-    int stage_bytes, off_ksz, off_vc, off_vsz, off_q, off_hdr;
+    int stage_bytes, off_ksz, off_vc, off_vsz, off_hdr;
     int bf_tile, bf_off_v;  // bf16 tiles: tokens per tile, offset of the V rows
     // per-warp scratch (floats): value weights (also the lanes' W/Z partials
     // when they are summed), then the warp's W/Z totals
     int warp_floats, off_tot;
-    int n_sets;            // coefficient sets (per-channel keys: 2 x blocks per tile)
+    int n_sets;            // per-channel keys: coefficient sets (2 x blocks per tile)
+    int slot_floats;       // floats per item slot
+    // byte offsets after the stage ring: item slots, per-channel sets, the
+    // warps' deposits, per-warp scratch, barriers and the small words
+    int off_slots, off_csets, off_dep, off_scr, off_bar;
     int64_t timeout_ns;
     int skip_tile;
 };
@@ -767,6 +785,104 @@ constexpr int decode_min_blocks(int km, int vm, int gkc, int gvc) {
     return (km == K_BF16 || (km == K_TOKEN && gkc == 0) || (vm == V_TOKEN && gvc == 0)) ? 1 : 2;
 }
 
+// Query rows of one item's GQA heads, rotated and scaled to log2 units, into
+// qs [GQA][128] (and unrotated into qs_raw for the sink tiles), then the key
+// coefficients of every head (token-wise and bf16 keys; per-channel keys
+// build theirs per tile from qs). Run by one warp: the heads' loads are issued
+// together, then the heads are rotated side by side.
+template <int GQA, int KM, int KBF, int GKC, bool SINK>
+__device__ __forceinline__ void build_item_query(const DecodeParams &p, const ItemInfo &inf, float *qs,
+                                                 float *qs_raw, float *coefs, int lane) {
+    using RG = RowGeo<KBF>;
+    constexpr int QHSTR = RG::nch * RG::cstr;
+    const int64_t row0 = static_cast<int64_t>(inf.seq) * p.Hq + inf.kvh * GQA;
+    float x[GQA][4];
+    if (p.q_dtype == KVQ_FP32) {
+        float4 v[GQA];
+#pragma unroll
+        for (int g = 0; g < GQA; ++g)
+            v[g] = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + (row0 + g) * kHeadDim) + lane);
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) { x[g][0] = v[g].x; x[g][1] = v[g].y; x[g][2] = v[g].z; x[g][3] = v[g].w; }
+    } else {
+        uint2 v[GQA];
+#pragma unroll
+        for (int g = 0; g < GQA; ++g)
+            v[g] = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.q) + (row0 + g) * kHeadDim) + lane);
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) {
+            const uint32_t w[2] = {v[g].x, v[g].y};
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (p.q_dtype == KVQ_BF16) {
+                    x[g][2 * j] = bf16_bits_to_float(w[j] & 0xFFFFu);
+                    x[g][2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
+                } else {
+                    x[g][2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] & 0xFFFFu)));
+                    x[g][2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] >> 16)));
+                }
+            }
+        }
+    }
+    if (SINK) {
+#pragma unroll
+        for (int g = 0; g < GQA; ++g)
+            *reinterpret_cast<float4 *>(qs_raw + g * kHeadDim + 4 * lane) =
+                make_float4(x[g][0] * p.qscale, x[g][1] * p.qscale, x[g][2] * p.qscale, x[g][3] * p.qscale);
+    }
+    if (p.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
+        const float4 sg = __ldg(reinterpret_cast<const float4 *>(p.signs) + lane);
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) { x[g][0] *= sg.x; x[g][1] *= sg.y; x[g][2] *= sg.z; x[g][3] *= sg.w; }
+    }
+    if (p.hb > 0) {
+#pragma unroll
+        for (int g = 0; g < GQA; ++g) {
+            if (p.hb > 1) { float a = x[g][0], b = x[g][1]; x[g][0] = a + b; x[g][1] = a - b;
+                            a = x[g][2]; b = x[g][3]; x[g][2] = a + b; x[g][3] = a - b; }
+            if (p.hb > 2) { float a = x[g][0], b = x[g][2]; x[g][0] = a + b; x[g][2] = a - b;
+                            a = x[g][1]; b = x[g][3]; x[g][1] = a + b; x[g][3] = a - b; }
+        }
+        for (int m = 1; m < 32 && 4 * m < p.hb; m <<= 1) {
+            const bool upper = (lane & m) != 0;
+#pragma unroll
+            for (int g = 0; g < GQA; ++g)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float o = __shfl_xor_sync(0xffffffffu, x[g][j], m);
+                    x[g][j] = upper ? o - x[g][j] : x[g][j] + o;
+                }
+        }
+#pragma unroll
+        for (int g = 0; g < GQA; ++g)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[g][j] *= p.hscale;
+    }
+#pragma unroll
+    for (int g = 0; g < GQA; ++g) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[g][j] *= p.qscale;
+        *reinterpret_cast<float4 *>(qs + g * kHeadDim + 4 * lane) = make_float4(x[g][0], x[g][1], x[g][2], x[g][3]);
+        if constexpr (KM == K_TOKEN)
+            build_head<GQA, KBF, 0, GKC>(x[g], nullptr, coefs + g * QHSTR, coefs + GQA * QHSTR, g, p.gk, lane);
+        if constexpr (KM == K_BF16)
+            build_head<GQA, 16, 2, 0>(x[g], nullptr, coefs + g * QHSTR, coefs + GQA * QHSTR, g, 128, lane);
+    }
+}
+
+// Warp roles of a CTA: warps 0..3 consume tiles, warp 4 streams them (bulk
+// copies into the stage ring), warp 5 prepares every item's query rows and
+// coefficients one item ahead and merges the consumers' item states into the
+// split's partial. The consumers never wait for each other: an item begins
+// when its coefficients are ready and ends with each warp depositing its
+// state; per-channel keys alone share per-tile coefficient builds.
+//
+// Item slots (kItemSlots, used round robin by the CTA's item ordinal n):
+//   posted[j]    producer -> helper: the item's coordinates are in info[j]
+//   coef_full[j] helper -> consumers: qs / coefficients of slot j are built
+//   slot_free[j] helper -> producer: item n merged, slot j may take n + 2
+// and, single-buffered, deposited (consumers -> helper: the four states of
+// item n are in dep) and merged (helper -> consumers: dep may take n + 1).
 template <int GQA, int KM, int VM, int KBITS, int VBITS, int GKC, int GVC, int TL>
 __global__ void __launch_bounds__(kThreads, decode_min_blocks(KM, VM, GKC, GVC))
 decode_splitk_kernel(const DecodeParams p) {
@@ -779,28 +895,42 @@ decode_splitk_kernel(const DecodeParams p) {
     using RG = RowGeo<KBF>;
     constexpr int QHSTR = RG::nch * RG::cstr;                 // coefficient floats per head
     constexpr int CBUF = GQA * QHSTR + kMaxGroups * GQA * 2;  // coefficients + group sums
+    constexpr int QF = GQA * kHeadDim;                        // floats of one set of query rows
+    constexpr int RSTR = kDepStride;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NS = p.ns;
 
     uint8_t *stages = smem;
-    uint8_t *tail = smem + static_cast<size_t>(NS) * p.stage_bytes;
-    float *qs = reinterpret_cast<float *>(tail);                    // [GQA][128]
-    float *qs_raw = qs + GQA * kHeadDim;                             // [GQA][128] unrotated (sinks only)
-    float *coefs = qs_raw + (SINK ? GQA * kHeadDim : 0);             // [n_sets][CBUF], CTA-shared
-    float *scratch_all = coefs + p.n_sets * CBUF;                    // [4][warp_floats]
-    uint64_t *full = reinterpret_cast<uint64_t *>(scratch_all + kConsumerWarps * p.warp_floats);
+    float *slots = reinterpret_cast<float *>(smem + p.off_slots);    // [kItemSlots][slot_floats]
+    float *csets = reinterpret_cast<float *>(smem + p.off_csets);    // per-channel keys: [n_sets][CBUF]
+    float *dep = reinterpret_cast<float *>(smem + p.off_dep);        // [warps][GQA][RSTR]
+    float *scratch_all = reinterpret_cast<float *>(smem + p.off_scr);  // [warps][warp_floats]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.off_bar);
     uint64_t *empty = full + kMaxStages;
-    int *abort_word = reinterpret_cast<int *>(empty + kMaxStages);
+    uint64_t *posted = empty + kMaxStages;
+    uint64_t *coef_full = posted + kItemSlots;
+    uint64_t *slot_free = coef_full + kItemSlots;
+    uint64_t *deposited = slot_free + kItemSlots;
+    uint64_t *merged = deposited + 1;
+    int *abort_word = reinterpret_cast<int *>(merged + 1);
     volatile int *abort_flag = abort_word;
-    int *pref = abort_word + 4;  // [S + 1]
-    int *lens = pref + p.S + 1;  // [S] clamped lengths
+    ItemInfo *info = reinterpret_cast<ItemInfo *>(abort_word + 4);  // [kItemSlots]
+    int *pref = reinterpret_cast<int *>(info + kItemSlots);         // [S + 1]
+    int *lens = pref + p.S + 1;                                      // [S] clamped lengths
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
+        for (int j = 0; j < kItemSlots; ++j) {
+            mbar_init(&posted[j], 1);
+            mbar_init(&coef_full[j], 32);
+            mbar_init(&slot_free[j], 32);
+        }
+        mbar_init(deposited, kConsumers);
+        mbar_init(merged, 32);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -809,8 +939,65 @@ decode_splitk_kernel(const DecodeParams p) {
     // waits for this grid's completion before reading anything.
     pdl_launch_dependents();
 
-    if (warp == kConsumerWarps) {
+    if (warp == kHelperWarp) {
+        // ------------------------- helper -------------------------
+        // Item n's coefficients are built once its coordinates are posted;
+        // item n is merged once its four states are deposited. Builds run one
+        // item ahead of merges.
+        auto build = [&](int j) {
+            float *slot = slots + j * p.slot_floats;
+            const ItemInfo inf = info[j];
+            build_item_query<GQA, KM, KBF, GKC, SINK>(p, inf, slot, slot + QF, slot + (SINK ? 2 : 1) * QF, lane);
+            mbar_arrive(&coef_full[j]);
+        };
+        if (!mbar_wait_bounded(&posted[0], 0, p.timeout_ns, p.status, abort_flag)) return;
+        if (info[0].done) return;
+        build(0);
+        for (int n = 0;; ++n) {
+            const int j = n % kItemSlots, j1 = (n + 1) % kItemSlots;
+            if (!mbar_wait_bounded(&posted[j1], ((n + 1) / kItemSlots) & 1, p.timeout_ns, p.status, abort_flag))
+                return;
+            const bool more = !info[j1].done;
+            if (more) build(j1);
+            if (!mbar_wait_bounded(deposited, n & 1, p.timeout_ns, p.status, abort_flag)) return;
+            // merge the warps' states of item n: head g, 4 channels per lane
+            const ItemInfo inf = info[j];
+#pragma unroll 1
+            for (int g = 0; g < GQA; ++g) {
+                float2 mlw[kConsumerWarps];
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    mlw[w] = *reinterpret_cast<const float2 *>(dep + (w * GQA + g) * RSTR + kHeadDim);
+                    M = fmaxf(M, mlw[w].x);
+                }
+                float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                float l = 0.0f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float e = (mlw[w].x == -INFINITY) ? 0.0f : fast_exp2(mlw[w].x - M);
+                    const float4 ov = ldsf4(dep + (w * GQA + g) * RSTR + 4 * lane);
+                    o.x = fmaf(e, ov.x, o.x); o.y = fmaf(e, ov.y, o.y);
+                    o.z = fmaf(e, ov.z, o.z); o.w = fmaf(e, ov.w, o.w);
+                    l = fmaf(e, mlw[w].y, l);
+                }
+                const int hq = inf.kvh * GQA + g;
+                const int64_t pi = (static_cast<int64_t>(inf.seq) * p.Hq + hq) * p.n_split + inf.split;
+                *reinterpret_cast<float4 *>(p.o_part + pi * kHeadDim + 4 * lane) = o;
+                if (lane == 0) p.ml[pi] = make_float2(M, l);
+            }
+            mbar_arrive(merged);
+            mbar_arrive(&slot_free[j]);
+            if (!more) return;
+        }
+    }
+
+    if (warp == kProducerWarp) {
         // ------------------------- producer -------------------------
+        // The first item is claimed before the prefix is built (the atomic's
+        // round trip overlaps the length loads), later ones one item ahead.
+        int next = 0;
+        if (lane == 0) next = atomicAdd(p.counter, 1);
         // Item prefix over sequences: sequence s has H * ceil(T_s / chunk) items.
         int carry = 0;
         for (int base = 0; base < p.S; base += 32) {
@@ -846,11 +1033,7 @@ decode_splitk_kernel(const DecodeParams p) {
         const int ngv = (VM == V_TOKEN) ? kHeadDim / p.gv : 0;
         int it = 0;  // tile counter of this CTA (stage it % NS, round it / NS)
         bool stop = false;
-        // The next item is claimed one item ahead, so the atomic's latency
-        // hides behind the current item's copies.
-        int next = 0;
-        if (lane == 0) next = atomicAdd(p.counter, 1);
-        while (!stop) {
+        for (int n_item = 0; !stop; ++n_item) {
             int item = __shfl_sync(0xffffffffu, next, 0);
             if (lane == 0 && item < n_items) next = atomicAdd(p.counter, 1);
             int seq = 0, kvh = 0, split = 0;
@@ -871,6 +1054,18 @@ decode_splitk_kernel(const DecodeParams p) {
                 n_wt = (WIN && t_end > w_begin) ? (t_end - w_begin + p.bf_tile - 1) / p.bf_tile : 0;
                 n_sink = (SINK && split == 0 && p.sink_len > 0) ? min(p.sink_len, T) : 0;
                 n_st = (n_sink + p.bf_tile - 1) / p.bf_tile;
+            }
+            // Post the item (or the end marker) in its slot for the helper.
+            {
+                const int j = n_item % kItemSlots, u = n_item / kItemSlots;
+                int ok = 1;
+                if (lane == 0 && u > 0)
+                    ok = mbar_wait_bounded(&slot_free[j], (u - 1) & 1, p.timeout_ns, p.status, abort_flag);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                if (lane == 0) {
+                    info[j] = ItemInfo{seq, kvh, split, item >= n_items ? 1 : 0};
+                    mbar_arrive(&posted[j]);
+                }
             }
             const int n_tiles = (item < n_items) ? n_qt + n_wt + n_st : 1;  // 1 = the done marker
             const int64_t sh = static_cast<int64_t>(seq) * p.H + kvh;
@@ -903,21 +1098,12 @@ decode_splitk_kernel(const DecodeParams p) {
                 const int n = sink ? min(p.bf_tile, n_sink - t0)
                                    : (window ? min(p.bf_tile, t_end - t0) : min(TILE, q_end - t0));
                 if (lane == 0) {
-                    hdr->seq = seq;
-                    hdr->kvh = kvh;
-                    hdr->split = split;
                     hdr->t0 = t0;
                     hdr->n = n;
                     hdr->start = (SINK && !window) ? max(0, p.sink_len - t0) : 0;
                     hdr->flags = (ti == 0 ? kFirst : 0) | (ti == n_tiles - 1 ? kLast : 0) |
                                  (window ? kWindow : 0) | (sink ? kSink : 0);
-                }
-                const uint32_t qb = (ti == 0) ? GQA * kHeadDim * p.q_bytes : 0;
-                if (qb && lane == 31) {  // the item's query rows ride with its first tile
-                    const uint8_t *qsrc = static_cast<const uint8_t *>(p.q) +
-                                          ((static_cast<int64_t>(seq) * p.Hq + kvh * GQA) * kHeadDim) * p.q_bytes;
-                    mbar_expect_tx(bar, qb);
-                    bulk_g2s(st + p.off_q, qsrc, qb, bar);
+                    hdr->item = n_item;
                 }
                 if (sink) {
                     const uint32_t bytes = n * kHeadDim * 2;
@@ -1013,8 +1199,6 @@ decode_splitk_kernel(const DecodeParams p) {
     float *scratch = scratch_all + warp * p.warp_floats;
     float *wsm = scratch;                  // value weights / W-Z partials of the lanes
     float *totals = scratch + p.off_tot;   // W-Z totals of the warp
-    float *red = scratch;                  // item merge (after the last tile), [GQA][132]
-    constexpr int RSTR = 132;
     const int slice = lane & 15;
 
     constexpr bool VCH = VM == V_CHANNEL;
@@ -1074,64 +1258,15 @@ decode_splitk_kernel(const DecodeParams p) {
         const uint8_t *sb = stages + static_cast<size_t>(s) * p.stage_bytes;
         const TileHdr hdr = *reinterpret_cast<const TileHdr *>(sb + p.off_hdr);
         if (hdr.flags & kDone) break;
+        const int jslot = hdr.item % kItemSlots;
+        const float *qs = slots + jslot * p.slot_floats;
+        const float *coefs = qs + (SINK ? 2 : 1) * QF;
 
         if (hdr.flags & kFirst) {
-            // ---- item prologue: the query rows arrived with this tile ----
-            // Warp g rotates head g, stores it (window tiles and per-channel
-            // rebuilds read it) and builds the head's key coefficients.
-            if (warp < GQA) {
-                const uint8_t *qrow = sb + p.off_q + warp * kHeadDim * p.q_bytes;
-                float x[4];
-                if (p.q_dtype == KVQ_FP32) {
-                    const uint4 v = lds128(qrow + 16 * lane);
-                    x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
-                    x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
-                } else {
-                    const uint2 v = lds64(qrow + 8 * lane);
-                    const uint32_t w[2] = {v.x, v.y};
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        if (p.q_dtype == KVQ_BF16) {
-                            x[2 * j] = bf16_bits_to_float(w[j] & 0xFFFFu);
-                            x[2 * j + 1] = bf16_bits_to_float(w[j] >> 16);
-                        } else {
-                            x[2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] & 0xFFFFu)));
-                            x[2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[j] >> 16)));
-                        }
-                    }
-                }
-                if (SINK)
-                    *reinterpret_cast<float4 *>(qs_raw + warp * kHeadDim + 4 * lane) =
-                        make_float4(x[0] * p.qscale, x[1] * p.qscale, x[2] * p.qscale, x[3] * p.qscale);
-                if (p.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
-                    const float4 sg = __ldg(reinterpret_cast<const float4 *>(p.signs) + lane);
-                    x[0] *= sg.x; x[1] *= sg.y; x[2] *= sg.z; x[3] *= sg.w;
-                }
-                if (p.hb > 0) {
-                    if (p.hb > 1) { float a = x[0], b = x[1]; x[0] = a + b; x[1] = a - b;
-                                    a = x[2]; b = x[3]; x[2] = a + b; x[3] = a - b; }
-                    if (p.hb > 2) { float a = x[0], b = x[2]; x[0] = a + b; x[2] = a - b;
-                                    a = x[1]; b = x[3]; x[1] = a + b; x[3] = a - b; }
-                    for (int m = 1; m < 32 && 4 * m < p.hb; m <<= 1) {
-                        const bool upper = (lane & m) != 0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float o = __shfl_xor_sync(0xffffffffu, x[j], m);
-                            x[j] = upper ? o - x[j] : x[j] + o;
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) x[j] *= p.hscale;
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) x[j] *= p.qscale;
-                *reinterpret_cast<float4 *>(qs + warp * kHeadDim + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
-                if constexpr (KM == K_TOKEN)
-                    build_head<GQA, KBF, 0, GKC>(x, nullptr, coefs + warp * QHSTR, coefs + GQA * QHSTR, warp, p.gk, lane);
-                if constexpr (KM == K_BF16)
-                    build_head<GQA, 16, 2, 0>(x, nullptr, coefs + warp * QHSTR, coefs + GQA * QHSTR, warp, 128, lane);
-            }
-            named_sync(1, kConsumers);
+            // ---- item start: the helper has built this slot's query rows ----
+            if (!mbar_wait_bounded(&coef_full[jslot], (hdr.item / kItemSlots) & 1, p.timeout_ns, p.status,
+                                   abort_flag))
+                break;
 #pragma unroll
             for (int g = 0; g < GQA; ++g) {
                 st.mref[g] = -INFINITY;
@@ -1157,7 +1292,7 @@ decode_splitk_kernel(const DecodeParams p) {
                 // the sets of this tile's parity (no warp still reads them:
                 // all passed the previous tile's barrier), then wait for all.
                 const int nbt = TILE / p.R;  // block sets per tile
-                float *sets = coefs + (kc_tiles & 1) * nbt * CBUF;
+                float *sets = csets + (kc_tiles & 1) * nbt * CBUF;
                 const int nb = (hdr.n + p.R - 1) / p.R;
                 for (int idx = warp; idx < nb * GQA; idx += kConsumerWarps) {
                     const int b = idx / GQA, g = idx - b * GQA;
@@ -1191,14 +1326,14 @@ decode_splitk_kernel(const DecodeParams p) {
             }
             // bf16 window keys against the query rows (coefficients = q), or
             // sink keys against the unrotated ones (one code path for both)
-            const float *qrows = (SINK && (hdr.flags & kSink)) ? qs_raw : qs;
+            const float *qrows = (SINK && (hdr.flags & kSink)) ? qs + QF : qs;
             process_tile<GQA, K_BF16, V_BF16, 16, 16, kWinTile / kConsumerWarps, kHeadDim, 0, NVG, false, false>(
                 sb, nullptr, sb + p.bf_off_v, nullptr, hdr.n, 0, qrows, kHeadDim, 8, nullptr, p.gk, p.gv, st,
                 wsm, warp, lane);
         }
 
         if (hdr.flags & kLast) {
-            // ---- item epilogue: merge the four warps, write the partial ----
+            // ---- item end: deposit this warp's state for the helper's merge ----
             if (VM == V_TOKEN && !folded) fold_values();
             if constexpr (VM == V_CHANNEL) {  // the folded sums join the window's
                 const bool hi = lane >= 16;
@@ -1210,7 +1345,10 @@ decode_splitk_kernel(const DecodeParams p) {
                         st.o[g][4 + j].x += hi ? st.of[g][j] : 0.0f;
                     }
             }
-            __syncwarp();
+            if (hdr.item > 0 &&
+                !mbar_wait_bounded(merged, (hdr.item - 1) & 1, p.timeout_ns, p.status, abort_flag))
+                break;
+            float *red = dep + warp * GQA * RSTR;
 #pragma unroll
             for (int g = 0; g < GQA; ++g) {
                 float lg = st.l[g];
@@ -1227,34 +1365,11 @@ decode_splitk_kernel(const DecodeParams p) {
                     *reinterpret_cast<float4 *>(rp) = make_float4(v[0], v[1], v[2], v[3]);
                     *reinterpret_cast<float4 *>(rp + 4) = make_float4(v[4], v[5], v[6], v[7]);
                 }
-                if (lane == 0) *reinterpret_cast<float2 *>(red + g * RSTR + 128) = make_float2(st.mref[g], lg);
+                if (lane == 0) *reinterpret_cast<float2 *>(red + g * RSTR + kHeadDim) = make_float2(st.mref[g], lg);
             }
-            named_sync(1, kConsumers);
-            if (warp < GQA) {  // warp g combines head g, 4 channels per lane
-                const int g = warp;
-                float2 mlw[kConsumerWarps];
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    mlw[w] = *reinterpret_cast<const float2 *>(scratch_all + w * p.warp_floats + g * RSTR + 128);
-                    M = fmaxf(M, mlw[w].x);
-                }
-                float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                float l = 0.0f;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float e = (mlw[w].x == -INFINITY) ? 0.0f : fast_exp2(mlw[w].x - M);
-                    const float4 ov = ldsf4(scratch_all + w * p.warp_floats + g * RSTR + 4 * lane);
-                    o.x = fmaf(e, ov.x, o.x); o.y = fmaf(e, ov.y, o.y);
-                    o.z = fmaf(e, ov.z, o.z); o.w = fmaf(e, ov.w, o.w);
-                    l = fmaf(e, mlw[w].y, l);
-                }
-                const int hq = hdr.kvh * GQA + g;
-                const int64_t pi = (static_cast<int64_t>(hdr.seq) * p.Hq + hq) * p.n_split + hdr.split;
-                *reinterpret_cast<float4 *>(p.o_part + pi * kHeadDim + 4 * lane) = o;
-                if (lane == 0) p.ml[pi] = make_float2(M, l);
-            }
+            mbar_arrive(deposited);
         }
+        __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
     }
 }
@@ -1263,14 +1378,13 @@ decode_splitk_kernel(const DecodeParams p) {
 // Host side
 // ---------------------------------------------------------------------------
 struct StageLayout {
-    int bytes, off_ksz, off_vc, off_vsz, off_q, off_hdr, bf_tile, bf_off_v;
+    int bytes, off_ksz, off_vc, off_vsz, off_hdr, bf_tile, bf_off_v;
 };
 
 inline int round16(int x) { return (x + 15) & ~15; }
 
-// Stage: tile data, then the query rows of a first tile (GQA x 128 x q_bytes,
-// at most 2 KB), then a 32-byte header.
-inline StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
+// Stage: tile data, then a 32-byte header.
+inline StageLayout stage_layout(const kvq_cache_desc &d) {
     StageLayout L{};
     int data;
     if (d.bits_k == 16) {  // every tile is bf16 rows: K at 0, V after it
@@ -1293,15 +1407,13 @@ inline StageLayout stage_layout(const kvq_cache_desc &d, int gqa, int q_bytes) {
         L.bf_off_v = kWinTile * 256;
         if (d.residual_len > 0 || d.sink_len > 0) data = std::max(data, 2 * kWinTile * 256);
     }
-    L.off_q = round16(data);
-    L.off_hdr = L.off_q + round16(gqa * kHeadDim * q_bytes);
+    L.off_hdr = round16(data);
     L.bytes = (L.off_hdr + static_cast<int>(sizeof(TileHdr)) + 127) & ~127;
     return L;
 }
 
 // Per-warp scratch (floats): the value weights of one tile, which also hold
-// the lanes' W/Z partials when they are summed, then the W/Z totals; the item
-// merge reuses the start of it ([GQA][132]).
+// the lanes' W/Z partials when they are summed, then the W/Z totals.
 struct ScratchLayout {
     int off_tot, floats;
 };
@@ -1310,7 +1422,7 @@ inline ScratchLayout scratch_layout(int gqa, int n_vg) {
     ScratchLayout S{};
     S.off_tot = 64 * gqa * n_vg + 128;  // 32 pair rows of (n_vg * gqa + 2) f32x2
     const int used = S.off_tot + 2 * gqa * n_vg;
-    S.floats = (std::max(used, gqa * 132) + 3) & ~3;
+    S.floats = (used + 3) & ~3;
     return S;
 }
 
@@ -1331,17 +1443,28 @@ kvq_status launch_variant(DecodeParams p, int max_items, cudaStream_t stream) {
     const ScratchLayout SL = scratch_layout(GQA, n_vg);
     p.warp_floats = SL.floats;
     p.off_tot = SL.off_tot;
-    p.n_sets = (KM == K_CHANNEL) ? 2 * (kTileQ / p.R) : 1;
-    const size_t q_rows = (SINK ? 2 : 1) * static_cast<size_t>(GQA) * kHeadDim;  // rotated (+ unrotated)
-    const size_t tail = sizeof(float) * (q_rows + static_cast<size_t>(p.n_sets) * cbuf +
+    p.n_sets = (KM == K_CHANNEL) ? 2 * (kTileQ / p.R) : 0;
+    // item slots: rotated query rows (+ unrotated for sinks), then the key
+    // coefficients (per-channel keys build theirs per tile in the sets)
+    p.slot_floats = (SINK ? 2 : 1) * GQA * kHeadDim + (KM == K_CHANNEL ? 0 : cbuf);
+    p.slot_floats = (p.slot_floats + 3) & ~3;
+    const size_t tail = sizeof(float) * (static_cast<size_t>(kItemSlots) * p.slot_floats +
+                                         static_cast<size_t>(p.n_sets) * cbuf +
+                                         static_cast<size_t>(kConsumerWarps) * GQA * kDepStride +
                                          kConsumerWarps * static_cast<size_t>(p.warp_floats)) +
-                        sizeof(uint64_t) * 2 * kMaxStages + 16 + sizeof(int) * (2 * p.S + 1);
+                        sizeof(uint64_t) * (2 * kMaxStages + 3 * kItemSlots + 2) + 16 +
+                        sizeof(ItemInfo) * kItemSlots + sizeof(int) * (2 * p.S + 1);
     // Ring depth: as many stages (2..4) as let the targeted CTAs per SM fit.
     const int per_sm_target = decode_min_blocks(KM, VM, GKC, GVC);
     const size_t budget = (232448 - 1024 * per_sm_target) / per_sm_target;
     int ns = static_cast<int>(std::min<size_t>(kMaxStages, (budget > tail ? budget - tail : 0) / p.stage_bytes));
     p.ns = std::max(2, ns);
-    const size_t smem = static_cast<size_t>(p.ns) * p.stage_bytes + tail;
+    p.off_slots = p.ns * p.stage_bytes;
+    p.off_csets = p.off_slots + static_cast<int>(sizeof(float)) * kItemSlots * p.slot_floats;
+    p.off_dep = p.off_csets + static_cast<int>(sizeof(float)) * p.n_sets * cbuf;
+    p.off_scr = p.off_dep + static_cast<int>(sizeof(float)) * kConsumerWarps * GQA * kDepStride;
+    p.off_bar = p.off_scr + static_cast<int>(sizeof(float)) * kConsumerWarps * p.warp_floats;
+    const size_t smem = static_cast<size_t>(p.off_slots) + tail;
     auto kern = decode_splitk_kernel<GQA, KM, VM, KBITS, VBITS, GKC, GVC, TL>;
     if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;  // too many sequences for one launch
     // The shared-memory opt-in and the occupancy query cost host time on every
