@@ -123,6 +123,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+// The same bounded wait for a warp whose wake-up is not latency critical: it
+// sleeps about `sleep_ns` between polls, so a long wait costs fewer issue
+// slots of the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t *bar, uint32_t parity, int64_t timeout_ns,
+                                                  int32_t *status, volatile int *abort_flag,
+                                                  uint32_t sleep_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(sleep_ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (static_cast<int64_t>(global_timer_ns() - t0) > timeout_ns) {
+            status_or(status, KVQ_DEV_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // Programmatic dependent launch: let the next kernel of the stream (launched
 // with programmatic stream serialization) be scheduled now; and, in that
 // kernel, wait until the previous grid has completed and its writes are
