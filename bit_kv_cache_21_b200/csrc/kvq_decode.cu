@@ -25,13 +25,14 @@ constexpr int kMergeGroups = 4;  // partial groups per merge CTA (128 threads ea
 template <bool PARTIAL>
 __global__ void __launch_bounds__(128 * kMergeGroups) decode_merge_kernel(const float *o_part, const float2 *ml,
                                                            const int32_t *seq_lens, float *out,
-                                                           float2 *out_ml, int Hq, int n_split,
-                                                           int chunk, int max_seq_len) {
+                                                           float2 *out_ml, int Hq, int max_seq_len,
+                                                           const __grid_constant__ SplitBounds sp) {
     __shared__ CombineSmem<kMergeGroups> sm;
     pdl_wait_prior_grid();
     const int hq = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
     const int T = min(__ldg(seq_lens + seq), max_seq_len);
-    const int nv = T > 0 ? (T + chunk - 1) / chunk : 0;
+    const int nv = splits_of(sp, T);
+    const int n_split = sp.n;
     const int64_t row = static_cast<int64_t>(seq) * Hq + hq;
     float M, o, l;
     combine_partials<kMergeGroups>(o_part, ml, row * n_split * kHeadDim, kHeadDim, row * n_split, 1, nv, sm, M,
@@ -64,15 +65,32 @@ __global__ void __launch_bounds__(128) merge_partials_kernel(const float *parts,
 bool plan_decode(const kvq_cache_desc &d, int num_seqs, int num_q_heads, int max_seq_len,
                  DecodePlan *plan) {
     if (num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0 || d.num_kv_heads <= 0) return false;
-    // About eight items per resident CTA (2 per SM) when every sequence is at
-    // max_seq_len; chunks of 256..4096 tokens, a multiple of the tiles.
+    // Splits of `chunk` tokens, about four items per resident split-K CTA
+    // (two per SM) when every sequence is at max_seq_len: a multiple of the
+    // 256-token tile, 256..4096 tokens, and at most kMaxDecodeSplits splits.
+    // The CTAs claim items split-major (every unit's first split, then every
+    // unit's second, ...), so a sequence's last, partial split is among the
+    // last items claimed and fills the launch's tail. Measured on the
+    // llama8b-shaped step (16 x 8 units at 8256 tokens): chunks of 1024
+    // tokens split-major 90.7 us per split-K pass, 512 96.2, 2048 99.0, and
+    // splits that shrink from 3584 to 256 tokens 110.6. The plan depends on
+    // the sizes alone, so the workspace query and the launches agree.
     const int64_t units = static_cast<int64_t>(num_seqs) * d.num_kv_heads;
-    const int64_t target_items = 8 * 2 * 148;
-    int64_t chunk = (units * std::max(1, max_seq_len) + target_items - 1) / target_items;
-    chunk = ((chunk + kTileQ - 1) / kTileQ) * kTileQ;
-    chunk = std::min<int64_t>(std::max<int64_t>(chunk, 256), 4096);
-    plan->chunk = static_cast<int>(chunk);
-    plan->n_split = static_cast<int>(std::max<int64_t>(1, (max_seq_len + chunk - 1) / chunk));
+    const int64_t target_items = 4 * 2 * 148;
+    const int64_t L = std::max(1, max_seq_len);
+    int64_t chunk = (units * L + target_items - 1) / target_items;
+    chunk = (chunk + kTileQ - 1) / kTileQ * kTileQ;
+    chunk = std::min<int64_t>(std::max<int64_t>(chunk, kTileQ), 4096);
+    const int64_t floor_c = ((L + kMaxDecodeSplits - 1) / kMaxDecodeSplits + kTileQ - 1) / kTileQ * kTileQ;
+    chunk = std::max(chunk, floor_c);
+    SplitBounds &sp = plan->splits;
+    sp.n = 0;
+    sp.b[0] = 0;
+    for (int64_t b = 0; b < L;) {
+        b += chunk;
+        sp.b[++sp.n] = static_cast<int>(std::min<int64_t>(b, INT32_MAX));
+    }
+    plan->n_split = sp.n;
     const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * plan->n_split;
     plan->ws_part = rows * kHeadDim * sizeof(float);
     plan->ws_ml = rows * sizeof(float2);
@@ -117,7 +135,7 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.max_pages = d.max_pages_per_seq;
     p.num_pages = d.num_pages;
     p.cap = d.capacity_tokens;
-    p.chunk = plan.chunk;
+    p.sp = plan.splits;
     p.n_split = plan.n_split;
     p.max_seq_len = max_seq_len;
     p.q_dtype = q_dtype;
@@ -160,13 +178,12 @@ kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int n_split = plan.n_split, chunk = plan.chunk;
     float2 *oml = reinterpret_cast<float2 *>(out_ml);
     const cudaError_t e =
         out_ml ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<true>, o_part, ml, seq_lens, out, oml,
-                                    num_q_heads, n_split, chunk, max_seq_len)
+                                    num_q_heads, max_seq_len, plan.splits)
                : cudaLaunchKernelEx(&cfg, decode_merge_kernel<false>, o_part, ml, seq_lens, out, oml,
-                                    num_q_heads, n_split, chunk, max_seq_len);
+                                    num_q_heads, max_seq_len, plan.splits);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

@@ -11,7 +11,10 @@
 // so no dequantized element is ever formed. Dual-QK (Abstract): queries take
 // the keys' orthogonal transform, so q~ . k~ = q . k.
 //
-// Work items are (sequence, KV head, split of `chunk` tokens). The kernel is
+// Work items are (sequence, KV head, split): a split is a token range, the
+// same for every sequence (the host's plan). Items are numbered split-major,
+// so the sequences' last, partial splits are claimed last and fill the
+// launch's tail. The kernel is
 // persistent: each CTA (4 consumer warps, 1 producer warp, 1 helper warp)
 // runs until a global item counter is exhausted. The producer warp claims
 // items and streams every item's tiles (K codes, K scale/zero, V codes, V
@@ -125,7 +128,8 @@ struct DecodeParams {
     float qscale;   // softmax_scale * log2(e)
     int R;
     int paged, page_size, max_pages, num_pages, cap;
-    int chunk, n_split, max_seq_len;
+    int n_split, max_seq_len;  // partials per query head; longest sequence attended
+    SplitBounds sp;            // token ranges of the splits
     int ns;                // ring depth (stages), <= kMaxStages
     int q_dtype, q_bytes;  // element type and bytes of q
     // shared-memory stage layout (bytes)
@@ -758,19 +762,32 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
     __syncwarp();
 }
 
-// Decode an item index into (sequence, KV head, split): items are numbered
-// sequence-major, pref[s] = first item of sequence s.
-__device__ __forceinline__ void item_coords(const int *pref, int S, int H, int item, int &seq,
-                                            int &kvh, int &split) {
-    int lo = 0, hi = S;  // last s with pref[s] <= item
+// Decode an item index into (sequence, KV head, split). Items are numbered
+// split-major: spref[j] is the first item of split j, whose items are the
+// (sequence, KV head) units of the sequences with more than j splits
+// (nsq[s] > j), in sequence order, KV head fastest. Run by a whole warp.
+__device__ __forceinline__ void item_coords(const int *spref, const int *nsq, int n_split, int S, int H,
+                                            int item, int &seq, int &kvh, int &split, int lane) {
+    int lo = 0, hi = n_split;  // last j with spref[j] <= item
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (pref[mid] <= item) lo = mid; else hi = mid;
+        if (spref[mid] <= item) lo = mid; else hi = mid;
     }
-    seq = lo;
-    const int r = item - pref[lo];
-    split = r / H;
-    kvh = r - split * H;
+    split = lo;
+    const int k = item - spref[lo];
+    int r = k / H;
+    kvh = k - r * H;
+    seq = 0;
+    // the r-th sequence with more than `split` splits
+    for (int base = 0; base < S; base += 32) {
+        const unsigned m = __ballot_sync(0xffffffffu, base + lane < S && nsq[base + lane] > split);
+        const int c = __popc(m);
+        if (r < c) {
+            seq = base + __fns(m, 0, r + 1);
+            break;
+        }
+        r -= c;
+    }
 }
 
 // Expected-transaction bytes for a bulk copy issued by this thread, without an
@@ -919,8 +936,9 @@ decode_splitk_kernel(const DecodeParams p) {
     int *abort_word = reinterpret_cast<int *>(merged + 1);
     volatile int *abort_flag = abort_word;
     ItemInfo *info = reinterpret_cast<ItemInfo *>(abort_word + 4);  // [kItemSlots]
-    int *pref = reinterpret_cast<int *>(info + kItemSlots);         // [S + 1]
-    int *lens = pref + p.S + 1;                                      // [S] clamped lengths
+    int *spref = reinterpret_cast<int *>(info + kItemSlots);        // [n_split + 1] first item of each split
+    int *lens = spref + p.sp.n + 1;                                  // [S] clamped lengths
+    int *nsq = lens + p.S;                                           // [S] splits of each sequence
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -1002,32 +1020,56 @@ decode_splitk_kernel(const DecodeParams p) {
         // round trip overlaps the length loads), later ones one item ahead.
         int next = 0;
         if (lane == 0) next = atomicAdd(p.counter, 1);
-        // Item prefix over sequences: sequence s has H * ceil(T_s / chunk) items.
-        int carry = 0;
-        for (int base = 0; base < p.S; base += 32) {
-            const int s = base + lane;
-            int cnt = 0, T_s = 0;
-            if (s < p.S) {
-                T_s = __ldg(p.seq_lens + s);
-                if (T_s > p.max_seq_len) {
-                    if (blockIdx.x == 0) status_or(p.status, KVQ_DEV_SEQLEN);
-                    T_s = p.max_seq_len;
-                }
-                cnt = T_s > 0 ? p.H * ((T_s + p.chunk - 1) / p.chunk) : 0;
+        // Lengths (clamped) and split counts of the sequences; items per
+        // split: H x the sequences with more than j splits; their prefix.
+        const int n_split = p.sp.n;
+        for (int j = lane; j <= n_split; j += 32) spref[j] = 0;  // histogram of split counts first
+        __syncwarp();
+        for (int s = lane; s < p.S; s += 32) {
+            int T_s = __ldg(p.seq_lens + s);
+            if (T_s > p.max_seq_len) {
+                if (blockIdx.x == 0) status_or(p.status, KVQ_DEV_SEQLEN);
+                T_s = p.max_seq_len;
             }
+            lens[s] = T_s;
+            const int ns = splits_of(p.sp, T_s);
+            nsq[s] = ns;
+            atomicAdd(&spref[ns], 1);
+        }
+        __syncwarp();
+        // G_j = #{s : n_s > j} (suffix sums of the histogram), from the top
+        int gsum = 0;
+        for (int base = ((n_split - 1) / 32) * 32; base >= 0; base -= 32) {
+            const int j = base + lane;
+            int v = (j < n_split) ? spref[j + 1] : 0;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const int o = __shfl_down_sync(0xffffffffu, v, m);
+                if (lane + m < 32) v += o;
+            }
+            const int G = v + gsum;
+            gsum += __shfl_sync(0xffffffffu, v, 0);
+            __syncwarp();
+            if (j < n_split) spref[j + 1] = G;  // G_j parked one slot up
+            __syncwarp();
+        }
+        // exclusive prefix of H * G_j: spref[j] = first item of split j
+        int carry = 0;
+        for (int base = 0; base < n_split; base += 32) {
+            const int j = base + lane;
+            const int cnt = (j < n_split) ? p.H * spref[j + 1] : 0;
             int incl = cnt;
 #pragma unroll
             for (int m = 1; m < 32; m <<= 1) {
                 const int o = __shfl_up_sync(0xffffffffu, incl, m);
                 if (lane >= m) incl += o;
             }
-            if (s < p.S) {
-                pref[s] = carry + incl - cnt;
-                lens[s] = T_s;
-            }
+            __syncwarp();
+            if (j < n_split) spref[j] = carry + incl - cnt;
             carry += __shfl_sync(0xffffffffu, incl, 31);
+            __syncwarp();
         }
-        if (lane == 0) pref[p.S] = carry;
+        if (lane == 0) spref[n_split] = carry;
         __syncwarp();
         const int n_items = carry;
 
@@ -1043,10 +1085,10 @@ decode_splitk_kernel(const DecodeParams p) {
             int seq = 0, kvh = 0, split = 0;
             int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0, n_sink = 0, n_st = 0;
             if (item < n_items) {
-                item_coords(pref, p.S, p.H, item, seq, kvh, split);
+                item_coords(spref, nsq, n_split, p.S, p.H, item, seq, kvh, split, lane);
                 const int T = lens[seq];
-                t_begin = split * p.chunk;
-                t_end = min(T, t_begin + p.chunk);
+                t_begin = p.sp.b[split];
+                t_end = min(T, p.sp.b[split + 1]);
                 Tq = quantized_len(T, p.R);
                 q_end = min(t_end, Tq);
                 // sink positions [0, sink_len) are read from the sink rows, in
@@ -1457,7 +1499,7 @@ kvq_status launch_variant(DecodeParams p, int max_items, cudaStream_t stream) {
                                          static_cast<size_t>(kConsumerWarps) * GQA * kDepStride +
                                          kConsumerWarps * static_cast<size_t>(p.warp_floats)) +
                         sizeof(uint64_t) * (2 * kMaxStages + 3 * kItemSlots + 2) + 16 +
-                        sizeof(ItemInfo) * kItemSlots + sizeof(int) * (2 * p.S + 1);
+                        sizeof(ItemInfo) * kItemSlots + sizeof(int) * (2 * p.S + p.sp.n + 1);
     // Ring depth: as many stages (2..4) as let the targeted CTAs per SM fit.
     const int per_sm_target = decode_min_blocks(KM, VM, GKC, GVC);
     const size_t budget = (232448 - 1024 * per_sm_target) / per_sm_target;

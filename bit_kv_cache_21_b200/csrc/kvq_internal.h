@@ -20,10 +20,30 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
                          kvq_dtype dtype, const int32_t *cu_new, int32_t *seq_lens,
                          int num_seqs, int total_new, cudaStream_t stream);
 
+// Token ranges of the splits, the same for every sequence: split j covers the
+// tokens [b[j], b[j+1]) below the sequence's length; b[0] = 0, and every
+// boundary is a multiple of the decode tiles. A sequence of length T has
+// n_T = #{j : b[j] < T} splits.
+constexpr int kMaxDecodeSplits = 512;
+struct SplitBounds {
+    int n;
+    int b[kMaxDecodeSplits + 1];
+};
+
+// Number of splits of a sequence of length T (0 for T <= 0).
+__host__ __device__ inline int splits_of(const SplitBounds &sp, int T) {
+    int lo = 0, hi = sp.n;  // first j in [0, n] with b[j] >= T
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (sp.b[mid] < T) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
 // Decode attention geometry chosen on the host from the sizes alone.
 struct DecodePlan {
-    int chunk;      // tokens per split (multiple of the tile)
-    int n_split;    // splits per (sequence, KV head)
+    SplitBounds splits;
+    int n_split;    // splits of the longest sequence (partials per query head)
     size_t ws_part; // bytes of partial outputs
     size_t ws_ml;   // bytes of (m, l) pairs
     size_t ws_total;
