@@ -18,6 +18,8 @@
 // single-rounding intrinsic, so nothing is contracted into an FMA):
 //   z = fp16_rd(min), s = fp16_ru(fp32(fp32(max - z) / L)),
 //   q = clamp(rint(fp32(fp32(x - z) * fp32(1/s))), 0, L), all q = 0 if s == 0.
+#include <algorithm>
+
 #include "kvq_common.cuh"
 #include "kvq_internal.h"
 
@@ -392,65 +394,408 @@ __device__ __forceinline__ bool dest_row(const AppendParams &p, int s, int pos, 
     return true;
 }
 
-// ---- kernel: per-token append ----------------------------------------------
-// grid.x: blocks of 64 vectors; grid.y: 0 = keys, 1 = values.
-template <int DT, bool HYB>
-__global__ void __launch_bounds__(256) append_tokens_kernel(const AppendParams p) {
-    pdl_launch_dependents();  // the length advance may be scheduled; it waits for us
-    const AppendTensor &T = p.t[blockIdx.y];
-    const int lane = threadIdx.x & 31;
-    const int part = lane & 3;
-    const int64_t n_vec = static_cast<int64_t>(p.total_tokens) * p.H;
-    const int64_t vec = (static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * 8 + (lane >> 2);
-    const bool active = vec < n_vec;
-    const int64_t v = active ? vec : n_vec - 1;  // idle lanes still join the shuffles
+// ---- kernel: per-token append, two lanes per (token, head) vector --------
+// A warp takes batches of 16 consecutive input vectors (one contiguous run of
+// the [N][H][128] input), staged into shared memory by cp.async; each warp
+// keeps kAppendStages batch buffers, so the copies of its next batches run
+// under this batch's arithmetic. Lanes 2t and 2t+1 own vector t of the batch, channels
+// [0, 64) and [64, 128): the rotation's stages of half-width 1..32 stay in
+// the lane and the stage 64 is one exchange with the partner; groups of up
+// to 64 lie in one lane and a group of 128 takes one exchange of extremes.
+// The steps and their rounding are those of the lane-group path (fwht_lane,
+// qparams, qcodes), so both give the oracle's bits.
+constexpr int kAppendWarps = 4;
+constexpr int kAppendBlocksPerSm = 3;
+constexpr int kAppendStages = 2;  // batches per warp: one in use, one in flight
 
-    float x[32];
-    load32<DT>(T.src, v, part, x);
-    if (T.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
-        const float4 *sg = reinterpret_cast<const float4 *>(T.signs + part * 32);
+template <int DT>
+struct StagedRows {
+    static constexpr int half_bytes = (DT == KVQ_FP32) ? 256 : 128;  // one lane's 64 channels
+    static constexpr int in_bytes = 2 * half_bytes;                   // one input row
+    // staged row: [half 0][16-byte pad][half 1][16-byte pad], so the eight
+    // lanes of a shared-memory phase read eight distinct bank groups
+    static constexpr int half_stride = half_bytes + 16;
+    static constexpr int stride = 2 * half_stride;
+    static constexpr int batch = 16 * stride;  // one warp's buffer
+};
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Copies of batch b (vectors [16b, 16b + 16) below n_vec) into buf: 16-byte
+// chunks, consecutive lanes on consecutive chunks of the run. Lane l copies
+// chunks l + 32 i; their places in the padded buffer are `dst_lane` (the
+// lane's first) plus i rows of 32 / CPR each.
+template <int DT>
+__device__ __forceinline__ void stage_batch(const void *src, int64_t b, int64_t n_vec, uint8_t *buf,
+                                            int dst_lane, int lane) {
+    using SR = StagedRows<DT>;
+    constexpr int CPR = SR::in_bytes / 16;  // chunks per row
+    constexpr int ROWS_PER_STEP = 32 / CPR;
+    const int64_t v0 = b * 16;
+    const int64_t left = n_vec - v0;
+    const uint8_t *g = static_cast<const uint8_t *>(src) + v0 * SR::in_bytes + lane * 16;
+    uint8_t *d = buf + dst_lane;
+    if (left >= 16) {
+#pragma unroll
+        for (int i = 0; i < CPR / 2; ++i) cp_async16(d + i * ROWS_PER_STEP * SR::stride, g + i * 512);
+    } else {
+        const int n_chunks = static_cast<int>(left) * CPR;
+#pragma unroll
+        for (int i = 0; i < CPR / 2; ++i)
+            if (lane + 32 * i < n_chunks) cp_async16(d + i * ROWS_PER_STEP * SR::stride, g + i * 512);
+    }
+}
+
+// Offset of lane l's first chunk in the padded batch buffer.
+template <int DT>
+__device__ __forceinline__ int stage_offset(int lane) {
+    using SR = StagedRows<DT>;
+    constexpr int CPR = SR::in_bytes / 16;
+    constexpr int CPH = SR::half_bytes / 16;
+    const int row = lane / CPR, col = lane % CPR;
+    const int hh = col >= CPH ? 1 : 0;
+    return row * SR::stride + hh * SR::half_stride + (col - hh * CPH) * 16;
+}
+
+// The lane's staged half row as 32 channel pairs {2k, 2k + 1} in fp32.
+template <int DT>
+__device__ __forceinline__ void read_half(const uint8_t *hrow, float2 v[32]) {
+    if constexpr (DT == KVQ_FP32) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(hrow + 16 * i);
+            v[2 * i] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+            v[2 * i + 1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+        }
+    } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float4 f = __ldg(sg + i);
-            x[4 * i] *= f.x; x[4 * i + 1] *= f.y; x[4 * i + 2] *= f.z; x[4 * i + 3] *= f.w;
+            const uint4 u = *reinterpret_cast<const uint4 *>(hrow + 16 * i);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if constexpr (DT == KVQ_BF16) {
+                    v[4 * i + j] = make_float2(bf16_bits_to_float(w[j] & 0xFFFFu), bf16_bits_to_float(w[j] >> 16));
+                } else {
+                    v[4 * i + j] = make_float2(__half2float(__ushort_as_half((unsigned short)(w[j] & 0xFFFFu))),
+                                               __half2float(__ushort_as_half((unsigned short)(w[j] >> 16))));
+                }
+            }
         }
     }
-    if (T.hb > 0) fwht_lane(x, T.hb, part, T.hscale);
+}
 
-    uint32_t words[4];
-    __half2 s[2];
-    int n_sz = 0;
-    if (T.bits == 4) quant_pack_lane<4, HYB>(x, T.group, words, s, n_sz, part);
-    else quant_pack_lane<2, HYB>(x, T.group, words, s, n_sz, part);
-    if (!active) return;
+// f32x2 register pairs: a float2 is one 64-bit register pair, so these are
+// moves the compiler drops.
+__device__ __forceinline__ unsigned long long u64_of(float2 a) {
+    return *reinterpret_cast<unsigned long long *>(&a);
+}
+__device__ __forceinline__ float2 f2_of(unsigned long long u) { return *reinterpret_cast<float2 *>(&u); }
 
-    const int tok = static_cast<int>(v / p.H);
-    const int h = static_cast<int>(v - static_cast<int64_t>(tok) * p.H);
-    const int seq = find_seq(p.cu_new, p.num_seqs, tok);
-    const int pos = __ldg(p.seq_lens + seq) + (tok - __ldg(p.cu_new + seq));
-    if (pos >= 0 && pos < p.sink_len) {
-        // attention-sink token: kept as the input rounded to bf16, not quantized
-        float raw[32];
-        load32<DT>(T.src, v, part, raw);
-        uint32_t w[16];
+// Normalized Sylvester Walsh-Hadamard transform of each HB-block of the 128
+// channels, the lane holding 64 of them (`half` says which): half-widths 1, 2,
+// ..., HB/2 in ascending order, butterfly (a, b) -> (a + b, a - b) with a the
+// lower index, each op rounded to fp32; then one multiply by
+// c = fp32(1/sqrt(HB)). The half-width 64 stage pairs the lane with its
+// partner (lane ^ 1): o + s x with s = +-1 in one fma rounds like the add or
+// subtract it stands for.
+template <int HB>
+__device__ __forceinline__ void fwht_half(float2 v[32], int half, float c) {
+    if constexpr (HB > 1) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(raw[2 * j], raw[2 * j + 1]);
-            w[j] = *reinterpret_cast<const uint32_t *>(&b2);
+        for (int k = 0; k < 32; ++k) v[k] = make_float2(__fadd_rn(v[k].x, v[k].y), __fsub_rn(v[k].x, v[k].y));
+    }
+#pragma unroll
+    for (int st = 0; st < 5; ++st) {  // pair half-width hp = 2^st: channel half-width 2 hp
+        const int hp = 1 << st;
+        if (2 * hp < HB) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {  // butterfly j: pairs k and k + hp
+                const int k = (j / hp) * 2 * hp + (j % hp);
+                const unsigned long long a = u64_of(v[k]), b = u64_of(v[k + hp]);
+                v[k] = f2_of(add2(a, b));
+                v[k + hp] = f2_of(sub2(a, b));
+            }
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(
-            p.sink[blockIdx.y] + ((static_cast<int64_t>(seq) * p.H + h) * p.sink_len + pos) * kHeadDim + part * 32);
+    }
+    if constexpr (HB == 128) {
+        const float sg = half ? -1.0f : 1.0f;  // upper: o - x, lower: x + o
+        const unsigned long long sg2 = f2u(sg, sg);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        return;
+        for (int k = 0; k < 32; ++k) {
+            const float o0 = __shfl_xor_sync(0xffffffffu, v[k].x, 1);
+            const float o1 = __shfl_xor_sync(0xffffffffu, v[k].y, 1);
+            v[k] = f2_of(fma2(sg2, u64_of(v[k]), f2u(o0, o1)));
+        }
     }
-    int64_t row;
-    if (!dest_row(p, seq, pos, h, row)) {
-        if (part == 0) status_or(p.status, KVQ_DEV_CAPACITY);
-        return;
+    const unsigned long long c2 = f2u(c, c);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) v[k] = f2_of(mul2(u64_of(v[k]), c2));
+}
+
+__device__ __forceinline__ void fwht_half_any(float2 v[32], int hb, int half, float c) {
+    switch (hb) {
+        case 2: fwht_half<2>(v, half, c); break;
+        case 4: fwht_half<4>(v, half, c); break;
+        case 8: fwht_half<8>(v, half, c); break;
+        case 16: fwht_half<16>(v, half, c); break;
+        case 32: fwht_half<32>(v, half, c); break;
+        case 64: fwht_half<64>(v, half, c); break;
+        default: fwht_half<128>(v, half, c); break;
     }
-    if (T.bits == 4) store_lane<4>(T.codes, T.sz, row, T.group, part, words, s, n_sz);
-    else store_lane<2>(T.codes, T.sz, row, T.group, part, words, s, n_sz);
+}
+
+// Quantize the lane's 64 channels in groups of G (16, 32, 64; or 128, shared
+// with the partner lane) and pack them: words[0 .. 64 * BITS / 32), and in
+// szb[b] the (scale, zero) pair of the group of 16-channel block b.
+// Extremes are taken per 16-channel block and combined within each group;
+// the group's parameters are computed once, at its first block. HYB: each
+// group takes the symmetric grid when its largest error is smaller (two
+// passes: errors, then codes).
+template <int BITS, bool HYB>
+__device__ __forceinline__ void quant_pack_half(const float2 v[32], int G, uint32_t words[8], __half2 szb[4]) {
+    constexpr int L = (1 << BITS) - 1;
+    const int bpg = G >> 4;  // 16-channel blocks per group
+    float mn[4], mx[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        float lo = fminf(v[8 * b].x, v[8 * b].y), hi = fmaxf(v[8 * b].x, v[8 * b].y);
+#pragma unroll
+        for (int k = 8 * b + 1; k < 8 * b + 8; ++k) {
+            lo = fminf(lo, fminf(v[k].x, v[k].y));
+            hi = fmaxf(hi, fmaxf(v[k].x, v[k].y));
+        }
+        mn[b] = lo;
+        mx[b] = hi;
+    }
+#pragma unroll
+    for (int step = 1; step < 4; step <<= 1) {  // every block gets its group's extremes
+        if (step < bpg) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if ((b & step) == 0) {
+                    const float lo = fminf(mn[b], mn[b | step]), hi = fmaxf(mx[b], mx[b | step]);
+                    mn[b] = lo; mn[b | step] = lo;
+                    mx[b] = hi; mx[b | step] = hi;
+                }
+        }
+    }
+    if (G == 128) {  // the group spans both lanes of the vector
+        const float lo = fminf(mn[0], __shfl_xor_sync(0xffffffffu, mn[0], 1));
+        const float hi = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], 1));
+#pragma unroll
+        for (int b = 0; b < 4; ++b) { mn[b] = lo; mx[b] = hi; }
+    }
+    const int lbpg = bpg < 4 ? bpg : 4;  // blocks per group within the lane
+    float zf[4], rf[4], sf[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        if (b == 0 || (b & (lbpg - 1)) == 0) {
+            const QParams p = qparams(mn[b], mx[b], L);
+            zf[b] = p.zf; rf[b] = p.r; sf[b] = p.sf;
+            szb[b] = p.sz;
+        } else {
+            zf[b] = zf[b - 1]; rf[b] = rf[b - 1]; sf[b] = sf[b - 1];
+            szb[b] = szb[b - 1];
+        }
+    }
+    bool sym[4] = {false, false, false, false};
+    SymParams ps[4];
+    if constexpr (HYB) {
+        float ea[4], es[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (b == 0 || (b & (lbpg - 1)) == 0) ps[b] = sym_params(mn[b], mx[b], BITS);
+            else ps[b] = ps[b - 1];
+            QParams pa;
+            pa.zf = zf[b]; pa.r = rf[b];
+            float a = 0.0f, e = 0.0f;
+#pragma unroll
+            for (int k = 8 * b; k < 8 * b + 8; ++k) {
+                a = max_err(v[k].x, qcode(v[k].x, pa, static_cast<float>(L)), sf[b], zf[b], a);
+                a = max_err(v[k].y, qcode(v[k].y, pa, static_cast<float>(L)), sf[b], zf[b], a);
+                e = max_err(v[k].x, sym_code(v[k].x, ps[b], BITS), ps[b].sf, ps[b].zf, e);
+                e = max_err(v[k].y, sym_code(v[k].y, ps[b], BITS), ps[b].sf, ps[b].zf, e);
+            }
+            ea[b] = a;
+            es[b] = e;
+        }
+#pragma unroll
+        for (int step = 1; step < 4; step <<= 1) {
+            if (step < bpg) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    if ((b & step) == 0) {
+                        const float a = fmaxf(ea[b], ea[b | step]), e = fmaxf(es[b], es[b | step]);
+                        ea[b] = a; ea[b | step] = a;
+                        es[b] = e; es[b | step] = e;
+                    }
+            }
+        }
+        if (G == 128) {
+            const float a = fmaxf(ea[0], __shfl_xor_sync(0xffffffffu, ea[0], 1));
+            const float e = fmaxf(es[0], __shfl_xor_sync(0xffffffffu, es[0], 1));
+#pragma unroll
+            for (int b = 0; b < 4; ++b) { ea[b] = a; es[b] = e; }
+        }
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            sym[b] = ps[b].ok && es[b] < ea[b];
+            if (sym[b]) szb[b] = ps[b].sz;
+        }
+    }
+    // codes, packed: INT4 byte i = q[2i] | q[2i+1] << 4; INT2 byte i holds
+    // q[4i + j] in bits 2j..2j+1
+    const unsigned long long magic = f2u(8388608.0f, 8388608.0f);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        uint32_t q[16];
+        if (HYB && sym[b]) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                q[2 * k] = sym_code(v[8 * b + k].x, ps[b], BITS);
+                q[2 * k + 1] = sym_code(v[8 * b + k].y, ps[b], BITS);
+            }
+        } else {
+            // q = rint_even(fp32(fp32(x - z) * r)) through the 2^23 trick; the
+            // lower clamp maps NaN to 0 (the upper one never binds)
+            const unsigned long long z2 = f2u(zf[b], zf[b]), r2 = f2u(rf[b], rf[b]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float2 t = f2_of(mul2(sub2(u64_of(v[8 * b + k]), z2), r2));
+                const float2 y = f2_of(add2(u64_of(make_float2(fmaxf(t.x, 0.0f), fmaxf(t.y, 0.0f))), magic));
+                q[2 * k] = __float_as_uint(y.x);
+                q[2 * k + 1] = __float_as_uint(y.y);
+            }
+        }
+        if constexpr (BITS == 4) {
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+                const uint32_t *c = q + 8 * w;
+                const uint32_t e = __byte_perm(__byte_perm(c[0], c[2], 0x0040), __byte_perm(c[4], c[6], 0x0040), 0x5410);
+                const uint32_t o = __byte_perm(__byte_perm(c[1], c[3], 0x0040), __byte_perm(c[5], c[7], 0x0040), 0x5410);
+                words[2 * b + w] = e + (o << 4);
+            }
+        } else {
+            uint32_t wv = 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) wv |= (q[j] & 3u) << (2 * j);
+            words[b] = wv;
+        }
+    }
+}
+
+template <int DT, bool HYB>
+__global__ void __launch_bounds__(kAppendWarps * 32, kAppendBlocksPerSm) append_rows_kernel(const AppendParams p) {
+    pdl_launch_dependents();  // the length advance may be scheduled; it waits for us
+    using SR = StagedRows<DT>;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const AppendTensor &T = p.t[blockIdx.y];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = lane & 1;
+    uint8_t *bufs = smem + warp * kAppendStages * SR::batch;
+    const int64_t n_vec = static_cast<int64_t>(p.total_tokens) * p.H;
+    const int64_t n_batches = (n_vec + 15) / 16;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kAppendWarps;
+    int64_t b = static_cast<int64_t>(blockIdx.x) * kAppendWarps + warp;
+    if (b >= n_batches) return;
+    const int dst_lane = stage_offset<DT>(lane);
+    // the first kAppendStages - 1 batches in flight (a commit per slot, empty
+    // groups past the end, so the wait count below is always the same)
+#pragma unroll
+    for (int j = 0; j < kAppendStages - 1; ++j) {
+        if (b + j * stride < n_batches)
+            stage_batch<DT>(T.src, b + j * stride, n_vec, bufs + j * SR::batch, dst_lane, lane);
+        cp_async_commit();
+    }
+    for (int i = 0; b < n_batches; ++i, b += stride) {
+        const uint8_t *cur = bufs + (i % kAppendStages) * SR::batch;
+        const int64_t ahead = b + (kAppendStages - 1) * stride;
+        if (ahead < n_batches)
+            stage_batch<DT>(T.src, ahead, n_vec, bufs + ((i + kAppendStages - 1) % kAppendStages) * SR::batch,
+                            dst_lane, lane);
+        cp_async_commit();
+        cp_async_wait<kAppendStages - 1>();
+        __syncwarp();
+        // idle lanes of a short last batch work on a copy of the batch's
+        // first vector (both lanes of a pair stay together for the exchanges)
+        const int64_t vraw = b * 16 + (lane >> 1);
+        const bool active = vraw < n_vec;
+        const int t = active ? (lane >> 1) : 0;
+        const int64_t vec = b * 16 + t;
+        float2 v[32];
+        read_half<DT>(cur + t * SR::stride + half * SR::half_stride, v);
+        __syncwarp();  // every lane has read its row: the buffer may be refilled
+        const uint32_t vec32 = static_cast<uint32_t>(vec);  // n_vec < 2^31 (host check)
+        const int tok = static_cast<int>(vec32 / static_cast<uint32_t>(p.H));
+        const int h = static_cast<int>(vec32 - static_cast<uint32_t>(tok) * static_cast<uint32_t>(p.H));
+        const int seq = find_seq(p.cu_new, p.num_seqs, tok);
+        const int pos = __ldg(p.seq_lens + seq) + (tok - __ldg(p.cu_new + seq));
+        const bool sink = pos >= 0 && pos < p.sink_len;  // the same for both lanes of a pair
+        if (sink) {
+            // attention-sink token: kept as the input rounded to bf16, not quantized
+            if (active) {
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    p.sink[blockIdx.y] + ((static_cast<int64_t>(seq) * p.H + h) * p.sink_len + pos) * kHeadDim +
+                    half * 64);
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4 * i4 + j].x, v[4 * i4 + j].y);
+                        w[j] = *reinterpret_cast<const uint32_t *>(&b2);
+                    }
+                    dst[i4] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            continue;
+        }
+        if (T.signs != nullptr) {  // randomized Hadamard: diag(signs) first (exact)
+            const float2 *sg = reinterpret_cast<const float2 *>(T.signs) + half * 32;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float2 s2 = __ldg(sg + k);
+                v[k].x *= s2.x;
+                v[k].y *= s2.y;
+            }
+        }
+        if (T.hb > 0) fwht_half_any(v, T.hb, half, T.hscale);
+        uint32_t words[8];
+        __half2 szb[4];
+        if (T.bits == 4) quant_pack_half<4, HYB>(v, T.group, words, szb);
+        else quant_pack_half<2, HYB>(v, T.group, words, szb);
+        if (!active) continue;
+        int64_t drow;
+        if (!dest_row(p, seq, pos, h, drow)) {
+            if (half == 0) status_or(p.status, KVQ_DEV_CAPACITY);
+            continue;
+        }
+        if (T.bits == 4) {
+            uint4 *dst = reinterpret_cast<uint4 *>(T.codes + drow * 64 + half * 32);
+            dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+            dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+        } else {
+            *reinterpret_cast<uint4 *>(T.codes + drow * 32 + half * 16) =
+                make_uint4(words[0], words[1], words[2], words[3]);
+        }
+        // the pairs of the groups that start in this lane: group (64 half + 16 b) / G
+        const int ng = kHeadDim / T.group;
+        __half2 *srow = T.sz + drow * ng;
+        const int bpg = T.group >> 4;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int blk = 4 * half + b;  // 16-channel block of the row
+            if ((blk & (bpg - 1)) == 0) srow[blk / bpg] = szb[b];
+        }
+    }
 }
 
 // ---- residual window: flush full blocks, then write the window ------------
@@ -632,6 +977,17 @@ __global__ void advance_lens_kernel(const int32_t *cu_new, int32_t *seq_lens, in
     if (s < num_seqs) seq_lens[s] += cu_new[s + 1] - cu_new[s];
 }
 
+template <int DT, bool HYB>
+kvq_status launch_rows(dim3 grid, const AppendParams &p, cudaStream_t stream) {
+    const size_t smem = static_cast<size_t>(kAppendWarps) * kAppendStages * StagedRows<DT>::batch;
+    auto kern = append_rows_kernel<DT, HYB>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    kern<<<grid, kAppendWarps * 32, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -689,22 +1045,26 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
         p.sink[1] = static_cast<uint16_t *>(d.v_sink);
         p.sink_len = d.sink_len;
         const int64_t n_vec = static_cast<int64_t>(total_new) * d.num_kv_heads;
-        const dim3 grid(static_cast<unsigned>((n_vec + 63) / 64), has_v ? 2 : 1);
+        if (n_vec >= (int64_t(1) << 31)) return KVQ_ERR_UNSUPPORTED;  // vector indices are 32-bit
+        const int64_t n_batches = (n_vec + 15) / 16;
+        int sms = 148, dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t blocks = std::min<int64_t>((n_batches + kAppendWarps - 1) / kAppendWarps,
+                                                 static_cast<int64_t>(kAppendBlocksPerSm) * std::max(sms, 1));
+        const dim3 grid(static_cast<unsigned>(blocks), has_v ? 2 : 1);
+        kvq_status st = KVQ_OK;
         switch (dtype) {
             case KVQ_BF16:
-                if (d.hybrid) append_tokens_kernel<KVQ_BF16, true><<<grid, 256, 0, stream>>>(p);
-                else append_tokens_kernel<KVQ_BF16, false><<<grid, 256, 0, stream>>>(p);
+                st = d.hybrid ? launch_rows<KVQ_BF16, true>(grid, p, stream) : launch_rows<KVQ_BF16, false>(grid, p, stream);
                 break;
             case KVQ_FP16:
-                if (d.hybrid) append_tokens_kernel<KVQ_FP16, true><<<grid, 256, 0, stream>>>(p);
-                else append_tokens_kernel<KVQ_FP16, false><<<grid, 256, 0, stream>>>(p);
+                st = d.hybrid ? launch_rows<KVQ_FP16, true>(grid, p, stream) : launch_rows<KVQ_FP16, false>(grid, p, stream);
                 break;
             default:
-                if (d.hybrid) append_tokens_kernel<KVQ_FP32, true><<<grid, 256, 0, stream>>>(p);
-                else append_tokens_kernel<KVQ_FP32, false><<<grid, 256, 0, stream>>>(p);
+                st = d.hybrid ? launch_rows<KVQ_FP32, true>(grid, p, stream) : launch_rows<KVQ_FP32, false>(grid, p, stream);
                 break;
         }
-        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+        if (st != KVQ_OK) return st;
     }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((num_seqs + 127) / 128);
