@@ -15,6 +15,8 @@
 // that has to start at zero (the item counter) on the stream. Calls whose
 // work overlaps on the GPU (other streams, or other host threads) race on the
 // array.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "kvq_common.cuh"
@@ -31,22 +33,58 @@ constexpr int kMaxDevices = 64;
 // below.
 __device__ __align__(256) unsigned char g_static_workspace[kStaticBytes];
 
-std::mutex g_lock;
-void *g_address[kMaxDevices];
+// The array's device address is valid in the context that loaded the module.
+// The lookups are cached per device together with the context they were made
+// in (read through the driver's cuCtxGetCurrent, reached via the runtime's
+// entry-point query so the library needs no link to the driver), and made
+// again when a different context is current on that device: a plugin that
+// runs in its own context, or a context created after cudaDeviceReset.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
 
-// Device address of the array on the current device, looked up once per
-// device (the first call on a device performs this set-up).
+struct Cached {
+    CUcontext ctx;
+    void *ptr;
+};
+std::mutex g_lock;
+Cached g_cache[kMaxDevices];
+CtxGetCurrentFn g_ctx_get = nullptr;
+bool g_ctx_get_looked_up = false;
+
+// The current context, or nullptr when it cannot be read (then nothing is
+// cached and every call looks the address up).
+CUcontext current_context() {
+    if (!g_ctx_get_looked_up) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get = reinterpret_cast<CtxGetCurrentFn>(fn);
+        g_ctx_get_looked_up = true;
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_get == nullptr || g_ctx_get(&ctx) != CUDA_SUCCESS) return nullptr;
+    return ctx;
+}
+
+// Device address of the array in the current context of the current device.
+// The first call on a device (and in each further context) performs this
+// set-up.
 kvq_status static_workspace(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
     std::lock_guard<std::mutex> guard(g_lock);
-    if (g_address[dev] == nullptr) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_static_workspace) != cudaSuccess || ptr == nullptr)
-            return KVQ_ERR_CUDA;
-        g_address[dev] = ptr;
+    CUcontext ctx = current_context();
+    if (ctx != nullptr && g_cache[dev].ctx == ctx && g_cache[dev].ptr != nullptr) {
+        *out = g_cache[dev].ptr;
+        return KVQ_OK;
     }
-    *out = g_address[dev];
+    // the lookup also makes the device's primary context current on this
+    // thread when no context was yet
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_workspace) != cudaSuccess || ptr == nullptr) return KVQ_ERR_CUDA;
+    if (ctx == nullptr) ctx = current_context();
+    g_cache[dev] = Cached{ctx, ptr};  // ctx == nullptr: never matches, looked up on every call
+    *out = ptr;
     return KVQ_OK;
 }
 

@@ -20,6 +20,12 @@ class DecodeStep:
     the caller refills them before every run. seq_lens, cu_new: device int32
     (seq_lens advances by the appended tokens on every run). The output lands
     in `out_host` (pinned fp32 [S][Hq][128]) once the stream is synchronized.
+
+    max_seq_len is fixed at capture: a replay that took a sequence past it
+    would make attention leave out its newest tokens (the kernels clamp and
+    flag KVQ_DEV_SEQLEN in the status word). So the step counts its replays
+    against the lengths it last read and `run()` raises before one would
+    overflow; after changing seq_lens by other means, call `sync_lengths()`.
     """
 
     def __init__(self, desc, seq_lens, cu_new, max_seq_len: int, softmax_scale: float, k_host, v_host,
@@ -54,6 +60,20 @@ class DecodeStep:
         with torch.cuda.graph(self.graph, stream=side, capture_error_mode="thread_local"):
             self._body()
         torch.cuda.current_stream(dev).wait_stream(side)
+        self.sync_lengths()
+
+    def sync_lengths(self) -> None:
+        """Read seq_lens and cu_new (one device synchronization) and recount
+        the replays left before a sequence would pass max_seq_len."""
+        lens = self.seq_lens.cpu().tolist()
+        cu = self.cu_new.cpu().tolist()
+        left = None
+        for s, t in enumerate(lens):
+            inc = cu[s + 1] - cu[s]
+            if inc > 0:
+                n = max(0, (self.max_seq_len - t) // inc)
+                left = n if left is None else min(left, n)
+        self.replays_left = left  # None: no sequence grows
 
     def _body(self):
         self.dk.copy_(self.k_host, non_blocking=True)
@@ -65,5 +85,11 @@ class DecodeStep:
         self.out_host.copy_(self.out, non_blocking=True)
 
     def run(self) -> None:
-        """Replay the step on the current stream (asynchronous)."""
+        """Replay the step on the current stream (asynchronous). Raises
+        before a replay would take a sequence past max_seq_len."""
+        if self.replays_left is not None:
+            if self.replays_left <= 0:
+                raise RuntimeError("DecodeStep: the next replay would take a sequence past max_seq_len=%d "
+                                   "(call sync_lengths() after changing seq_lens)" % self.max_seq_len)
+            self.replays_left -= 1
         self.graph.replay()

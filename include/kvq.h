@@ -297,8 +297,10 @@ KVQ_API kvq_status kvq_merge_partials(const float *parts, int32_t n_part, int32_
  * declares; it is reserved on every GPU that loads the library until the
  * process exits. Sizes whose workspace (kvq_decode_workspace_size) exceeds
  * 16 MiB are rejected with KVQ_ERR_CAPACITY before anything is launched.
- * The first call on a device looks up the array's device address (once per
- * device); make that first call before any stream capture. All calls share the
+ * The first call on a device looks up the array's device address (again
+ * whenever another context is current on that device, e.g. after
+ * cudaDeviceReset or inside a plugin's own context); make the first call in
+ * each context before any stream capture. All calls share the
  * array and it keeps the previous call's contents (what must start at zero is
  * cleared on the stream by each call), so calls whose work overlaps on the GPU
  * -- on different streams or from different host threads -- race on it.
