@@ -58,7 +58,8 @@ def flush_l2(buf):
     buf.amax()
 # the timed split-K variant: the kernel template and the unit that instantiates it
 DECODE_SRC = [os.path.join(ROOT, "bit_kv_cache_21_b200", "csrc", f)
-              for f in ("kvq_decode_kernel.cuh", "kvq_decode_plain.cu")]
+              for f in ("kvq_decode_kernel.cuh", "kvq_decode_plain.cu", "kvq_decode.cu", "kvq_common.cuh",
+                        "kvq_internal.h")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_splitk_llama8b_traffic.json")
 
 
@@ -319,14 +320,39 @@ def run_ours(args, rank, world, local_rank):
         if i >= args.warmup:
             e2e_s.append(t1 - t0)
             e2e_bytes += (CTX + j + 1) * BATCH * HKV * BYTES_PER_TOKEN_HEAD
+    # Where the end-to-end time goes, from a separate pass of the same steps
+    # (events would perturb the timed one): device time of the graph replay
+    # (copies + kernels) against the host's wall time around replay + wait.
+    bd_wall, bd_dev = [], []
+    n_bd = min(EPISODE, max(8, args.steps // 4))
+    lens.copy_(ctx_lens)
+    for gs in graph_steps:
+        gs.sync_lengths()
+    for j in range(n_bd):
+        flush_l2(flush)
+        torch.cuda.synchronize()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        ea.record(stream)
+        graph_steps[j].run()
+        eb.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        bd_wall.append((t1 - t0) * 1e6)
+        bd_dev.append(ea.elapsed_time(eb) * 1e3)
     assert cache.device_status() == 0, "device status %d after the graph steps" % cache.device_status()
+    kernels_us = statistics.mean(step_ms) * 1e3
+    e2e_breakdown = {"steps": n_bd, "host_wall_us": statistics.mean(bd_wall),
+                     "graph_device_us": statistics.mean(bd_dev), "kernels_device_us": kernels_us,
+                     "copies_and_gaps_us": statistics.mean(bd_dev) - kernels_us,
+                     "host_launch_and_wait_us": statistics.mean(bd_wall) - statistics.mean(bd_dev)}
     h2d = hk[0].numel() * 2 + hv[0].numel() * 2 + hq[0].numel() * 2
     d2h = hout.numel() * 4
 
     res = {"total_ms": total_ms, "bytes": bytes_total, "split_ms": split_ms, "attn_ms": attn_ms,
            "split_bytes": split_bytes,
            "append1_ms": append1_ms, "step_ms": step_ms, "clocks": clocks.summary(),
-           "append": append_info, "e2e_s": sum(e2e_s), "e2e_bytes": e2e_bytes,
+           "append": append_info, "e2e_s": sum(e2e_s), "e2e_bytes": e2e_bytes, "e2e_breakdown": e2e_breakdown,
            "h2d": h2d, "d2h": d2h, "tokens": tokens}
     return res
 
@@ -1079,7 +1105,8 @@ def main():
                                                "sample": "%d units cycling over 16 (%.1f s)"
                                                          % (cpu_done, cpu_s)}},
             "e2e": {"value": e2e_bytes / e2e_s / 1e9, "unit": "GB/s",
-                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                    "breakdown": res["e2e_breakdown"]},
             "gpu_launches": 4 * args.steps,   # append, advance lengths, split-K, merge
             "clocks": res["clocks"],
         }
