@@ -86,7 +86,7 @@ constexpr int kBarBytes = 512;
 constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kRingBytes) + kBarBytes;
 
 static_assert(kBBytes % 1024 == 0 && kOffStage % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-static_assert(kOffCRing % 128 == 0 && kCStageBytes % 128 == 0, "TMA destination alignment");
+static_assert(kOffCRing % 256 == 0 && kCStageBytes % 256 == 0, "TMA destination alignment (32-byte swizzle)");
 static_assert(kNumBars * 8 + 8 <= kBarBytes, "barrier area");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(kCStages % kDeqGroups == 0, "a codes slot always goes to the same group");
@@ -275,16 +275,20 @@ __device__ __forceinline__ float two_sum_err(float a, float b) {
     return __fadd_rn(__fsub_rn(a, ap), __fsub_rn(b, bp));
 }
 
-// One row's 32 code bytes and its scale/zero word from shared memory.
-__device__ __forceinline__ void lds_codes(const uint8_t *codes, const uint8_t *sz, uint4 &c0, uint4 &c1,
+// One row's 32 code bytes and its scale/zero word from shared memory. The
+// codes box lands with the 32-byte swizzle: 16-byte chunk c of row r sits at
+// chunk c ^ ((r >> 2) & 1), so the eight rows of a shared-memory phase (32
+// bytes apart) hit eight distinct bank groups.
+__device__ __forceinline__ void lds_codes(const uint8_t *codes, int r, const uint8_t *sz, uint4 &c0, uint4 &c1,
                                           uint32_t &szw) {
+    const int f = (r >> 2) & 1;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(c0.x), "=r"(c0.y), "=r"(c0.z), "=r"(c0.w)
-                 : "r"(smem_addr(codes))
+                 : "r"(smem_addr(codes + 16 * f))
                  : "memory");
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(c1.x), "=r"(c1.y), "=r"(c1.z), "=r"(c1.w)
-                 : "r"(smem_addr(codes + 16))
+                 : "r"(smem_addr(codes + 16 * (f ^ 1)))
                  : "memory");
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(szw) : "r"(smem_addr(sz)) : "memory");
 }
@@ -539,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t *cs = c_ring + sc * kCStageBytes;
                 uint4 c0, c1;
                 uint32_t szw;
-                lds_codes(cs + row * 32, cs + kCodeBytes + row * 4, c0, c1, szw);
+                lds_codes(cs + row * 32, row, cs + kCodeBytes + row * 4, c0, c1, szw);
                 const __half2 sz = *reinterpret_cast<const __half2 *>(&szw);
                 uint32_t xv[32];
                 dequant_row(c0, c1, __low2float(sz), __high2float(sz), xv);
@@ -907,7 +911,7 @@ kvq_status launch_remat(const kvq_cache_desc &x, const void *w_kv, int n_kv_head
     if (!make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_kv, hidden, n_rows, hidden * 2,
                      kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, x.k_codes, kHeadDim / 2, code_rows,
-                     kHeadDim / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     kHeadDim / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
         return KVQ_ERR_CUDA;
     // Outputs [B][H][T][128] bf16 as rows of 128 channels, stored in boxes of
     // 128 positions x 64 channels.
@@ -956,7 +960,7 @@ kvq_status launch_remat_attention(const kvq_cache_desc &x, const void *w_kv, int
     if (!make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_kv, hidden, n_rows, hidden * 2,
                      kBK, kHeadDim, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, x.k_codes, kHeadDim / 2, code_rows,
-                     kHeadDim / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     kHeadDim / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_32B))
         return KVQ_ERR_CUDA;
     RematParams p{};
     p.x_sz = static_cast<const __half2 *>(x.k_sz);
