@@ -162,7 +162,8 @@ kvq_status kvq_decode_merge(const kvq_cache_desc *desc, int32_t num_q_heads,
                             void *stream) {
     kvq_status s = validate_desc(desc, true);
     if (s != KVQ_OK) return s;
-    if (out == nullptr || seq_lens == nullptr || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)
+    if (out == nullptr || !aligned16(out) || seq_lens == nullptr || num_seqs <= 0 || num_q_heads <= 0 ||
+        max_seq_len < 0)
         return KVQ_ERR_INVALID_ARG;
     DecodePlan plan;
     if (!plan_decode(*desc, num_seqs, num_q_heads, max_seq_len, &plan)) return KVQ_ERR_INVALID_ARG;
@@ -203,7 +204,7 @@ kvq_status kvq_decode_attention(const kvq_cache_desc *desc, const void *q, kvq_d
                                 int32_t num_q_heads, const int32_t *seq_lens, int32_t num_seqs,
                                 int32_t max_seq_len, float softmax_scale, float *out,
                                 void *workspace, size_t workspace_bytes, void *stream) {
-    if (out == nullptr) return KVQ_ERR_INVALID_ARG;
+    if (out == nullptr || !aligned16(out)) return KVQ_ERR_INVALID_ARG;
     kvq_status s = kvq_decode_splitk(desc, q, q_dtype, num_q_heads, seq_lens, num_seqs,
                                      max_seq_len, softmax_scale, workspace, workspace_bytes, stream);
     if (s != KVQ_OK) return s;

@@ -123,26 +123,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
-// The same bounded wait for a warp whose wake-up is not latency critical: it
-// sleeps about `sleep_ns` between polls, so a long wait costs fewer issue
-// slots of the warps that share its scheduler.
-__device__ __forceinline__ bool mbar_wait_backoff(uint64_t *bar, uint32_t parity, int64_t timeout_ns,
-                                                  int32_t *status, volatile int *abort_flag,
-                                                  uint32_t sleep_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        __nanosleep(sleep_ns);
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (static_cast<int64_t>(global_timer_ns() - t0) > timeout_ns) {
-            status_or(status, KVQ_DEV_TIMEOUT);
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
-
 // Programmatic dependent launch: let the next kernel of the stream (launched
 // with programmatic stream serialization) be scheduled now; and, in that
 // kernel, wait until the previous grid has completed and its writes are
@@ -245,6 +225,60 @@ __device__ __forceinline__ void combine_partials(const float *o_part, const floa
             o += sm.o[g][d];
             l += sm.l[g];
         }
+    }
+}
+
+// The same combination by a CTA of 32 * NW threads with one partial per warp
+// at a time: warp w takes the partials j = w, w + NW, ..., lane i channels
+// 4i..4i+3 of each, so every o load is 16 bytes and NW partials are read per
+// step (the loop is unrolled, several steps in flight). o rows must be 16-byte
+// aligned (o0 and o_step multiples of 4). The warps' sums are added in warp
+// order; the results are valid in warp 0 (o = channels 4*lane..4*lane+3).
+template <int NW>
+struct CombineSmemW {
+    float4 o[NW][32];
+    float l[NW];
+    float red[NW];
+};
+
+template <int NW>
+__device__ __forceinline__ void combine_partials_w(const float *o_part, const float2 *ml, int64_t o0,
+                                                   int64_t o_step, int64_t m0, int64_t m_step, int n,
+                                                   CombineSmemW<NW> &sm, float &M, float4 &o, float &l) {
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    float m = -INFINITY;
+    for (int j = t; j < n; j += NW * 32) m = fmaxf(m, ml[m0 + j * m_step].x);
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, k));
+    if (lane == 0) sm.red[w] = m;
+    __syncthreads();
+    float mm = sm.red[0];
+#pragma unroll
+    for (int k = 1; k < NW; ++k) mm = fmaxf(mm, sm.red[k]);
+    M = mm;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float ll = 0.0f;
+#pragma unroll 4
+    for (int j = w; j < n; j += NW) {
+        const float2 v = ml[m0 + j * m_step];
+        const float4 ov = *reinterpret_cast<const float4 *>(o_part + o0 + j * o_step + 4 * lane);
+        const float e = (v.x == -INFINITY) ? 0.0f : fast_exp2(v.x - M);
+        acc.x = fmaf(e, ov.x, acc.x);
+        acc.y = fmaf(e, ov.y, acc.y);
+        acc.z = fmaf(e, ov.z, acc.z);
+        acc.w = fmaf(e, ov.w, acc.w);
+        ll = fmaf(e, v.y, ll);
+    }
+    sm.o[w][lane] = acc;
+    if (lane == 0) sm.l[w] = ll;
+    __syncthreads();
+    o = sm.o[0][lane];
+    l = sm.l[0];
+#pragma unroll
+    for (int k = 1; k < NW; ++k) {
+        const float4 b = sm.o[k][lane];
+        o.x += b.x; o.y += b.y; o.z += b.z; o.w += b.w;
+        l += sm.l[k];
     }
 }
 

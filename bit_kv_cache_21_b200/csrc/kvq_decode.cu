@@ -14,35 +14,39 @@ namespace kvq {
 using namespace dec;
 
 namespace {
-// One CTA of 128 threads per (query head, sequence): combine the splits into
-// the output, or (PARTIAL) into this cache's unnormalized partial (o, m, l)
-// for a merge with the partials of other caches that hold other token ranges
-// of the same sequences. Launched as a programmatic dependent of the split-K
-// pass: its CTAs may start while that pass drains and wait here until its
-// partials are complete.
-constexpr int kMergeGroups = 4;  // partial groups per merge CTA (128 threads each)
+// One CTA of 32 * NW threads per (query head, sequence): combine the splits
+// into the output, or (PARTIAL) into this cache's unnormalized partial
+// (o, m, l) for a merge with the partials of other caches that hold other
+// token ranges of the same sequences. Launched as a programmatic dependent of
+// the split-K pass: its CTAs may start while that pass drains and wait here
+// until its partials are complete. NW partials are read per step (one per
+// warp, 16 bytes per lane): 4 warps for up to kMergeFewSplits splits, else 16
+// (long sequences have few rows and many splits).
+constexpr int kMergeFewSplits = 32;
 
-template <bool PARTIAL>
-__global__ void __launch_bounds__(128 * kMergeGroups) decode_merge_kernel(const float *o_part, const float2 *ml,
+template <bool PARTIAL, int NW>
+__global__ void __launch_bounds__(32 * NW) decode_merge_kernel(const float *o_part, const float2 *ml,
                                                            const int32_t *seq_lens, float *out,
                                                            float2 *out_ml, int Hq, int max_seq_len,
                                                            const __grid_constant__ SplitBounds sp) {
-    __shared__ CombineSmem<kMergeGroups> sm;
+    __shared__ CombineSmemW<NW> sm;
     pdl_wait_prior_grid();
-    const int hq = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
+    const int hq = blockIdx.x, seq = blockIdx.y;
     const int T = min(__ldg(seq_lens + seq), max_seq_len);
     const int nv = splits_of(sp, T);
     const int n_split = sp.n;
     const int64_t row = static_cast<int64_t>(seq) * Hq + hq;
-    float M, o, l;
-    combine_partials<kMergeGroups>(o_part, ml, row * n_split * kHeadDim, kHeadDim, row * n_split, 1, nv, sm, M,
-                                   o, l);
-    if (d >= kHeadDim) return;
+    float M, l;
+    float4 o;
+    combine_partials_w<NW>(o_part, ml, row * n_split * kHeadDim, kHeadDim, row * n_split, 1, nv, sm,
+                                    M, o, l);
+    if (threadIdx.x >= 32) return;
+    float4 *dst = reinterpret_cast<float4 *>(out + row * kHeadDim) + threadIdx.x;
     if constexpr (PARTIAL) {
-        out[row * kHeadDim + d] = o;
-        if (d == 0) out_ml[row] = make_float2(M, l);
+        *dst = o;
+        if (threadIdx.x == 0) out_ml[row] = make_float2(M, l);
     } else {
-        out[row * kHeadDim + d] = (l > 0.0f) ? o / l : 0.0f;
+        *dst = (l > 0.0f) ? make_float4(o.x / l, o.y / l, o.z / l, o.w / l) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
 }
 
@@ -168,9 +172,10 @@ kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, 
     const float *o_part = static_cast<const float *>(workspace);
     const float2 *ml =
         reinterpret_cast<const float2 *>(static_cast<const uint8_t *>(workspace) + plan.ws_part);
+    const bool few = plan.n_split <= kMergeFewSplits;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(num_q_heads, num_seqs);
-    cfg.blockDim = dim3(128 * kMergeGroups);
+    cfg.blockDim = dim3(few ? 128 : 512);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -179,11 +184,18 @@ kvq_status launch_decode_merge(const kvq_cache_desc &d, const DecodePlan &plan, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     float2 *oml = reinterpret_cast<float2 *>(out_ml);
-    const cudaError_t e =
-        out_ml ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<true>, o_part, ml, seq_lens, out, oml,
-                                    num_q_heads, max_seq_len, plan.splits)
-               : cudaLaunchKernelEx(&cfg, decode_merge_kernel<false>, o_part, ml, seq_lens, out, oml,
-                                    num_q_heads, max_seq_len, plan.splits);
+    const SplitBounds &sp = plan.splits;
+    cudaError_t e;
+    if (out_ml)
+        e = few ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<true, 4>, o_part, ml, seq_lens, out, oml, num_q_heads,
+                                     max_seq_len, sp)
+                : cudaLaunchKernelEx(&cfg, decode_merge_kernel<true, 16>, o_part, ml, seq_lens, out, oml,
+                                     num_q_heads, max_seq_len, sp);
+    else
+        e = few ? cudaLaunchKernelEx(&cfg, decode_merge_kernel<false, 4>, o_part, ml, seq_lens, out, oml,
+                                     num_q_heads, max_seq_len, sp)
+                : cudaLaunchKernelEx(&cfg, decode_merge_kernel<false, 16>, o_part, ml, seq_lens, out, oml,
+                                     num_q_heads, max_seq_len, sp);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

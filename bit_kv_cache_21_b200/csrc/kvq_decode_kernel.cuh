@@ -78,9 +78,6 @@ constexpr int kHelperWarp = kConsumerWarps + 1;    // query rows, coefficients, 
 constexpr int kThreads = kConsumers + 64;
 constexpr int kItemSlots = 2;      // items in flight per CTA (query rows and coefficients)
 constexpr int kDepStride = 132;    // floats per (warp, head) deposit: o[128], (m, l), pad
-// Polling intervals of the producer's and the helper's waits (ns): a stage is
-// consumed in microseconds, so these wake-ups are not on the critical path.
-constexpr uint32_t kProducerSleepNs = 256, kHelperSleepNs = 1024;
 constexpr int kMaxGroups = 8;      // kHeadDim / smallest token-wise group (16)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -971,17 +968,16 @@ decode_splitk_kernel(const DecodeParams p) {
             build_item_query<GQA, KM, KBF, GKC, SINK>(p, inf, slot, slot + QF, slot + (SINK ? 2 : 1) * QF, lane);
             mbar_arrive(&coef_full[j]);
         };
-        if (!mbar_wait_backoff(&posted[0], 0, p.timeout_ns, p.status, abort_flag, kHelperSleepNs)) return;
+        if (!mbar_wait_bounded(&posted[0], 0, p.timeout_ns, p.status, abort_flag)) return;
         if (info[0].done) return;
         build(0);
         for (int n = 0;; ++n) {
             const int j = n % kItemSlots, j1 = (n + 1) % kItemSlots;
-            if (!mbar_wait_backoff(&posted[j1], ((n + 1) / kItemSlots) & 1, p.timeout_ns, p.status, abort_flag,
-                                   kHelperSleepNs))
+            if (!mbar_wait_bounded(&posted[j1], ((n + 1) / kItemSlots) & 1, p.timeout_ns, p.status, abort_flag))
                 return;
             const bool more = !info[j1].done;
             if (more) build(j1);
-            if (!mbar_wait_backoff(deposited, n & 1, p.timeout_ns, p.status, abort_flag, kHelperSleepNs)) return;
+            if (!mbar_wait_bounded(deposited, n & 1, p.timeout_ns, p.status, abort_flag)) return;
             // merge the warps' states of item n: head g, 4 channels per lane
             const ItemInfo inf = info[j];
 #pragma unroll 1
@@ -1106,8 +1102,7 @@ decode_splitk_kernel(const DecodeParams p) {
                 const int j = n_item % kItemSlots, u = n_item / kItemSlots;
                 int ok = 1;
                 if (lane == 0 && u > 0)
-                    ok = mbar_wait_backoff(&slot_free[j], (u - 1) & 1, p.timeout_ns, p.status, abort_flag,
-                                           kProducerSleepNs);
+                    ok = mbar_wait_bounded(&slot_free[j], (u - 1) & 1, p.timeout_ns, p.status, abort_flag);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) break;
                 if (lane == 0) {
                     info[j] = ItemInfo{seq, kvh, split, item >= n_items ? 1 : 0};
@@ -1120,8 +1115,7 @@ decode_splitk_kernel(const DecodeParams p) {
                 const int s = it % NS, r = it / NS;
                 int ok = 1;
                 if (lane == 0 && r > 0)
-                    ok = mbar_wait_backoff(&empty[s], (r - 1) & 1, p.timeout_ns, p.status, abort_flag,
-                                           kProducerSleepNs);
+                    ok = mbar_wait_bounded(&empty[s], (r - 1) & 1, p.timeout_ns, p.status, abort_flag);
                 if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     stop = true;
                     break;

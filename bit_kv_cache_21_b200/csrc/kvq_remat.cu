@@ -251,11 +251,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-    return r;
-}
+// Byte permute through the intrinsic, so constant operands stay immediates.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) { return __byte_perm(a, b, sel); }
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     unsigned long long r;
@@ -811,15 +808,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// One CTA of 128 threads per (query head, sequence): the fused kernel's
-// per-tile partials combined into the output.
+// One CTA of 512 threads per (query head, sequence): the fused kernel's
+// per-tile partials combined into the output, one partial per warp at a time.
 __global__ void __launch_bounds__(512) remat_merge_kernel(const float *o_part, const float2 *ml, int n_blk,
                                                           float *out) {
-    __shared__ CombineSmem<4> sm;
+    __shared__ CombineSmemW<16> sm;
     const int64_t row = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
-    float M, o, l;
-    combine_partials<4>(o_part, ml, row * n_blk * kHeadDim, kHeadDim, row * n_blk, 1, n_blk, sm, M, o, l);
-    if (threadIdx.x < kHeadDim) out[row * kHeadDim + threadIdx.x] = (l > 0.0f) ? o / l : 0.0f;
+    float M, l;
+    float4 o;
+    combine_partials_w<16>(o_part, ml, row * n_blk * kHeadDim, kHeadDim, row * n_blk, 1, n_blk, sm, M, o, l);
+    if (threadIdx.x < 32)
+        reinterpret_cast<float4 *>(out + row * kHeadDim)[threadIdx.x] =
+            (l > 0.0f) ? make_float4(o.x / l, o.y / l, o.z / l, o.w / l) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
 // cos/sin(p * theta^(-2i/D)) in float64, rounded once to fp32.
