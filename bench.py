@@ -411,10 +411,11 @@ def run_remat(args, dev):
         step()
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.remat_steps)]
-    for i in range(args.remat_steps):
-        flush_l2(flush)
-        step(evs[i])
-    torch.cuda.synchronize()
+    with ClockSampler(dev) as remat_clocks:   # a GEMM under the 1 kW cap: the clock it ran at
+        for i in range(args.remat_steps):
+            flush_l2(flush)
+            step(evs[i])
+        torch.cuda.synchronize()
     assert cache.device_status() == 0 and int(status[0]) == 0
     remat_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
@@ -454,6 +455,7 @@ def run_remat(args, dev):
                                       "frac": flops / (fused * 1e-3) / 1e12 / peak_b,
                                       "speedup_vs_unfused": (remat_ms + attn_ms) / fused,
                                       "max_abs_diff_vs_unfused": fused_diff},
+            "clocks": remat_clocks.summary(),
             "gpu_launches_per_step": 4}
 
 

@@ -7,6 +7,8 @@
 // and R-token block, bf16), the code widths, compile-time group sizes and the
 // item's bf16 tail (none, the recent window, the attention sinks); each family
 // is instantiated in its own unit (kvq_decode_plain/window/innerq/sink.cu).
+#include <cmath>
+
 #include "kvq_decode_kernel.cuh"
 
 namespace kvq {
@@ -23,6 +25,12 @@ namespace {
 // warp, 16 bytes per lane): 4 warps for up to kMergeFewSplits splits, else 16
 // (long sequences have few rows and many splits).
 constexpr int kMergeFewSplits = 32;
+
+// Split plan: SMs of the B200 whose resident CTAs the items are balanced over,
+// items per resident CTA aimed at, and the longest split in tiles.
+constexpr int kBalanceSms = 148;
+constexpr double kMinItemsPerCta = 1.9, kMaxItemsPerCta = 4.5;
+constexpr int kMaxSplitTiles = 8;
 
 template <bool PARTIAL, int NW>
 __global__ void __launch_bounds__(32 * NW) decode_merge_kernel(const float *o_part, const float2 *ml,
@@ -69,24 +77,54 @@ __global__ void __launch_bounds__(128) merge_partials_kernel(const float *parts,
 bool plan_decode(const kvq_cache_desc &d, int num_seqs, int num_q_heads, int max_seq_len,
                  DecodePlan *plan) {
     if (num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0 || d.num_kv_heads <= 0) return false;
-    // Splits of `chunk` tokens, about four items per resident split-K CTA
-    // (two per SM) when every sequence is at max_seq_len: a multiple of the
-    // 256-token tile, 256..4096 tokens, and at most kMaxDecodeSplits splits.
-    // The CTAs claim items split-major (every unit's first split, then every
-    // unit's second, ...), so a sequence's last, partial split is among the
-    // last items claimed and fills the launch's tail. Measured on the
-    // llama8b-shaped step (16 x 8 units at 8256 tokens): chunks of 1024
-    // tokens split-major 90.7 us per split-K pass, 512 96.2, 2048 99.0, and
-    // splits that shrink from 3584 to 256 tokens 110.6. The plan depends on
-    // the sizes alone, so the workspace query and the launches agree.
+    // Every (sequence, KV head) unit is cut into splits of `chunk` tokens (1 to
+    // kMaxSplitTiles whole 256-token tiles), the last one partial; the CTAs
+    // claim the items split-major, so the partial splits come last. The chunk
+    // balances the launch with every sequence at max_seq_len: the full items
+    // should fill a whole number of rounds of the resident CTAs (two per SM
+    // on the B200's 148 SMs), 1.9..4.5 items per CTA;
+    // among the chunks that do, the most even one wins, then the one whose
+    // trailing split is the smallest share of a chunk. With more work than
+    // that the longest chunk is taken, with less the shortest. Measured on
+    // B200 (split-K pass): llama8b-shaped step, 128 units of 8256 tokens:
+    // 1024-token chunks 89.1 us, 768 94.4, 1280 95.3, 1536 95.9, 2048 97.9;
+    // long_int2, 8 units of 131072: 1792 107.2 us, 1280 116.5, 1024 117.9,
+    // 2048 122.6; paged_mix (ragged, split-K + merge): 2048 277.6 us, 3072
+    // 282.5, 4096 304.9. The plan depends on the sizes alone, so the workspace
+    // query and the launches agree.
     const int64_t units = static_cast<int64_t>(num_seqs) * d.num_kv_heads;
-    const int64_t target_items = 4 * 2 * 148;
     const int64_t L = std::max(1, max_seq_len);
-    int64_t chunk = (units * L + target_items - 1) / target_items;
-    chunk = (chunk + kTileQ - 1) / kTileQ * kTileQ;
-    chunk = std::min<int64_t>(std::max<int64_t>(chunk, kTileQ), 4096);
-    const int64_t floor_c = ((L + kMaxDecodeSplits - 1) / kMaxDecodeSplits + kTileQ - 1) / kTileQ * kTileQ;
-    chunk = std::max(chunk, floor_c);
+    const int64_t ctas = 2 * kBalanceSms;
+    // at most kMaxDecodeSplits splits
+    const int64_t m_floor = (L + static_cast<int64_t>(kMaxDecodeSplits) * kTileQ - 1) /
+                            (static_cast<int64_t>(kMaxDecodeSplits) * kTileQ);
+    int64_t m_best = -1;
+    double best_even = -1.0, best_tail = 2.0;
+    bool all_above = true;
+    for (int64_t m = std::max<int64_t>(1, m_floor); m <= std::max<int64_t>(m_floor, kMaxSplitTiles); ++m) {
+        const int64_t c = m * kTileQ;
+        const double k = static_cast<double>(units * (L / c)) / static_cast<double>(ctas);
+        if (k <= kMaxItemsPerCta) all_above = false;
+        if (k < kMinItemsPerCta || k > kMaxItemsPerCta) continue;
+        const double even = k / std::ceil(k);
+        const double tail = static_cast<double>(L % c) / static_cast<double>(c);
+        if (even > best_even + 1e-9 || (even > best_even - 1e-9 && tail < best_tail - 1e-9)) {
+            best_even = even;
+            best_tail = tail;
+            m_best = m;
+        }
+    }
+    if (m_best < 0) m_best = all_above ? std::max<int64_t>(m_floor, kMaxSplitTiles) : std::max<int64_t>(1, m_floor);
+    int64_t chunk = m_best * kTileQ;
+    if (d.bits_k == 16) {
+        // bf16 caches (one CTA per SM, 66 KB stages): about eight items per SM
+        // in 256..4096-token chunks measured best (remat leg's attention over
+        // 64 units of 16384 tokens: 1024-token chunks 0.156-0.161 ms, 1792
+        // 0.167 ms).
+        chunk = (units * L + 8 * kBalanceSms - 1) / (8 * kBalanceSms);
+        chunk = std::min<int64_t>(std::max<int64_t>((chunk + kTileQ - 1) / kTileQ * kTileQ, kTileQ), 4096);
+        chunk = std::max(chunk, m_floor * kTileQ);
+    }
     SplitBounds &sp = plan->splits;
     sp.n = 0;
     sp.b[0] = 0;
