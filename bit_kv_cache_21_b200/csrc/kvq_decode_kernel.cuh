@@ -417,8 +417,10 @@ struct WarpState : FoldedSums<GQA, VCH> {
     float mref[GQA];       // reference maximum per head (log2 units; warp-uniform)
     float thr[GQA];        // mref + slack: scores above it move the reference
     float l[GQA];          // this lane's tokens: sum of the weights p
-    float W[GQA][NVG];     //                     sum of p * s per value group
+    float W[GQA][NVG];     //                     sum of p * s per value group (one group)
     float Z[GQA][NVG];     //                     sum of p * z per value group
+    float Wv[GQA];         // several value groups: sum of p * s of this lane's group
+                           // over the token pairs its half-warp takes (value pass)
     float2 o[GQA][8];      // value accumulators: 8 channels x GQA heads, one
                            // token of a pair in each half (summed at the end)
 };
@@ -444,7 +446,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // (window tiles are bf16). GKC: compile-time key group size (0 = runtime
 // gk_rt); GVC likewise for the values (0 = runtime, NVG groups at most).
 template <int GQA, int KMT, int VMT, int KB, int VBITS, int TPW, int GKC, int GVC, int NVG, bool FULL,
-          bool SNK, bool VCH>
+          bool SNK, bool VCH, bool WV = false>
 __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *ks,
                                              const uint8_t *vc, const uint8_t *vs, int n, int start,
                                              const float *coef, int hstr, int cstr,
@@ -619,6 +621,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
                 st.l[g] *= alpha;
 #pragma unroll
                 for (int v = 0; v < NVG; ++v) { st.W[g][v] *= alpha; st.Z[g][v] *= alpha; }
+                if constexpr (WV) st.Wv[g] *= alpha;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) { st.o[g][c].x *= alpha; st.o[g][c].y *= alpha; }
                 if constexpr (VCH) {
@@ -668,7 +671,7 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
 #pragma unroll
                     for (int g = 0; g < GQA; ++g) {
                         w[m][g] = p[m][g] * szf.x;
-                        st.W[g][v] += w[m][g];
+                        if constexpr (!WV) st.W[g][v] += w[m][g];
                         st.Z[g][v] = fmaf(p[m][g], szf.y, st.Z[g][v]);
                     }
                 }
@@ -714,6 +717,12 @@ __device__ __forceinline__ void process_tile(const uint8_t *kc, const uint8_t *k
         } else {
             const uint2 u = lds64(wrow);
             w[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+        }
+        // WV (several value groups): the lanes of a group sum its weights here
+        // and the key side keeps Z only, which frees GQA x (NVG - 1) registers
+        if constexpr (VMT == V_TOKEN && WV) {
+#pragma unroll
+            for (int g = 0; g < GQA; ++g) st.Wv[g] += w[g].x + w[g].y;
         }
 #pragma unroll
         for (int g = 0; g < GQA; ++g)
@@ -906,6 +915,8 @@ decode_splitk_kernel(const DecodeParams p) {
     constexpr bool SINK = TL == kTailSink;
     constexpr bool WIN = TL == kTailWindow;
     constexpr int NVG = (VM != V_TOKEN) ? 1 : (GVC ? kHeadDim / GVC : kMaxGroups);
+    // weight sums of several value groups in the value pass (see process_tile)
+    constexpr bool WV = NVG > 1;
     constexpr int KBF = (KM == K_BF16) ? 16 : KBITS;  // key form of quantized tiles
     constexpr int TILE = (KM == K_BF16) ? kTileB : kTileQ;
     constexpr int TPW = TILE / kConsumerWarps;
@@ -1253,15 +1264,16 @@ decode_splitk_kernel(const DecodeParams p) {
     // the halves still sum.
     auto fold_values = [&]() {
         const int n_vg = GVC ? kHeadDim / GVC : kHeadDim / p.gv;
-        const int nv = 2 * GQA * n_vg;  // values per lane: W then Z, [g][v]
+        const int nw = WV ? 0 : GQA * n_vg;
+        const int nv = nw + GQA * n_vg;  // values per lane: W (one group) then Z, [g][v]
         const int rs = nv + 1;          // odd row stride: the lanes' rows hit distinct banks
 #pragma unroll
         for (int g = 0; g < GQA; ++g)
 #pragma unroll
             for (int v = 0; v < NVG; ++v)
                 if (v < n_vg) {
-                    wsm[lane * rs + g * n_vg + v] = st.W[g][v];
-                    wsm[lane * rs + GQA * n_vg + g * n_vg + v] = st.Z[g][v];
+                    if constexpr (!WV) wsm[lane * rs + g * n_vg + v] = st.W[g][v];
+                    wsm[lane * rs + nw + g * n_vg + v] = st.Z[g][v];
                 }
         __syncwarp();
         for (int col = lane; col < nv; col += 32) {
@@ -1278,8 +1290,15 @@ decode_splitk_kernel(const DecodeParams p) {
         const bool first_half = lane < 16;
 #pragma unroll
         for (int g = 0; g < GQA; ++g) {
-            const float Wg = first_half ? totals[g * n_vg + gv_lane] : 0.0f;
-            const float Zg = first_half ? totals[GQA * n_vg + g * n_vg + gv_lane] : 0.0f;
+            float Wg;
+            if constexpr (WV) {  // the two half-warps took the even and the odd pairs
+                const float ws = st.Wv[g] + __shfl_xor_sync(0xffffffffu, st.Wv[g], 16);
+                Wg = first_half ? ws : 0.0f;
+                st.Wv[g] = 0.0f;
+            } else {
+                Wg = first_half ? totals[g * n_vg + gv_lane] : 0.0f;
+            }
+            const float Zg = first_half ? totals[nw + g * n_vg + gv_lane] : 0.0f;
             float a[8], ch[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) a[c] = st.o[g][c].x + st.o[g][c].y;
@@ -1316,6 +1335,7 @@ decode_splitk_kernel(const DecodeParams p) {
                 st.l[g] = 0.0f;
 #pragma unroll
                 for (int v = 0; v < NVG; ++v) { st.W[g][v] = 0.0f; st.Z[g][v] = 0.0f; }
+                st.Wv[g] = 0.0f;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) st.o[g][c] = make_float2(0.0f, 0.0f);
                 if constexpr (VCH) {
@@ -1356,7 +1376,7 @@ decode_splitk_kernel(const DecodeParams p) {
             // one code path for full and partial tiles: the masks cost a few
             // instructions per tile, a second unrolled copy costs instruction
             // cache misses
-            process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, false, SINK>(
+            process_tile<GQA, KM, VM, KBF, VBITS, TPW, GKC_T, GVC, NVG, false, SINK, VM == V_CHANNEL, WV>(
                     sb, sb + p.off_ksz, sb + p.off_vc, vsz, hdr.n, SINK ? hdr.start : 0, coef, QHSTR,
                     RG::cstr, coef + GQA * QHSTR, p.gk, p.gv, st, wsm, warp, lane);
         } else if constexpr (KM != K_BF16 && TL != kTailNone) {
