@@ -36,7 +36,7 @@ template <bool PARTIAL, int NW>
 __global__ void __launch_bounds__(32 * NW) decode_merge_kernel(const float *o_part, const float2 *ml,
                                                            const int32_t *seq_lens, float *out,
                                                            float2 *out_ml, int Hq, int max_seq_len,
-                                                           const __grid_constant__ SplitBounds sp) {
+                                                           const SplitBounds sp) {
     __shared__ CombineSmemW<NW> sm;
     pdl_wait_prior_grid();
     const int hq = blockIdx.x, seq = blockIdx.y;
@@ -126,12 +126,8 @@ bool plan_decode(const kvq_cache_desc &d, int num_seqs, int num_q_heads, int max
         chunk = std::max(chunk, m_floor * kTileQ);
     }
     SplitBounds &sp = plan->splits;
-    sp.n = 0;
-    sp.b[0] = 0;
-    for (int64_t b = 0; b < L;) {
-        b += chunk;
-        sp.b[++sp.n] = static_cast<int>(std::min<int64_t>(b, INT32_MAX));
-    }
+    sp.chunk = static_cast<int>(chunk);
+    sp.n = static_cast<int>((L + chunk - 1) / chunk);
     plan->n_split = sp.n;
     const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * plan->n_split;
     plan->ws_part = rows * kHeadDim * sizeof(float);

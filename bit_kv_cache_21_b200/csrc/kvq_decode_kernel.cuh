@@ -1094,8 +1094,8 @@ decode_splitk_kernel(const DecodeParams p) {
             if (item < n_items) {
                 item_coords(spref, nsq, n_split, p.S, p.H, item, seq, kvh, split, lane);
                 const int T = lens[seq];
-                t_begin = p.sp.b[split];
-                t_end = min(T, p.sp.b[split + 1]);
+                t_begin = split_begin(p.sp, split);
+                t_end = min(T, split_begin(p.sp, split + 1));
                 Tq = quantized_len(T, p.R);
                 q_end = min(t_end, Tq);
                 // sink positions [0, sink_len) are read from the sink rows, in

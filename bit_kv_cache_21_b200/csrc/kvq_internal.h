@@ -20,24 +20,27 @@ kvq_status launch_append(const kvq_cache_desc &d, const void *k_new, const void 
                          kvq_dtype dtype, const int32_t *cu_new, int32_t *seq_lens,
                          int num_seqs, int total_new, cudaStream_t stream);
 
-// Token ranges of the splits, the same for every sequence: split j covers the
-// tokens [b[j], b[j+1]) below the sequence's length; b[0] = 0, and every
-// boundary is a multiple of the decode tiles. A sequence of length T has
-// n_T = #{j : b[j] < T} splits.
+// Token ranges of the splits, the same for every sequence: split j < n covers
+// the tokens [j * chunk, (j + 1) * chunk) below the sequence's length; chunk
+// is a multiple of the decode tiles. A sequence of length T has
+// ceil(T / chunk) splits (at most n).
 constexpr int kMaxDecodeSplits = 512;
 struct SplitBounds {
-    int n;
-    int b[kMaxDecodeSplits + 1];
+    int n;      // splits of the longest sequence
+    int chunk;  // tokens per split
 };
+
+// First token of split j (j <= n; clamped to the int range).
+__host__ __device__ inline int split_begin(const SplitBounds &sp, int j) {
+    const long long b = static_cast<long long>(j) * sp.chunk;
+    return b < 0x7fffffffLL ? static_cast<int>(b) : 0x7fffffff;
+}
 
 // Number of splits of a sequence of length T (0 for T <= 0).
 __host__ __device__ inline int splits_of(const SplitBounds &sp, int T) {
-    int lo = 0, hi = sp.n;  // first j in [0, n] with b[j] >= T
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (sp.b[mid] < T) lo = mid + 1; else hi = mid;
-    }
-    return lo;
+    if (T <= 0) return 0;
+    const int n = static_cast<int>((static_cast<long long>(T) + sp.chunk - 1) / sp.chunk);
+    return n < sp.n ? n : sp.n;
 }
 
 // Decode attention geometry chosen on the host from the sizes alone.
