@@ -1023,10 +1023,9 @@ decode_splitk_kernel(const DecodeParams p) {
 
     if (warp == kProducerWarp) {
         // ------------------------- producer -------------------------
-        // The first item is claimed before the prefix is built (the atomic's
-        // round trip overlaps the length loads), later ones one item ahead.
-        int next = 0;
-        if (lane == 0) next = atomicAdd(p.counter, 1);
+        // CTA b takes item b first (no atomic on the start-up path); later
+        // items come from the counter, offset by the grid, one item ahead.
+        int next = static_cast<int>(blockIdx.x);
         // Lengths (clamped) and split counts of the sequences; items per
         // split: H x the sequences with more than j splits; their prefix.
         const int n_split = p.sp.n;
@@ -1088,7 +1087,7 @@ decode_splitk_kernel(const DecodeParams p) {
         bool stop = false;
         for (int n_item = 0; !stop; ++n_item) {
             int item = __shfl_sync(0xffffffffu, next, 0);
-            if (lane == 0 && item < n_items) next = atomicAdd(p.counter, 1);
+            if (lane == 0 && item < n_items) next = atomicAdd(p.counter, 1) + static_cast<int>(gridDim.x);
             int seq = 0, kvh = 0, split = 0;
             int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0, n_sink = 0, n_st = 0;
             if (item < n_items) {
