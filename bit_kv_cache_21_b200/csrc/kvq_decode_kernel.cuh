@@ -948,6 +948,8 @@ decode_splitk_kernel(const DecodeParams p) {
     int *lens = spref + p.sp.n + 1;                                  // [S] clamped lengths
     int *nsq = lens + p.S;                                           // [S] splits of each sequence
 
+    // The producer's first length load is issued before the set-up barrier.
+    const int t_first = (warp == kProducerWarp && lane < p.S) ? __ldg(p.seq_lens + lane) : 0;
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
@@ -1026,13 +1028,15 @@ decode_splitk_kernel(const DecodeParams p) {
         // CTA b takes item b first (no atomic on the start-up path); later
         // items come from the counter, offset by the grid, one item ahead.
         int next = static_cast<int>(blockIdx.x);
-        // Lengths (clamped) and split counts of the sequences; items per
-        // split: H x the sequences with more than j splits; their prefix.
+        // Lengths (clamped) and split counts of the sequences. When every
+        // sequence has all n_split splits the items are regular (split
+        // item / units, unit item % units); otherwise items per split are
+        // H x the sequences with more than j splits, and their prefix gives
+        // the first item of each split.
         const int n_split = p.sp.n;
-        for (int j = lane; j <= n_split; j += 32) spref[j] = 0;  // histogram of split counts first
-        __syncwarp();
+        bool full_lane = true;
         for (int s = lane; s < p.S; s += 32) {
-            int T_s = __ldg(p.seq_lens + s);
+            int T_s = (s == lane) ? t_first : __ldg(p.seq_lens + s);
             if (T_s > p.max_seq_len) {
                 if (blockIdx.x == 0) status_or(p.status, KVQ_DEV_SEQLEN);
                 T_s = p.max_seq_len;
@@ -1040,44 +1044,52 @@ decode_splitk_kernel(const DecodeParams p) {
             lens[s] = T_s;
             const int ns = splits_of(p.sp, T_s);
             nsq[s] = ns;
-            atomicAdd(&spref[ns], 1);
+            full_lane = full_lane && ns == n_split;
         }
-        __syncwarp();
-        // G_j = #{s : n_s > j} (suffix sums of the histogram), from the top
-        int gsum = 0;
-        for (int base = ((n_split - 1) / 32) * 32; base >= 0; base -= 32) {
-            const int j = base + lane;
-            int v = (j < n_split) ? spref[j + 1] : 0;
+        const bool regular = __all_sync(0xffffffffu, full_lane);
+        const int units = p.S * p.H;
+        int n_items = n_split * units;
+        if (!regular) {
+            for (int j = lane; j <= n_split; j += 32) spref[j] = 0;  // histogram of split counts
+            __syncwarp();
+            for (int s = lane; s < p.S; s += 32) atomicAdd(&spref[nsq[s]], 1);
+            __syncwarp();
+            // G_j = #{s : n_s > j} (suffix sums of the histogram), from the top
+            int gsum = 0;
+            for (int base = ((n_split - 1) / 32) * 32; base >= 0; base -= 32) {
+                const int j = base + lane;
+                int v = (j < n_split) ? spref[j + 1] : 0;
 #pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const int o = __shfl_down_sync(0xffffffffu, v, m);
-                if (lane + m < 32) v += o;
+                for (int m = 1; m < 32; m <<= 1) {
+                    const int o = __shfl_down_sync(0xffffffffu, v, m);
+                    if (lane + m < 32) v += o;
+                }
+                const int G = v + gsum;
+                gsum += __shfl_sync(0xffffffffu, v, 0);
+                __syncwarp();
+                if (j < n_split) spref[j + 1] = G;  // G_j parked one slot up
+                __syncwarp();
             }
-            const int G = v + gsum;
-            gsum += __shfl_sync(0xffffffffu, v, 0);
-            __syncwarp();
-            if (j < n_split) spref[j + 1] = G;  // G_j parked one slot up
-            __syncwarp();
-        }
-        // exclusive prefix of H * G_j: spref[j] = first item of split j
-        int carry = 0;
-        for (int base = 0; base < n_split; base += 32) {
-            const int j = base + lane;
-            const int cnt = (j < n_split) ? p.H * spref[j + 1] : 0;
-            int incl = cnt;
+            // exclusive prefix of H * G_j: spref[j] = first item of split j
+            int carry = 0;
+            for (int base = 0; base < n_split; base += 32) {
+                const int j = base + lane;
+                const int cnt = (j < n_split) ? p.H * spref[j + 1] : 0;
+                int incl = cnt;
 #pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const int o = __shfl_up_sync(0xffffffffu, incl, m);
-                if (lane >= m) incl += o;
+                for (int m = 1; m < 32; m <<= 1) {
+                    const int o = __shfl_up_sync(0xffffffffu, incl, m);
+                    if (lane >= m) incl += o;
+                }
+                __syncwarp();
+                if (j < n_split) spref[j] = carry + incl - cnt;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+                __syncwarp();
             }
+            if (lane == 0) spref[n_split] = carry;
             __syncwarp();
-            if (j < n_split) spref[j] = carry + incl - cnt;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-            __syncwarp();
+            n_items = carry;
         }
-        if (lane == 0) spref[n_split] = carry;
-        __syncwarp();
-        const int n_items = carry;
 
         constexpr int KROW = RowGeo<KBF>::bytes;
         constexpr int VROW = (VM == V_BF16) ? kHeadDim * 2 : kHeadDim * VBITS / 8;
@@ -1091,7 +1103,14 @@ decode_splitk_kernel(const DecodeParams p) {
             int seq = 0, kvh = 0, split = 0;
             int t_begin = 0, t_end = 0, Tq = 0, q_end = 0, n_qt = 0, w_begin = 0, n_wt = 0, n_sink = 0, n_st = 0;
             if (item < n_items) {
-                item_coords(spref, nsq, n_split, p.S, p.H, item, seq, kvh, split, lane);
+                if (regular) {
+                    split = item / units;
+                    const int u = item - split * units;
+                    seq = u / p.H;
+                    kvh = u - seq * p.H;
+                } else {
+                    item_coords(spref, nsq, n_split, p.S, p.H, item, seq, kvh, split, lane);
+                }
                 const int T = lens[seq];
                 t_begin = split_begin(p.sp, split);
                 t_end = min(T, split_begin(p.sp, split + 1));
