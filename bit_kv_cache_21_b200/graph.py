@@ -17,7 +17,10 @@ class DecodeStep:
 
     k_host, v_host: pinned host [n_new][H][128] (bf16, fp16 or fp32), the
     step's new tokens in cu_new order; q_host: pinned host [S][Hq][128];
-    the caller refills them before every run. seq_lens, cu_new: device int32
+    the caller refills them before every run. When k_host, v_host and q_host
+    lie back to back in one pinned buffer (k, then v, then q, each a multiple
+    of 16 bytes), the step uploads them with one copy instead of three.
+    seq_lens, cu_new: device int32
     (seq_lens advances by the appended tokens on every run). The output lands
     in `out_host` (pinned fp32 [S][Hq][128]) once the stream is synchronized.
 
@@ -38,9 +41,25 @@ class DecodeStep:
         self.desc, self.seq_lens, self.cu_new = desc, seq_lens, cu_new
         self.max_seq_len, self.scale = max_seq_len, float(softmax_scale)
         self.k_host, self.v_host, self.q_host = k_host, v_host, q_host
-        self.dk = torch.empty(k_host.shape, dtype=k_host.dtype, device=dev)
-        self.dv = torch.empty(v_host.shape, dtype=v_host.dtype, device=dev)
-        self.dq = torch.empty(q_host.shape, dtype=q_host.dtype, device=dev)
+        parts = (k_host, v_host, q_host)
+        self.h_all = None
+        if (all(t.is_contiguous() for t in parts) and k_host.nbytes % 16 == 0 and v_host.nbytes % 16 == 0
+                and all(a.untyped_storage().data_ptr() == b.untyped_storage().data_ptr()
+                        and a.data_ptr() + a.nbytes == b.data_ptr() for a, b in zip(parts, parts[1:]))):
+            # one upload: the three as byte ranges of one host and one device buffer
+            total = sum(t.nbytes for t in parts)
+            base = k_host.storage_offset() * k_host.element_size()
+            self.h_all = torch.empty(0, dtype=torch.uint8).set_(k_host.untyped_storage(), base, (total,))
+            self.d_all = torch.empty(total, dtype=torch.uint8, device=dev)
+            views, off = [], 0
+            for t in parts:
+                views.append(self.d_all[off:off + t.nbytes].view(t.dtype).view(t.shape))
+                off += t.nbytes
+            self.dk, self.dv, self.dq = views
+        else:
+            self.dk = torch.empty(k_host.shape, dtype=k_host.dtype, device=dev)
+            self.dv = torch.empty(v_host.shape, dtype=v_host.dtype, device=dev)
+            self.dq = torch.empty(q_host.shape, dtype=q_host.dtype, device=dev)
         S, Hq = q_host.shape[0], q_host.shape[1]
         self.out = torch.empty((S, Hq, 128), dtype=torch.float32, device=dev)
         self.out_host = out_host if out_host is not None else torch.empty(
@@ -76,9 +95,12 @@ class DecodeStep:
         self.replays_left = left  # None: no sequence grows
 
     def _body(self):
-        self.dk.copy_(self.k_host, non_blocking=True)
-        self.dv.copy_(self.v_host, non_blocking=True)
-        self.dq.copy_(self.q_host, non_blocking=True)
+        if self.h_all is not None:
+            self.d_all.copy_(self.h_all, non_blocking=True)
+        else:
+            self.dk.copy_(self.k_host, non_blocking=True)
+            self.dv.copy_(self.v_host, non_blocking=True)
+            self.dq.copy_(self.q_host, non_blocking=True)
         B.quantize_append(self.desc, self.dk, self.dv, self.cu_new, self.seq_lens)
         B.decode_attention(self.desc, self.dq, self.seq_lens, self.max_seq_len, self.scale, out=self.out,
                            workspace=self.ws)

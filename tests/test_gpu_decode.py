@@ -208,9 +208,11 @@ def test_decode_randomized_hadamard(hb, gqa):
         assert_close(out[s_], oracle_decode_tokens(ks[s_], vs[s_], q[s_], spec, signs=signs), "seq %d" % s_)
 
 
-def test_decode_step_graph_replays_the_eager_step():
+@pytest.mark.parametrize("packed", [False, True])
+def test_decode_step_graph_replays_the_eager_step(packed):
     # the CUDA-graph step (uploads, append, decode, download) gives the eager
-    # calls' results bit for bit, step after step, and advances the lengths
+    # calls' results bit for bit, step after step, and advances the lengths;
+    # packed: k, v and q back to back in one pinned buffer, uploaded by one copy
     import workloads as W
     S, H, Hq, T0, steps = 3, 2, 8, 300, 4
     g = np.random.default_rng(77)
@@ -227,10 +229,18 @@ def test_decode_step_graph_replays_the_eager_step():
         caches.append(c)
         lens.append(sl)
     cu_one = torch.arange(0, S + 1, dtype=torch.int32, device="cuda")
-    hk = torch.empty((S, H, D), dtype=torch.bfloat16).pin_memory()
-    hv = torch.empty_like(hk).pin_memory()
-    hq = torch.empty((S, Hq, D), dtype=torch.bfloat16).pin_memory()
+    if packed:
+        buf = torch.empty(2 * (2 * S * H * D + S * Hq * D), dtype=torch.uint8).pin_memory()
+        n_kv = 2 * S * H * D
+        hk = buf[:n_kv].view(torch.bfloat16).view(S, H, D)
+        hv = buf[n_kv:2 * n_kv].view(torch.bfloat16).view(S, H, D)
+        hq = buf[2 * n_kv:].view(torch.bfloat16).view(S, Hq, D)
+    else:
+        hk = torch.empty((S, H, D), dtype=torch.bfloat16).pin_memory()
+        hv = torch.empty_like(hk).pin_memory()
+        hq = torch.empty((S, Hq, D), dtype=torch.bfloat16).pin_memory()
     step = K.DecodeStep(caches[1].desc, lens[1], cu_one, 384, SCALE, hk, hv, hq)
+    assert (step.h_all is not None) == packed
     for i in range(steps):
         kk = torch.from_numpy(hist_k[:, T0 + i]).to(torch.bfloat16)
         vv = torch.from_numpy(hist_v[:, T0 + i]).to(torch.bfloat16)
