@@ -12,12 +12,12 @@
 // the keys' orthogonal transform, so q~ . k~ = q . k.
 //
 // Work items are (sequence, KV head, split): a split is a token range, the
-// same for every sequence (the host's plan). Items are numbered split-major,
-// so the sequences' last, partial splits are claimed last and fill the
-// launch's tail. The kernel is
-// persistent: each CTA (4 consumer warps, 1 producer warp, 1 helper warp)
-// runs until a global item counter is exhausted. The producer warp claims
-// items and streams every item's tiles (K codes, K scale/zero, V codes, V
+// same for every sequence (the host's plan: equal chunks of whole tiles).
+// Items are numbered split-major, so the sequences' last, partial splits are
+// claimed last and fill the launch's tail. The kernel is persistent: each CTA
+// (4 consumer warps, 1 producer warp, 1 helper warp) takes item blockIdx.x
+// first and then claims items from a global counter until none are left. The
+// producer warp claims items and streams every item's tiles (K codes, K scale/zero, V codes, V
 // scale/zero; bf16 rows for the recent-token window) into a shared-memory ring
 // with 1-D bulk copies (TMA engine, mbarrier complete_tx); its lanes issue the
 // copies of a tile in parallel, one page per lane for paged caches. Each stage
