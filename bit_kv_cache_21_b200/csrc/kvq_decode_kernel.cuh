@@ -1096,6 +1096,7 @@ decode_splitk_kernel(const DecodeParams p) {
         const int ngk = (KM == K_TOKEN) ? kHeadDim / p.gk : 0;
         const int ngv = (VM == V_TOKEN) ? kHeadDim / p.gv : 0;
         int it = 0;  // tile counter of this CTA (stage it % NS, round it / NS)
+        int ps = 0, pr = 0;  // it % NS and it / NS, carried
         bool stop = false;
         for (int n_item = 0; !stop; ++n_item) {
             int item = __shfl_sync(0xffffffffu, next, 0);
@@ -1140,8 +1141,8 @@ decode_splitk_kernel(const DecodeParams p) {
             }
             const int n_tiles = (item < n_items) ? n_qt + n_wt + n_st : 1;  // 1 = the done marker
             const int64_t sh = static_cast<int64_t>(seq) * p.H + kvh;
-            for (int ti = 0; ti < n_tiles; ++ti, ++it) {
-                const int s = it % NS, r = it / NS;
+            for (int ti = 0; ti < n_tiles; ++ti, ++it, (++ps == NS) ? (ps = 0, ++pr) : 0) {
+                const int s = ps, r = pr;
                 int ok = 1;
                 if (lane == 0 && r > 0)
                     ok = mbar_wait_bounded(&empty[s], (r - 1) & 1, p.timeout_ns, p.status, abort_flag);
@@ -1331,9 +1332,9 @@ decode_splitk_kernel(const DecodeParams p) {
     };
 
     int kc_tiles = 0;  // quantized tiles seen (parity of the per-channel coefficient sets)
-    for (int it = 0;; ++it) {
-        const int s = it % NS, r = it / NS;
-        if (!mbar_wait_bounded(&full[s], r & 1, p.timeout_ns, p.status, abort_flag)) break;
+    // stage s of the ring and the parity of its round, carried from tile to tile
+    for (int s = 0, ph = 0;; (++s == NS) ? (s = 0, ph ^= 1) : 0) {
+        if (!mbar_wait_bounded(&full[s], ph, p.timeout_ns, p.status, abort_flag)) break;
         const uint8_t *sb = stages + static_cast<size_t>(s) * p.stage_bytes;
         const TileHdr hdr = *reinterpret_cast<const TileHdr *>(sb + p.off_hdr);
         if (hdr.flags & kDone) break;
