@@ -168,6 +168,8 @@ kvq_status launch_decode_splitk(const kvq_cache_desc &d, const DecodePlan &plan,
     p.hscale = hadamard_scale(d.hadamard_block_k);
     p.qscale = softmax_scale * kLog2e;
     p.R = d.residual_len;
+    p.r_shift = 0;
+    while (p.R > 0 && (1 << p.r_shift) < p.R) ++p.r_shift;  // R is a power of two (validated)
     p.paged = d.paged;
     p.page_size = d.page_size;
     p.max_pages = d.max_pages_per_seq;

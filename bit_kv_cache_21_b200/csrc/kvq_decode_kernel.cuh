@@ -124,6 +124,7 @@ struct DecodeParams {
     float hscale;   // fp32(1/sqrt(hb))
     float qscale;   // softmax_scale * log2(e)
     int R;
+    int r_shift;    // log2(R) (R is 64, 128 or 256 when non-zero)
     int paged, page_size, max_pages, num_pages, cap;
     int n_split, max_seq_len;  // partials per query head; longest sequence attended
     SplitBounds sp;            // token ranges of the splits
@@ -1208,7 +1209,7 @@ decode_splitk_kernel(const DecodeParams p) {
                         bulk_g2s(st + p.off_ksz, p.k_sz + row * ngk, b, bar);
                     } else if (lane == 2 && KM == K_CHANNEL) {
                         // the channel scales of every block the tile touches
-                        const int b0 = t0 / p.R, nb = (t0 + n - 1) / p.R - b0 + 1;
+                        const int b0 = t0 >> p.r_shift, nb = ((t0 + n - 1) >> p.r_shift) - b0 + 1;
                         mbar_expect_tx(bar, nb * kHeadDim * 4);
                         bulk_g2s(st + p.off_ksz, p.k_sz + (sh * (p.cap / p.R) + b0) * kHeadDim,
                                  nb * kHeadDim * 4, bar);
@@ -1217,7 +1218,7 @@ decode_splitk_kernel(const DecodeParams p) {
                         mbar_expect_tx(bar, b);
                         bulk_g2s(st + p.off_vsz, p.v_sz + row * ngv, b, bar);
                     } else if (lane == 3 && VM == V_CHANNEL) {
-                        const int b0 = t0 / p.R, nb = (t0 + n - 1) / p.R - b0 + 1;
+                        const int b0 = t0 >> p.r_shift, nb = ((t0 + n - 1) >> p.r_shift) - b0 + 1;
                         mbar_expect_tx(bar, nb * kHeadDim * 4);
                         bulk_g2s(st + p.off_vsz, p.v_sz + (sh * (p.cap / p.R) + b0) * kHeadDim,
                                  nb * kHeadDim * 4, bar);
@@ -1372,9 +1373,9 @@ decode_splitk_kernel(const DecodeParams p) {
                 // coefficients: the warps share the (block, head) builds into
                 // the sets of this tile's parity (no warp still reads them:
                 // all passed the previous tile's barrier), then wait for all.
-                const int nbt = TILE / p.R;  // block sets per tile
+                const int nbt = TILE >> p.r_shift;  // block sets per tile
                 float *sets = csets + (kc_tiles & 1) * nbt * CBUF;
-                const int nb = (hdr.n + p.R - 1) / p.R;
+                const int nb = (hdr.n + p.R - 1) >> p.r_shift;
                 for (int idx = warp; idx < nb * GQA; idx += kConsumerWarps) {
                     const int b = idx / GQA, g = idx - b * GQA;
                     const float4 xv = ldsf4(qs + g * kHeadDim + 4 * lane);
@@ -1385,13 +1386,13 @@ decode_splitk_kernel(const DecodeParams p) {
                 }
                 named_sync(2, kConsumers);
                 ++kc_tiles;
-                coef = sets + min((warp * TPW) / p.R, nbt - 1) * CBUF;
+                coef = sets + min((warp * TPW) >> p.r_shift, nbt - 1) * CBUF;
             }
             constexpr int GKC_T = (KM == K_TOKEN) ? GKC : kHeadDim;
             // per-channel values: this warp's block among the tile's staged ones
             const uint8_t *vsz = sb + p.off_vsz;
             if constexpr (VM == V_CHANNEL)
-                vsz += ((hdr.t0 + warp * TPW) / p.R - hdr.t0 / p.R) * kHeadDim * 4;
+                vsz += (((hdr.t0 + warp * TPW) >> p.r_shift) - (hdr.t0 >> p.r_shift)) * kHeadDim * 4;
             // one code path for full and partial tiles: the masks cost a few
             // instructions per tile, a second unrolled copy costs instruction
             // cache misses
